@@ -1,0 +1,290 @@
+"""Pins of the oracle's quantizer, scale strategies, dequantizer, MSE and FOCUS.
+
+Pages: "Finer is Better (with the Right Scaling)" (手法 1-2: E2M1 data, E4M3
+scales, block sizes 4/8/16/32, abs-max / prevent-zero / 4-over-6 / brute force
+/ hierarchical scaling; 主要な発見と結果: prevent-zero removes the underflow
+spike, 4-over-6 lowers MSE, brute force improves strictly with finer blocks);
+"Bridging the Gap Between Promise and Performance for Microscaling FP4
+Quantization" (技術概要 §1: MXFP4 E8M0 scales; §2.1: rotation helps MXFP4
+under RTN); "FOCUS: FP4 Optimization via Coupled-Relaxation and
+Dual-Granularity Scaling" (Metodologia §1-§4).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from microscaling_fp4_quantization_bf16_b200 import synth
+
+E2M1 = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6, -0.0, -0.5, -1, -1.5, -2, -3, -4, -6], np.float64)
+
+
+def bf16_bits(a):
+    return synth.bits16(synth.to_bf16(np.asarray(a, np.float64)))
+
+
+def f32_of_bf16(bits):
+    return (bits.astype(np.uint32) << 16).view(np.float32)
+
+
+def e4m3_table(ref):
+    return np.array([ref.e4m3_value(c) for c in range(0x7F)], np.float64)
+
+
+# --------------------------------------------------------------- hand examples
+
+def test_packing_and_scale_hand_example(ref):
+    # s_g = 2688 / 2688 = 1; block max 6 -> raw = 6 / (6 * 1) = 1 -> E4M3 code 0x38,
+    # S = 1, r = 1; element codes are then the E2M1 codes of the values themselves.
+    y = [0.5, 1, 1.5, 2, 3, 4, 6, 0, -0.5, -1, -1.5, -2, -3, -4, -6, -0.0]
+    x = bf16_bits([y])
+    out = ref.quantize(x, "nvfp4", 16, "absmax", 0, global_amax=2688.0, dq="f32")
+    assert out["global_scale"] == 1.0
+    assert out["scales"].tolist() == [[0x38]]
+    # element 2j -> low nibble, 2j+1 -> high nibble
+    assert out["codes"].tolist() == [[0x21, 0x43, 0x65, 0x07, 0xA9, 0xCB, 0xED, 0x8F]]
+    assert out["mse"].tolist() == [[0.0]]
+    assert np.array_equal(out["dq"].view(np.uint32), np.array([y], np.float32).view(np.uint32))
+
+
+def test_mxfp4_hand_example(ref):
+    # block max 5.0 -> floor(log2 5) - 2 = 0 -> byte 127, S = 1; 5 -> tie 4/6 -> 4
+    y = [5.0, -0.25, 0.75, 2.5] + [0.0] * 28
+    out = ref.quantize(bf16_bits([y]), "mxfp4", 32, "absmax", 0, dq="f32")
+    assert out["scales"].tolist() == [[127]]
+    codes = ref.unpack_codes(out["codes"])[0]
+    assert codes[:4].tolist() == [6, 8, 2, 4]  # 4, -0, 1, 2
+    assert out["dq"][0, :4].tolist() == [4.0, -0.0, 1.0, 2.0]
+    sse = (5 - 4) ** 2 + 0.25 ** 2 + 0.25 ** 2 + 0.5 ** 2
+    assert out["mse"][0, 0] == np.float32(sse / 32)
+
+
+# ------------------------------------------------------------------ round trips
+
+@pytest.mark.parametrize("block", [4, 8, 16, 32])
+@pytest.mark.parametrize("strategy", ["absmax", "prevent_zero", "four_over_six", "brute_force"])
+def test_nvfp4_exact_round_trip(ref, block, strategy):
+    rng = np.random.default_rng(block)
+    rows, cols = 8, 64
+    nb = cols // block
+    c = rng.integers(1, 0x7F, size=(rows, nb))
+    q = rng.integers(0, 16, size=(rows, cols))
+    # force one element of every block to +-6 so the block abs-max is 6 * e4m3(c)
+    q.reshape(rows, nb, block)[:, :, 0] = rng.choice([7, 15], size=(rows, nb))
+    S = e4m3_table(ref)[c]
+    y = E2M1[q] * np.repeat(S, block, axis=1)
+    x = bf16_bits(y)
+    assert np.array_equal(f32_of_bf16(x).astype(np.float64), y)  # exactly representable
+    out = ref.quantize(x, "nvfp4", block, strategy, 0, global_amax=2688.0, dq="f32")
+    assert np.array_equal(out["scales"], c.astype(np.uint8))
+    assert np.array_equal(ref.unpack_codes(out["codes"]), q.astype(np.uint8))
+    assert np.array_equal(out["dq"].astype(np.float64), y)
+    assert np.all(out["mse"] == 0)
+
+
+def test_mxfp4_exact_round_trip(ref):
+    rng = np.random.default_rng(7)
+    rows, cols = 16, 128
+    e = rng.integers(-120, 120, size=(rows, cols // 32))
+    q = rng.integers(0, 16, size=(rows, cols))
+    q.reshape(rows, -1, 32)[:, :, 0] = rng.choice([6, 7, 14, 15], size=e.shape)  # max |val| in {4, 6}
+    y = E2M1[q] * np.repeat(2.0 ** e, 32, axis=1)
+    x = bf16_bits(y)
+    out = ref.quantize(x, "mxfp4", 32, "absmax", 0, dq="f32")
+    assert np.array_equal(out["scales"].astype(np.int64), e + 127)
+    assert np.array_equal(ref.unpack_codes(out["codes"]), q.astype(np.uint8))
+    assert np.array_equal(out["dq"].astype(np.float64), y)
+
+
+# -------------------------------------------------------------- scales & zeros
+
+def test_global_scale_closed_form(ref):
+    x = synth.workload("c1_nvfp4_roundtrip", rows=64, cols=256)["x"]
+    xb = synth.bits16(x)
+    amax = np.abs(x.float().numpy()).max()  # library max over the widened tensor
+    assert ref.global_amax(xb, 0) == amax
+    out = ref.quantize(xb, "nvfp4", 16, "absmax", 0)
+    assert out["global_scale"] == np.float32(amax) / np.float32(2688.0)
+    assert ref.global_scale(0.0) == 1.0 and ref.global_scale(-1.0) == 1.0
+    assert ref.global_scale(float("inf")) == 1.0 and ref.global_scale(float("nan")) == 1.0
+
+
+def test_zero_tensor(ref):
+    x = np.zeros((4, 64), np.uint16)
+    nv = ref.quantize(x, "nvfp4", 16, "absmax", 0, dq="f32")
+    assert nv["global_scale"] == 1.0
+    assert np.all(nv["scales"] == 0) and np.all(nv["codes"] == 0) and np.all(nv["mse"] == 0)
+    assert np.all(nv["dq"].view(np.uint32) == 0)
+    pz = ref.quantize(x, "nvfp4", 16, "prevent_zero", 0)
+    assert np.all(pz["scales"] == 1) and np.all(pz["codes"] == 0)
+    mx = ref.quantize(x, "mxfp4", 32, "absmax", 0)
+    assert np.all(mx["scales"] == 0) and np.all(mx["codes"] == 0)
+
+
+def test_mxfp4_scale_bytes_from_frexp(ref):
+    x = synth.workload("c2_mxfp4_laplace_outliers", rows=32, cols=512)["x"]
+    xb = synth.bits16(x)
+    for rot in (0, 32, 128):
+        y = f32_of_bf16(xb)
+        if rot:
+            y = ref.fwht(y.reshape(-1, rot), rot).reshape(y.shape)
+        amax = np.abs(y.reshape(32, -1, 32)).max(axis=2)
+        want = np.array([[max(-127, min(127, math.frexp(float(a))[1] - 1 - 2)) + 127 if a > 0
+                          else 0 for a in row] for row in amax])
+        out = ref.quantize(xb, "mxfp4", 32, "absmax", rot)
+        assert np.array_equal(out["scales"].astype(np.int64), want)
+
+
+# ------------------------------------------------------------------ strategies
+
+def _with_tiny_rows(x: torch.Tensor) -> torch.Tensor:
+    a = x.float().numpy().copy()
+    a[::4] *= 1e-6  # blocks far below the tensor abs-max: their E4M3 scale underflows
+    return synth.to_bf16(a)
+
+
+@pytest.mark.parametrize("block", [4, 8, 16, 32])
+def test_strategy_relations_exact(ref, block):
+    x = _with_tiny_rows(synth.workload("c3_strategy_sweep_t3", rows=32, cols=256)["x"])
+    xb = synth.bits16(x)
+    res = {s: ref.quantize(xb, "nvfp4", block, s, 0, dq="f32")
+           for s in ("absmax", "prevent_zero", "four_over_six", "brute_force")}
+    am, pz, fs, bf = (res[s] for s in ("absmax", "prevent_zero", "four_over_six", "brute_force"))
+    sg = am["global_scale"]
+    assert all(r["global_scale"] == sg for r in res.values())
+    # prevent-zero never stores scale 0 and equals abs-max whenever abs-max's code >= 1
+    assert np.all(pz["scales"] >= 1)
+    same = am["scales"] >= 1
+    assert np.any(~same), "the data must exercise the underflow regime"
+    assert np.array_equal(pz["scales"][same], am["scales"][same])
+    assert np.array_equal(pz["mse"][same], am["mse"][same])
+    # ...and removes the underflow-to-zero error spike: never worse, element by element
+    assert np.all(pz["mse"][~same] <= am["mse"][~same])
+    assert np.mean(pz["mse"][~same]) < np.mean(am["mse"][~same])
+    # 4-over-6: never worse than abs-max (its target-6 candidate IS abs-max)
+    assert np.all(fs["mse"] <= am["mse"])
+    moved = fs["scales"] != am["scales"]
+    assert np.any(moved)
+    assert np.all(fs["mse"][moved] < am["mse"][moved])  # target 4 only on a strict gain
+    # brute force: the minimum over every positive code, so never worse than any
+    # strategy that stores a positive code
+    pos = fs["scales"] >= 1
+    assert np.all(bf["mse"] <= pz["mse"]) and np.all(bf["mse"][pos] <= fs["mse"][pos])
+    assert np.all(bf["scales"] >= 1)
+    # dequantize / block_mse reproduce quantize's own outputs bit for bit
+    for r in res.values():
+        dq = ref.dequantize(r["codes"], r["scales"], sg, *xb.shape, "nvfp4", block, "f32")
+        assert np.array_equal(dq.view(np.uint32), r["dq"].view(np.uint32))
+        m = ref.block_mse(xb, r["codes"], r["scales"], sg, "nvfp4", block, 0)
+        assert np.array_equal(m.view(np.uint32), r["mse"].view(np.uint32))
+        # the MSE is the mean squared error, checked in float64
+        err = (f32_of_bf16(xb).astype(np.float64) - r["dq"]) ** 2
+        want = err.reshape(err.shape[0], -1, block).mean(axis=2)
+        assert np.allclose(r["mse"], want, rtol=1e-5, atol=1e-45)
+
+
+def _nearest_e2m1_double(u):
+    mags = np.abs(E2M1[:8])
+    a = np.minimum(np.abs(u), 6.0)
+    idx = np.argmin(np.abs(a[..., None] - mags), axis=-1)
+    return np.sign(u) * mags[idx]
+
+
+def test_brute_force_is_minimum_in_double(ref):
+    rng = np.random.default_rng(21)
+    tab = e4m3_table(ref)
+    for block in (4, 8):
+        x = bf16_bits(rng.standard_t(3, size=(4, 8 * block)) * 0.02)
+        out = ref.quantize(x, "nvfp4", block, "brute_force", 0)
+        sg = float(out["global_scale"])
+        y = f32_of_bf16(x).astype(np.float64).reshape(-1, block)
+        S = tab[1:0x7F][:, None, None] * sg  # [126, 1, 1]
+        sse = ((y[None] - _nearest_e2m1_double(y[None] / S) * S) ** 2).sum(axis=2)  # [126, nblk]
+        best = sse.min(axis=0)
+        chosen = sse[out["scales"].reshape(-1).astype(np.int64) - 1, np.arange(y.shape[0])]
+        assert np.all(chosen <= best * (1 + 1e-5) + 1e-30)
+
+
+def test_finer_is_better_exact_and_statistical(ref):
+    x = synth.workload("c1_nvfp4_roundtrip", rows=64, cols=512)["x"]  # Gaussian data
+    xb = synth.bits16(x)
+    sse, means = {}, {}
+    for B in (4, 8, 16, 32):
+        o = ref.quantize(xb, "nvfp4", B, "brute_force", 0)
+        sse[B] = o["mse"].astype(np.float32) * np.float32(B)  # exact: B is a power of two
+        means[B] = float(np.mean(o["mse"]))
+    for B in (4, 8, 16):
+        l, r = sse[B][:, 0::2], sse[B][:, 1::2]
+        assert np.all((l + r).astype(np.float32) <= sse[2 * B])
+    assert means[4] < means[8] < means[16] < means[32]
+
+
+def test_hadamard_helps_mxfp4_on_laplace_outliers(ref):
+    x = synth.bits16(synth.workload("c2_mxfp4_laplace_outliers", rows=256, cols=1024)["x"])
+    m0 = ref.quantize(x, "mxfp4", 32, "absmax", 0)["mse"].mean()
+    m32 = ref.quantize(x, "mxfp4", 32, "absmax", 32)["mse"].mean()
+    assert m32 < m0
+
+
+# ----------------------------------------------------------------------- FOCUS
+
+@pytest.mark.parametrize("fmt,block", [("nvfp4", 16), ("mxfp4", 32)])
+def test_focus_unit_coefficients_equal_absmax_round_trip(ref, fmt, block):
+    d = synth.workload("c4_focus", rows=32, cols=256)
+    w = synth.bits16(d["w"])
+    ones = synth.bits16(torch.ones(32, 256 // 8, dtype=torch.float16))
+    f = ref.focus_fwd(w, ones, fmt, block, 8, out="f32")
+    q = ref.quantize(w, fmt, block, "absmax", 0, dq="f32")
+    assert np.array_equal(f["w_hat"].view(np.uint32), q["dq"].view(np.uint32))
+    assert np.array_equal(f["codes"], q["codes"]) and np.array_equal(f["scales"], q["scales"])
+    fb = ref.focus_fwd(w, ones, fmt, block, 8, out="bf16")
+    qb = ref.quantize(w, fmt, block, "absmax", 0, dq="bf16")
+    assert np.array_equal(fb["w_hat"], qb["dq"])
+
+
+def test_focus_hand_example(ref):
+    # s_g = 1 (amax 2688 supplied); block max 6 -> S_dq = 1. Sub-block 0 has c = 1,
+    # sub-block 1 has c = 2: u = W * (1 / 2), so 6 -> 3 and 3 -> 1.5, dequantized
+    # with S_dq = 1 (the coefficient is not stored).
+    w = [6, 3, 0, 0, 0, 0, 0, 0, 6, 3, 1, 0, 0, 0, 0, 0]
+    c = synth.bits16(torch.tensor([[1.0, 2.0]], dtype=torch.float16))
+    f = ref.focus_fwd(bf16_bits([w]), c, "nvfp4", 16, 8, global_amax=2688.0, out="f32")
+    assert f["scales"].tolist() == [[0x38]]
+    assert f["w_hat"][0].tolist() == [6, 3, 0, 0, 0, 0, 0, 0, 3, 1.5, 0.5, 0, 0, 0, 0, 0]
+
+
+def test_focus_coefficients_are_local_and_monotone(ref):
+    d = synth.workload("c4_focus", rows=16, cols=128)
+    w = synth.bits16(d["w"])
+    c = d["c"].clone()
+    base = ref.focus_fwd(w, synth.bits16(c), "nvfp4", 16, 8, out="f32")
+    c2 = c.clone()
+    c2[3, 5] = 1.5  # sub-block 5 of row 3: elements 40..47
+    pert = ref.focus_fwd(w, synth.bits16(c2), "nvfp4", 16, 8, out="f32")
+    diff = base["w_hat"] != pert["w_hat"]
+    assert diff[3, 40:48].any() and diff.sum() == diff[3, 40:48].sum()
+    assert np.array_equal(base["scales"], pert["scales"])  # S_dq does not depend on c
+    # a larger c shrinks u = W / (S_dq c), so code magnitudes can only fall
+    mag = lambda o: ref.unpack_codes(o["codes"]) & 7
+    big = ref.focus_fwd(w, synth.bits16(c * 1.25), "nvfp4", 16, 8, out="f32")
+    assert np.all(mag(big) <= mag(base)) and np.any(mag(big) < mag(base))
+
+
+@pytest.mark.parametrize("sub", [4, 8, 16])
+def test_focus_bwd_closed_form_and_ste(ref, sub):
+    d = synth.workload("c4_focus", rows=16, cols=256)
+    w, g = synth.bits16(d["w"]), synth.bits16(d["g"])
+    c = synth.focus_coeffs(16, 256, sub, seed=9)
+    dc = ref.focus_bwd(w, g, synth.bits16(c), sub)
+    W = f32_of_bf16(w).astype(np.float64).reshape(16, -1, sub)
+    G = f32_of_bf16(g).astype(np.float64).reshape(16, -1, sub)
+    C = c.float().numpy().astype(np.float64)
+    want = -(G * W).sum(axis=2) / C ** 2
+    scale = np.maximum(np.abs(want), np.abs(G * W).sum(axis=2) / C ** 2)
+    assert np.all(np.abs(dc - want) <= 1e-5 * scale)
+    # straight-through surrogate: W_hat ~ W / c, L = sum g * W_hat; central differences
+    h = 1e-6
+    L = lambda cc: (G * W / cc[..., None]).sum(axis=2)
+    fd = (L(C + h) - L(C - h)) / (2 * h)
+    assert np.allclose(dc, fd, rtol=1e-4, atol=1e-6 * np.abs(fd).max())
