@@ -1,0 +1,486 @@
+#!/usr/bin/env python
+"""Throughput of the block-scaled FP4 quantization hot path on B200.
+
+Headline workload: MXFP4 (E8M0 scales, block 32) quantization of a
+4096 x 4096 bf16 weight drawn from Laplace(0, 0.02) with 0.1% of entries
+times 50, run without rotation and with a 32-wide blockwise Hadamard; one step
+= both runs. Inputs are resident in HBM; L2 is flushed (a 2 x L2 write)
+before every launch, outside the timed events. ``value`` is quantized
+elements per second over the whole job (all ranks: independent replicas,
+weak scaling). One JSON line is printed by rank 0.
+
+``--impl reference`` times the oracle (plain C, host cores) on a bounded
+sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("quantized elements/s and achieved HBM GB/s (% of B200 roofline) per "
+          "format/strategy")
+WORKLOAD = "c2_mxfp4_laplace_outliers"
+ROWS, COLS = 4096, 4096
+ROTS = (0, 32)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+SM_COUNT_NOMINAL, FP32_LANES_PER_SM, SM_MAX_MHZ_NOMINAL = 148, 128, 1965.0
+
+
+def bytes_per_elem(block: int, codes=True, scales=True, mse=False, dq=0, extra_in=0.0):
+    """Algorithmic bytes per element: one bf16 read plus every output written."""
+    b = 2.0 + extra_in
+    if codes:
+        b += 0.5
+    if scales:
+        b += 1.0 / block
+    if mse:
+        b += 4.0 / block
+    b += dq
+    return b
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "microscaling_fp4_quantization_bf16_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """dram bytes per launch from a committed ncu summary, if the kernels
+    have not changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p))
+    e = d.get(kernel)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons with NVML in a thread."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples = []
+        self.ok = False
+        self.period = period_s
+        self._stop = threading.Event()
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # NVML missing: report that instead of clocks
+            self.err = repr(e)
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                rs = get(self.h)
+                self.samples.append((time.perf_counter(), mhz, rs))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self, t0: float, t1: float):
+        if not self.ok:
+            return {"error": getattr(self, "err", "nvml unavailable")}
+        inside = [s for s in self.samples if t0 <= s[0] <= t1]
+        window = "timed region"
+        if len(inside) < 3:
+            inside = self.samples
+            window = "soak + warm-up + timed region (timed region too short to sample)"
+        mhz = [s[1] for s in inside]
+        mask = 0
+        for s in inside:
+            mask |= s[2]
+        reasons = [n for b, n in self.REASONS.items() if mask & b and n != "gpu_idle"]
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(inside), "window": window}
+
+
+# ---------------------------------------------------------------- our arm
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import microscaling_fp4_quantization_bf16_b200 as fp4q
+    from microscaling_fp4_quantization_bf16_b200 import synth
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=dev)
+    fp4q.load()
+    peaks = load_peaks()
+    props = torch.cuda.get_device_properties(dev)
+    flush = torch.empty(2 * props.L2_cache_size // 4, dtype=torch.float32, device=dev)
+
+    x = synth.workload(WORKLOAD)["x"].to(dev)
+    n = x.numel()
+    outs = {r: fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
+                              torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
+                              None, None, None) for r in ROTS}
+    evs = {r: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for r in ROTS}
+
+    def step(times):
+        for r in ROTS:
+            flush.zero_()  # keeps the GPU busy while the launch is enqueued
+            s, e = evs[r]
+            s.record()
+            fp4q.quantize(x, "mxfp4", 32, "absmax", r, out=outs[r])
+            e.record()
+        torch.cuda.synchronize()
+        for r in ROTS:
+            times[r].append(evs[r][0].elapsed_time(evs[r][1]))
+
+    sampler = ClockSampler(local_rank)
+    with sampler:
+        soak_end = time.perf_counter() + args.soak
+        scratch = {r: [] for r in ROTS}
+        while time.perf_counter() < soak_end:
+            step(scratch)
+        for _ in range(args.warmup):
+            step(scratch)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        times = {r: [] for r in ROTS}
+        for _ in range(args.steps):
+            step(times)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        t1 = time.perf_counter()
+    clocks = sampler.summary(t0, t1)
+
+    total_ms = sum(sum(v) for v in times.values())
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    elems = n * len(ROTS) * args.steps * world
+    value = elems / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    # roofline of the dominant kernel (the launch with the larger mean time)
+    mean = {r: statistics.mean(times[r]) for r in ROTS}
+    dom = max(ROTS, key=lambda r: mean[r])
+    alg_bytes = bytes_per_elem(32) * n
+    achieved = alg_bytes / (mean[dom] / 1e3) / 1e9
+    kname = f"quant_kernel<32,{dom},mx>"
+    traffic = recorded_traffic(kname)
+    roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "algorithmic_bytes_per_launch": int(alg_bytes),
+                "peak_source": peaks["source"] + " (copy bandwidth, burst)",
+                "per_launch_us": {f"rot{r}": round(mean[r] * 1e3, 2) for r in ROTS}}
+
+    # end to end through the public API: pinned host input -> device -> both
+    # runs -> codes and scales back to pinned host memory, every step
+    xh = synth.workload(WORKLOAD)["x"].pin_memory()
+    xd = torch.empty_like(x)
+    ch = {r: torch.empty(ROWS, COLS // 2, dtype=torch.uint8).pin_memory() for r in ROTS}
+    sh = {r: torch.empty(ROWS, COLS // 32, dtype=torch.uint8).pin_memory() for r in ROTS}
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        for r in ROTS:
+            fp4q.quantize(xd, "mxfp4", 32, "absmax", r, out=outs[r])
+            ch[r].copy_(outs[r].codes, non_blocking=True)
+            sh[r].copy_(outs[r].scales, non_blocking=True)
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        e2e_step()
+    if world > 1:
+        dist.barrier()
+    te0 = time.perf_counter()
+    for _ in range(args.steps):
+        e2e_step()
+    te = time.perf_counter() - te0
+    if world > 1:
+        t = torch.tensor([te], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        te = float(t.item())
+    h2d = xh.numel() * xh.element_size()
+    d2h = sum(ch[r].numel() + sh[r].numel() for r in ROTS)
+    e2e = {"value": elems / te, "unit": "elements/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": round(te / args.steps * 1e3, 4),
+           "path": "pinned host bf16 -> cudaMemcpyAsync -> fp4q_quantize x2 -> codes+scales "
+                   "to pinned host, synchronised every step (wall clock)"}
+
+    line = {"metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic",
+            "config": {"workload": f"{WORKLOAD}: MXFP4 E8M0 block 32 on a {ROWS}x{COLS} bf16 "
+                                   "Laplace(0,0.02) weight with 0.1% entries x50; one step = "
+                                   "rot 0 + rot 32 (Hadamard) runs",
+                       "rows": ROWS, "cols": COLS, "format": "mxfp4", "block": 32,
+                       "rot": list(ROTS), "outputs": "packed codes + scale bytes",
+                       "l2": "flushed before every launch (2 x L2 write, outside the events)",
+                       "parallelism": f"replicas x{world} (independent tensors, no collective)",
+                       "soak_s": args.soak},
+            "roofline": roofline, "e2e": e2e, "gpu_launches": len(ROTS) * args.steps,
+            "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0 and world == 1 and not args.no_breakdown:
+        line["breakdown"] = breakdown(dev, flush, peaks)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- breakdown
+
+def breakdown(dev, flush, peaks, reps: int = 10):
+    """Every run of every workload, one line each: elements/s, algorithmic
+    GB/s and its fraction of the HBM roofline (FP32 ops for brute force)."""
+    import torch
+
+    import microscaling_fp4_quantization_bf16_b200 as fp4q
+    from microscaling_fp4_quantization_bf16_b200 import synth
+
+    fp32_peak = SM_COUNT_NOMINAL * FP32_LANES_PER_SM * SM_MAX_MHZ_NOMINAL * 1e6
+    rows_out = []
+
+    def timeit(fn, n_launch=1):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts = []
+        for i in range(reps + 3):
+            flush.zero_()
+            s.record()
+            fn()
+            e.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(s.elapsed_time(e))
+        return statistics.median(ts) / 1e3
+
+    def add(name, n, secs, bpe, launches, fp32_ops=None, note=None):
+        gbs = n * bpe / secs / 1e9
+        d = {"run": name, "elements": n, "us": round(secs * 1e6, 2),
+             "elements_per_s": n / secs, "alg_GBps": round(gbs, 1),
+             "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_elem": round(bpe, 5),
+             "launches": launches}
+        if fp32_ops is not None:
+            d["fp32_ops_per_s"] = fp32_ops / secs
+            d["fp32_frac"] = round(fp32_ops / secs / fp32_peak, 4)
+            d["bound"] = "alu"
+        if note:
+            d["note"] = note
+        rows_out.append(d)
+
+    def quant_runs(wl, runs, want_mse=False, dq=None):
+        x = synth.workload(wl)["x"].to(dev)
+        n = x.numel()
+        R, C = x.shape
+        for fmt, block, strat, rot in runs:
+            nv = fmt == "nvfp4"
+            out = fp4q.Quantized(
+                torch.empty(R, C // 2, dtype=torch.uint8, device=dev),
+                torch.empty(R, C // block, dtype=torch.uint8, device=dev),
+                torch.empty(1, device=dev) if nv else None,
+                torch.empty(R, C // block, device=dev) if want_mse else None,
+                torch.empty(R, C, dtype=dq, device=dev) if dq is not None else None)
+            dqb = 0 if dq is None else torch.tensor([], dtype=dq).element_size()
+            bpe = bytes_per_elem(block, mse=want_mse, dq=dqb)
+            ops = n * 126 * 5 if strat == "brute_force" else None
+            tag = f"{wl} {fmt} B{block} {strat} H{rot}"
+            if nv:
+                ga = fp4q.global_amax(x, rot)
+                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, global_amax=ga,
+                                                    out=out))
+                add(tag + " (abs-max supplied, 1 pass)", n, secs, bpe, 1, ops)
+                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, out=out))
+                add(tag + " (abs-max computed, 2 passes)", n, secs, bpe, 3, ops,
+                    note="memset + amax + quantize + finalize; bytes count one read")
+            else:
+                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, out=out))
+                add(tag, n, secs, bpe, 1, ops)
+        del x
+        torch.cuda.empty_cache()
+
+    quant_runs("c1_nvfp4_roundtrip", [("nvfp4", 16, "absmax", 0)], want_mse=True, dq=torch.float32)
+    quant_runs("c2_mxfp4_laplace_outliers", [("mxfp4", 32, "absmax", 0), ("mxfp4", 32, "absmax", 32)])
+    quant_runs("c3_strategy_sweep_t3", [("nvfp4", b, s, 0) for b in (4, 8, 16, 32)
+                                        for s in ("absmax", "prevent_zero", "four_over_six",
+                                                  "brute_force")], want_mse=True)
+    quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
+                                          ("mxfp4", 32, "absmax", 128)])
+    # FOCUS
+    d = synth.workload("c4_focus")
+    w, c, g = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)
+    n = w.numel()
+    for fmt, block in (("nvfp4", 16), ("mxfp4", 32)):
+        fo = fp4q.FocusOut(torch.empty_like(w), torch.empty(1, device=dev) if fmt == "nvfp4" else None,
+                           None, None)
+        ga = fp4q.global_amax(w, 0) if fmt == "nvfp4" else None
+        secs = timeit(lambda: fp4q.focus_fwd(w, c, fmt, block, 8, global_amax=ga, out=fo))
+        add(f"c4_focus fwd {fmt} B{block} sub8 -> bf16", n, secs, 2 + 0.25 + 2, 1)
+    dc = torch.empty(4096, 512, device=dev)
+    secs = timeit(lambda: fp4q.focus_bwd(w, g, c, 8, out=dc))
+    add("c4_focus bwd sub8 -> fp32 dc", n, secs, 2 + 2 + 0.25 + 0.5, 1)
+    return rows_out
+
+
+# ---------------------------------------------------------------- oracle
+
+def cpu_baseline(seconds: float):
+    """The oracle (single-threaded C) on row slices of the headline tensor,
+    both runs, until about `seconds` of CPU work."""
+    import oracle
+    from microscaling_fp4_quantization_bf16_b200 import synth
+
+    x = synth.bits16(synth.workload(WORKLOAD)["x"])
+    oracle.lib()
+    done, t = 0, 0.0
+    r0, chunk = 0, 64
+    while t < seconds:
+        xs = x[r0:r0 + chunk]
+        t0 = time.perf_counter()
+        for r in ROTS:
+            oracle.quantize(xs, "mxfp4", 32, "absmax", r, want_mse=False)
+        t += time.perf_counter() - t0
+        done += xs.size * len(ROTS)
+        r0 = (r0 + chunk) % ROWS
+    return {"value": done / t, "unit": "elements/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done // len(ROTS)} elements ({done // len(ROTS) // COLS} rows of 64) of "
+                      f"the {ROWS}x{COLS} tensor, rot 0 and rot 32 each, single-threaded C "
+                      f"oracle, {t:.1f} s"}
+
+
+def run_reference(args, rank, world):
+    """The oracle as the reference arm: rank 0 times it on a bounded sample
+    per step; other ranks exit without work."""
+    if rank != 0:
+        return
+    import oracle
+    from microscaling_fp4_quantization_bf16_b200 import synth
+
+    x = synth.bits16(synth.workload(WORKLOAD)["x"])
+    oracle.lib()
+    # size each step so the whole run takes about args.ref_seconds
+    t0 = time.perf_counter()
+    oracle.quantize(x[:8], "mxfp4", 32, "absmax", 32, want_mse=False)
+    per_elem = (time.perf_counter() - t0) / (8 * COLS)
+    per_step_s = args.ref_seconds / max(1, args.steps + args.warmup)
+    rows = int(max(1, min(ROWS, per_step_s / (per_elem * COLS * len(ROTS)))))
+    r0 = 0
+
+    def step():
+        nonlocal r0
+        xs = x[r0:r0 + rows] if r0 + rows <= ROWS else x[:rows]
+        for r in ROTS:
+            oracle.quantize(xs, "mxfp4", 32, "absmax", r, want_mse=False)
+        r0 = (r0 + rows) % ROWS
+        return xs.size * len(ROTS)
+
+    for _ in range(args.warmup):
+        step()
+    done = 0
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        done += step()
+    t = time.perf_counter() - t0
+    value = done / t
+    sample = (f"{rows} rows x {COLS} of the {ROWS}x{COLS} tensor per step, rot 0 and rot 32, "
+              "single-threaded C oracle")
+    line = {"metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": f"{WORKLOAD}: MXFP4 E8M0 block 32, rot 0 + rot 32",
+                       "rows": ROWS, "cols": COLS, "format": "mxfp4", "block": 32,
+                       "rot": list(ROTS), "sample_rows_per_step": rows},
+            "cpu_baseline": {"value": value, "unit": "elements/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before warm-up")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--ref-seconds", type=float, default=60.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-breakdown", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if world != args.gpus:
+        print(f"note: WORLD_SIZE={world} but --gpus {args.gpus}", file=sys.stderr)
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+    else:
+        run_ours(args, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,188 @@
+/*
+ * fp4q.h -- C ABI of the B200 (sm_100a) block-scaled FP4 quantization library.
+ *
+ * Formats. A tensor is a row-major bf16 matrix [rows, cols]; blocks of
+ * `block` consecutive elements along a row share one scale.
+ *   NVFP4: E2M1 elements, one OCP E4M3 scale byte per block and one FP32
+ *          per-tensor global scale s_g = amax / (448 * 6) (hierarchical
+ *          scaling); block 16 is the hardware block, 4 / 8 / 32 are also
+ *          provided ("Finer is Better (with the Right Scaling)", 手法 1-2).
+ *   MXFP4: E2M1 elements, one E8M0 (power-of-two) scale byte per block of 32
+ *          ("Bridging the Gap Between Promise and Performance for
+ *          Microscaling FP4 Quantization", 技術概要 §1).
+ *
+ * Storage. codes: uint8 [rows, cols/2], element 2j in the low nibble of byte
+ * j and element 2j+1 in the high nibble; 4-bit code = sign bit (bit 3) and
+ * E2M1 magnitude index (bits 0-2). scales: uint8 [rows, cols/block]
+ * row-major (E4M3 code, or E8M0 byte = exponent + 127). Per-block MSE:
+ * float [rows, cols/block]. Dequantized values: [rows, cols] fp32 or bf16.
+ *
+ * Arithmetic. Every result is bit-identical to the plain CPU definition of
+ * the operation: one IEEE binary32 operation per step, no fused
+ * multiply-add, E2M1 / E4M3 round-to-nearest-even with saturation, the
+ * optional Hadamard rotation applied as a Walsh-Hadamard butterfly with
+ * ascending stages, and block sums taken with the adjacent-pair tree.
+ *
+ * Conventions for every entry point:
+ *  - All array pointers are DEVICE pointers owned by the caller, 16-byte
+ *    aligned, dense row-major (leading dimension = cols). The library never
+ *    allocates, frees, or keeps memory or state between calls, and never
+ *    synchronises: work is enqueued on `stream` (0 = legacy default stream)
+ *    and the call returns before it completes.
+ *  - Arguments are validated on the host before anything is enqueued; on an
+ *    error nothing is launched and outputs are untouched.
+ *  - rows == 0 or cols == 0 is an empty tensor: nothing is computed except
+ *    that NVFP4 global_scale_out receives 1.0.
+ *  - Inputs must be finite. Outputs must not overlap inputs or each other.
+ *  - FP4Q_ERR_CUDA means a launch was rejected by the CUDA runtime; the
+ *    runtime's code is available from fp4q_last_cuda_error(). Faults that
+ *    happen while the kernels run surface at the caller's next
+ *    synchronisation, as for any CUDA work.
+ */
+#ifndef FP4Q_H
+#define FP4Q_H
+
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    FP4Q_OK = 0,
+    FP4Q_ERR_NULL = 1,        /* a required pointer is NULL */
+    FP4Q_ERR_SHAPE = 2,       /* negative sizes, or cols not a multiple of block / rot / sub */
+    FP4Q_ERR_ALIGN = 3,       /* an array pointer is not 16-byte aligned (4 for scalars) */
+    FP4Q_ERR_UNSUPPORTED = 4, /* format / block / strategy / rotation / sub not offered */
+    FP4Q_ERR_ALIAS = 5,       /* global_amax_in and global_scale_out are the same address */
+    FP4Q_ERR_CUDA = 6         /* the CUDA runtime rejected a launch */
+} fp4q_status;
+
+typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1 } fp4q_format;
+
+/* Block-scale selection ("Finer is Better (with the Right Scaling)", 手法 2).
+ * MXFP4 offers FP4Q_ABSMAX only. */
+typedef enum {
+    FP4Q_ABSMAX = 0,        /* code = RNE_E4M3(amax / (6 s_g)) */
+    FP4Q_PREVENT_ZERO = 1,  /* abs-max code clipped below at 0x01 (2^-9) */
+    FP4Q_FOUR_OVER_SIX = 2, /* targets 6 and 4; keep 4 only if its block SSE is lower */
+    FP4Q_BRUTE_FORCE = 3    /* minimum block SSE over codes 0x01..0x7E; ties -> lower code */
+} fp4q_strategy;
+
+typedef enum { FP4Q_OUT_F32 = 0, FP4Q_OUT_BF16 = 1 } fp4q_dtype;
+
+/*
+ * fp4q_quantize -- rotate (optional) -> per-block scale -> E2M1 RNE -> pack,
+ * with optional dequantized values and per-block MSE.
+ *
+ * x                bf16 [rows, cols].
+ * fmt, block       NVFP4 with block in {4, 8, 16, 32}; MXFP4 with block 32.
+ * strat            see fp4q_strategy.
+ * rot              0 (none) or the blockwise Hadamard size 16, 32, 64, 128:
+ *                  every rot-wide chunk of a row becomes H_rot x / sqrt(rot)
+ *                  before scaling ("Bridging the Gap ...", 技術概要 §2.2
+ *                  item 3); codes, dq and MSE are in the rotated domain.
+ * global_amax_in   NVFP4: NULL to compute the abs-max of the (rotated)
+ *                  tensor on the device (an extra read of x), or a device
+ *                  float holding a calibrated abs-max (single pass). Ignored
+ *                  for MXFP4.
+ * global_scale_out NVFP4: required device float, receives s_g. Ignored for
+ *                  MXFP4. When global_amax_in is NULL it is also used to
+ *                  accumulate the abs-max before s_g replaces it.
+ * codes            uint8 [rows, cols/2], required.
+ * scales           uint8 [rows, cols/block], required.
+ * block_mse        float [rows, cols/block] or NULL.
+ * dq               [rows, cols] of dq_dtype, or NULL.
+ * Errors: NULL, SHAPE (cols % block, cols % rot), ALIGN, UNSUPPORTED
+ * (MXFP4 with a strategy other than ABSMAX, unknown enum values), ALIAS, CUDA.
+ */
+fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                          fp4q_strategy strat, int rot, const float* global_amax_in,
+                          float* global_scale_out, uint8_t* codes, uint8_t* scales,
+                          float* block_mse, void* dq, fp4q_dtype dq_dtype, cudaStream_t stream);
+
+/*
+ * fp4q_dequantize -- value(code) * S with S = E4M3(scale) * s_g (NVFP4) or
+ * 2^(scale - 127) (MXFP4); only the dequantization scale is needed at
+ * inference ("FOCUS: FP4 Optimization via Coupled-Relaxation and
+ * Dual-Granularity Scaling", Metodologia §4).
+ * global_scale: NVFP4 device float s_g (required); ignored for MXFP4.
+ * out: [rows, cols] of out_dtype (bf16 output is the RNE rounding of the fp32 value).
+ */
+fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
+                            const float* global_scale, int64_t rows, int64_t cols,
+                            fp4q_format fmt, int block, void* out, fp4q_dtype out_dtype,
+                            cudaStream_t stream);
+
+/*
+ * fp4q_block_mse -- per-block mean squared error of x (rotated by rot first)
+ * against dequantize(codes, scales): tree sum of (y - yhat)^2 divided by
+ * block ("Finer is Better (with the Right Scaling)", 手法 1: MSE per block
+ * size). Equal bit for bit to fp4q_quantize's block_mse for its own codes.
+ */
+fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,
+                           const float* global_scale, int64_t rows, int64_t cols,
+                           fp4q_format fmt, int block, int rot, float* block_mse,
+                           cudaStream_t stream);
+
+/*
+ * fp4q_focus_fwd -- FOCUS decoupled fake quantization (CRS + DGS):
+ * W_hat = S_dq * Q(W / (S_dq * c_k)) where S_dq is the format's abs-max block
+ * scale (shared by the hardware block) and c_k is the fp16 coefficient of
+ * sub-block k ("FOCUS: ...", Metodologia §2 S_q = S_dq * c_i, §3 sub-block
+ * formula). sub == block is CRS alone.
+ * w        bf16 [rows, cols]; c: fp16 [rows, cols/sub]; sub in {2,4,8,16,32},
+ *          dividing block.
+ * global_amax_in / global_scale_out: as fp4q_quantize (NVFP4; abs-max of W).
+ * w_hat    [rows, cols] of out_dtype, required.
+ * codes, scales: optional deployable export (both or neither): the FP4 codes
+ *          Q(W / (S_dq * c_k)) and the S_dq bytes; the coefficients are not
+ *          part of it (Metodologia §4).
+ */
+fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t cols,
+                           fp4q_format fmt, int block, int sub, const float* global_amax_in,
+                           float* global_scale_out, void* w_hat, fp4q_dtype out_dtype,
+                           uint8_t* codes, uint8_t* scales, cudaStream_t stream);
+
+/*
+ * fp4q_focus_bwd -- straight-through gradient of the coefficients
+ * ("FOCUS: ...", Metodologia §1 STE): with dQ/du taken as 1,
+ * dL/dc_k = -(sum over sub-block k of g_j * W_j) / (c_k * c_k), the sum in
+ * fp32 with the adjacent-pair tree. S_dq receives no gradient.
+ * w, g     bf16 [rows, cols] (g = dL/dW_hat); c: fp16 [rows, cols/sub];
+ * dc       float [rows, cols/sub]; sub in {2,4,8,16,32}.
+ */
+fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t rows,
+                           int64_t cols, int sub, float* dc, cudaStream_t stream);
+
+/*
+ * fp4q_global_amax -- abs-max of the (rotated) tensor into *amax_out (device
+ * float): the per-tensor statistic of hierarchical scaling ("Finer is Better
+ * (with the Right Scaling)", 手法 2). Feed it to global_amax_in of the calls
+ * above to run them as a single pass.
+ */
+fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax_out,
+                             cudaStream_t stream);
+
+/*
+ * Element-wise rounding primitives used by every kernel above, exposed so
+ * that they can be checked exhaustively: one output byte per input float.
+ * fp4q_e2m1_encode: 4-bit E2M1 code (sign kept, RNE, saturating at +-6).
+ * fp4q_e4m3_encode: E4M3 code of v >= 0 (RNE, saturating at 448).
+ */
+fp4q_status fp4q_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t stream);
+fp4q_status fp4q_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t stream);
+
+/* Human-readable name of a status code (static string). */
+const char* fp4q_status_string(fp4q_status s);
+
+/* The cudaError_t of the last FP4Q_ERR_CUDA returned on this host thread. */
+int fp4q_last_cuda_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP4Q_H */

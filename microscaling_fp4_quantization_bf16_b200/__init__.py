@@ -1,0 +1,178 @@
+"""B200-native block-scaled FP4 quantization (MXFP4 / NVFP4) and FOCUS.
+
+PyTorch is used for device memory and streams only: every function below
+allocates its outputs with torch (unless given preallocated ones), then calls
+the C ABI of libfp4q.so on ``torch.cuda.current_stream()``. All arithmetic
+runs in the library's sm_100a kernels. Nothing here computes on the CPU.
+
+Pages: "Finer is Better (with the Right Scaling)" (scale strategies, block
+sizes), "Bridging the Gap Between Promise and Performance for Microscaling FP4
+Quantization" (MXFP4 / NVFP4, blockwise Hadamard rotation), "FOCUS: FP4
+Optimization via Coupled-Relaxation and Dual-Granularity Scaling" (decoupled
+fake quantization and its straight-through gradient).
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from ._abi import Fp4qError, load  # noqa: F401
+from . import _abi
+
+FORMATS = {"nvfp4": 0, "mxfp4": 1}
+STRATEGIES = {"absmax": 0, "prevent_zero": 1, "four_over_six": 2, "brute_force": 3}
+DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else t.data_ptr()
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _check(t: torch.Tensor, dtype, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _fmt(fmt) -> int:
+    return FORMATS[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+def _strat(s) -> int:
+    return STRATEGIES[s] if isinstance(s, str) else int(s)
+
+
+@dataclass
+class Quantized:
+    codes: torch.Tensor                   # uint8 [rows, cols/2]
+    scales: torch.Tensor                  # uint8 [rows, cols/block]
+    global_scale: Optional[torch.Tensor]  # float32 [1] (NVFP4) or None
+    mse: Optional[torch.Tensor]           # float32 [rows, cols/block] or None
+    dq: Optional[torch.Tensor]            # [rows, cols] float32/bfloat16 or None
+
+
+def quantize(x: torch.Tensor, fmt="nvfp4", block: int = 16, strategy="absmax", rot: int = 0,
+             global_amax: Optional[torch.Tensor] = None, want_mse: bool = False,
+             dq_dtype: Optional[torch.dtype] = None, out: Optional[Quantized] = None) -> Quantized:
+    """Quantize a bf16 [rows, cols] tensor. See fp4q_quantize in include/fp4q.h."""
+    _check(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    f = _fmt(fmt)
+    if out is None:
+        dev = x.device
+        out = Quantized(
+            codes=torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+            scales=torch.empty(rows, cols // block, dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev) if f == 0 else None,
+            mse=torch.empty(rows, cols // block, dtype=torch.float32, device=dev) if want_mse else None,
+            dq=torch.empty(rows, cols, dtype=dq_dtype, device=dev) if dq_dtype is not None else None,
+        )
+    if global_amax is not None:
+        _check(global_amax, torch.float32, "global_amax")
+    _abi.call("fp4q_quantize", x.data_ptr(), rows, cols, f, block, _strat(strategy), rot,
+              _ptr(global_amax), _ptr(out.global_scale), out.codes.data_ptr(),
+              out.scales.data_ptr(), _ptr(out.mse), _ptr(out.dq),
+              DTYPES[out.dq.dtype] if out.dq is not None else 0, _stream())
+    return out
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, global_scale: Optional[torch.Tensor],
+               fmt="nvfp4", block: int = 16, dtype: torch.dtype = torch.float32,
+               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    rows, half = codes.shape
+    cols = 2 * half
+    if out is None:
+        out = torch.empty(rows, cols, dtype=dtype, device=codes.device)
+    _abi.call("fp4q_dequantize", codes.data_ptr(), scales.data_ptr(), _ptr(global_scale), rows,
+              cols, _fmt(fmt), block, out.data_ptr(), DTYPES[out.dtype], _stream())
+    return out
+
+
+def block_mse(x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor,
+              global_scale: Optional[torch.Tensor], fmt="nvfp4", block: int = 16, rot: int = 0,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _check(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty(rows, cols // block, dtype=torch.float32, device=x.device)
+    _abi.call("fp4q_block_mse", x.data_ptr(), codes.data_ptr(), scales.data_ptr(),
+              _ptr(global_scale), rows, cols, _fmt(fmt), block, rot, out.data_ptr(), _stream())
+    return out
+
+
+@dataclass
+class FocusOut:
+    w_hat: torch.Tensor
+    global_scale: Optional[torch.Tensor]
+    codes: Optional[torch.Tensor]
+    scales: Optional[torch.Tensor]
+
+
+def focus_fwd(w: torch.Tensor, c: torch.Tensor, fmt="nvfp4", block: int = 16, sub: int = 8,
+              global_amax: Optional[torch.Tensor] = None, out_dtype: torch.dtype = torch.bfloat16,
+              want_codes: bool = False, out: Optional[FocusOut] = None) -> FocusOut:
+    """FOCUS fake quantization W_hat = S_dq * Q(W / (S_dq * c_k))."""
+    _check(w, torch.bfloat16, "w")
+    _check(c, torch.float16, "c")
+    rows, cols = w.shape
+    f = _fmt(fmt)
+    if out is None:
+        dev = w.device
+        out = FocusOut(
+            w_hat=torch.empty(rows, cols, dtype=out_dtype, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev) if f == 0 else None,
+            codes=torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev) if want_codes else None,
+            scales=torch.empty(rows, cols // block, dtype=torch.uint8, device=dev) if want_codes else None,
+        )
+    _abi.call("fp4q_focus_fwd", w.data_ptr(), c.data_ptr(), rows, cols, f, block, sub,
+              _ptr(global_amax), _ptr(out.global_scale), out.w_hat.data_ptr(),
+              DTYPES[out.w_hat.dtype], _ptr(out.codes), _ptr(out.scales), _stream())
+    return out
+
+
+def focus_bwd(w: torch.Tensor, g: torch.Tensor, c: torch.Tensor, sub: int = 8,
+              out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Straight-through dL/dc_k = -(sum_k g * W) / c_k^2, fp32 [rows, cols/sub]."""
+    _check(w, torch.bfloat16, "w")
+    _check(g, torch.bfloat16, "g")
+    _check(c, torch.float16, "c")
+    rows, cols = w.shape
+    if out is None:
+        out = torch.empty(rows, cols // sub, dtype=torch.float32, device=w.device)
+    _abi.call("fp4q_focus_bwd", w.data_ptr(), g.data_ptr(), c.data_ptr(), rows, cols, sub,
+              out.data_ptr(), _stream())
+    return out
+
+
+def global_amax(x: torch.Tensor, rot: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _check(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    if out is None:
+        out = torch.empty(1, dtype=torch.float32, device=x.device)
+    _abi.call("fp4q_global_amax", x.data_ptr(), rows, cols, rot, out.data_ptr(), _stream())
+    return out
+
+
+def e2m1_encode(u: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _check(u, torch.float32, "u")
+    if out is None:
+        out = torch.empty(u.shape, dtype=torch.uint8, device=u.device)
+    _abi.call("fp4q_e2m1_encode", u.data_ptr(), u.numel(), out.data_ptr(), _stream())
+    return out
+
+
+def e4m3_encode(v: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    _check(v, torch.float32, "v")
+    if out is None:
+        out = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
+    _abi.call("fp4q_e4m3_encode", v.data_ptr(), v.numel(), out.data_ptr(), _stream())
+    return out

@@ -1,0 +1,338 @@
+// api.cu -- the extern "C" entry points declared in include/fp4q.h.
+//
+// Host side only: validate every argument, then enqueue kernels on the
+// caller's stream. Nothing is allocated and nothing is synchronised.
+#include <cstdint>
+
+#include "fp4q.h"
+#include "internal.h"
+
+using namespace fp4q;
+
+namespace {
+
+thread_local int g_last_cuda_error = 0;
+
+fp4q_status cuda_status(cudaError_t e)
+{
+    if (e == cudaSuccess)
+        return FP4Q_OK;
+    g_last_cuda_error = (int)e;
+    return FP4Q_ERR_CUDA;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+bool valid_rot(int rot) { return rot == 0 || rot == 16 || rot == 32 || rot == 64 || rot == 128; }
+
+bool valid_sub(int sub) { return sub == 2 || sub == 4 || sub == 8 || sub == 16 || sub == 32; }
+
+// Largest tensor accepted: 2^40 elements (far above any device's memory);
+// keeps every derived index and grid size inside int64 / 2^31 blocks.
+constexpr int64_t kMaxElems = (int64_t)1 << 40;
+
+// Shared checks of format, block and rotation against the shape.
+fp4q_status check_format(int64_t rows, int64_t cols, int fmt, int block, int rot)
+{
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_FMT_MXFP4 && block != 32)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_FMT_NVFP4 && block != 4 && block != 8 && block != 16 && block != 32)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (!valid_rot(rot))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0)
+        return FP4Q_ERR_SHAPE;
+    if (cols % block != 0 || (rot > 0 && cols % rot != 0))
+        return FP4Q_ERR_SHAPE;
+    if (cols > 0 && rows > kMaxElems / cols)
+        return FP4Q_ERR_SHAPE;
+    return FP4Q_OK;
+}
+
+cudaError_t launch_quant(int block, int strat, int rot, const QuantArgs& a, cudaStream_t st)
+{
+    switch (block) {
+    case 4: return launch_quant_b4(strat, rot, a, st);
+    case 8: return launch_quant_b8(strat, rot, a, st);
+    case 16: return launch_quant_b16(strat, rot, a, st);
+    case 32: return launch_quant_b32(strat, rot, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// NVFP4 global abs-max without a caller value: zero the output float, fold
+// the tensor's abs-max into it (atomicMax on the bits), and return it as the
+// amax pointer for the kernel that follows.
+fp4q_status accumulate_amax(const void* x, int64_t n, int rot, float* global_scale_out,
+                            cudaStream_t st)
+{
+    cudaError_t e = cudaMemsetAsync(global_scale_out, 0, sizeof(float), st);
+    if (e != cudaSuccess)
+        return cuda_status(e);
+    return cuda_status(launch_amax(static_cast<const uint16_t*>(x), n, rot,
+                                   reinterpret_cast<unsigned*>(global_scale_out), st));
+}
+
+}  // namespace
+
+extern "C" {
+
+fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                          fp4q_strategy strat, int rot, const float* global_amax_in,
+                          float* global_scale_out, uint8_t* codes, uint8_t* scales,
+                          float* block_mse, void* dq, fp4q_dtype dq_dtype, cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, rot);
+    if (st != FP4Q_OK)
+        return st;
+    if (strat < FP4Q_ABSMAX || strat > FP4Q_BRUTE_FORCE)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (fmt == FP4Q_FMT_MXFP4 && strat != FP4Q_ABSMAX)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (dq != nullptr && dq_dtype != FP4Q_OUT_F32 && dq_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    if (x == nullptr || codes == nullptr || scales == nullptr || (nv && global_scale_out == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(block_mse) ||
+        !aligned16(dq))
+        return FP4Q_ERR_ALIGN;
+    if (nv && (!aligned4(global_scale_out) || !aligned4(global_amax_in)))
+        return FP4Q_ERR_ALIGN;
+    if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
+        return FP4Q_ERR_ALIAS;
+
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
+
+    QuantArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.n = n;
+    a.codes = codes;
+    a.scales = scales;
+    a.mse = block_mse;
+    a.dq = dq;
+    a.dq_kind = dq == nullptr ? 0 : (dq_dtype == FP4Q_OUT_F32 ? 1 : 2);
+    a.amax = nullptr;
+    a.sg_out = nullptr;
+    int kstrat = nv ? (int)strat : K_MX;
+    if (nv) {
+        if (global_amax_in != nullptr) {
+            a.amax = global_amax_in;
+            a.sg_out = global_scale_out;
+        } else {
+            st = accumulate_amax(x, n, rot, global_scale_out, stream);
+            if (st != FP4Q_OK)
+                return st;
+            a.amax = global_scale_out;  // holds the abs-max until finalised below
+        }
+    }
+    st = cuda_status(launch_quant(block, kstrat, rot, a, stream));
+    if (st != FP4Q_OK)
+        return st;
+    if (nv && global_amax_in == nullptr)
+        st = cuda_status(launch_finalize_sg(global_scale_out, stream));
+    return st;
+}
+
+fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
+                            const float* global_scale, int64_t rows, int64_t cols,
+                            fp4q_format fmt, int block, void* out, fp4q_dtype out_dtype,
+                            cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, 0);
+    if (st != FP4Q_OK)
+        return st;
+    if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    if (codes == nullptr || scales == nullptr || out == nullptr || (nv && global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (nv && !aligned4(global_scale)))
+        return FP4Q_ERR_ALIGN;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    DequantArgs a;
+    a.codes = codes;
+    a.scales = scales;
+    a.sg = nv ? global_scale : nullptr;
+    a.n = n;
+    a.out = out;
+    a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
+    return cuda_status(launch_dequant(nv ? 0 : 1, block, a, stream));
+}
+
+fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,
+                           const float* global_scale, int64_t rows, int64_t cols,
+                           fp4q_format fmt, int block, int rot, float* block_mse,
+                           cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, rot);
+    if (st != FP4Q_OK)
+        return st;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    if (x == nullptr || codes == nullptr || scales == nullptr || block_mse == nullptr ||
+        (nv && global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(block_mse) ||
+        (nv && !aligned4(global_scale)))
+        return FP4Q_ERR_ALIGN;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    MseArgs a;
+    a.x = static_cast<const uint16_t*>(x);
+    a.codes = codes;
+    a.scales = scales;
+    a.sg = nv ? global_scale : nullptr;
+    a.n = n;
+    a.mse = block_mse;
+    return cuda_status(launch_block_mse(nv ? 0 : 1, block, rot, a, stream));
+}
+
+fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t cols,
+                           fp4q_format fmt, int block, int sub, const float* global_amax_in,
+                           float* global_scale_out, void* w_hat, fp4q_dtype out_dtype,
+                           uint8_t* codes, uint8_t* scales, cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, 0);
+    if (st != FP4Q_OK)
+        return st;
+    if (!valid_sub(sub) || sub > block)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    if (w == nullptr || c == nullptr || w_hat == nullptr || (nv && global_scale_out == nullptr))
+        return FP4Q_ERR_NULL;
+    if ((codes == nullptr) != (scales == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(w) || !aligned16(c) || !aligned16(w_hat) || !aligned16(codes) || !aligned16(scales))
+        return FP4Q_ERR_ALIGN;
+    if (nv && (!aligned4(global_scale_out) || !aligned4(global_amax_in)))
+        return FP4Q_ERR_ALIGN;
+    if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
+        return FP4Q_ERR_ALIAS;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
+
+    FocusFwdArgs a;
+    a.w = static_cast<const uint16_t*>(w);
+    a.c = static_cast<const uint16_t*>(c);
+    a.n = n;
+    a.amax = nullptr;
+    a.sg_out = nullptr;
+    a.w_hat = w_hat;
+    a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
+    a.codes = codes;
+    a.scales = scales;
+    if (nv) {
+        if (global_amax_in != nullptr) {
+            a.amax = global_amax_in;
+            a.sg_out = global_scale_out;
+        } else {
+            st = accumulate_amax(w, n, 0, global_scale_out, stream);
+            if (st != FP4Q_OK)
+                return st;
+            a.amax = global_scale_out;
+        }
+    }
+    st = cuda_status(launch_focus_fwd(nv ? 0 : 1, block, sub, a, stream));
+    if (st != FP4Q_OK)
+        return st;
+    if (nv && global_amax_in == nullptr)
+        st = cuda_status(launch_finalize_sg(global_scale_out, stream));
+    return st;
+}
+
+fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t rows,
+                           int64_t cols, int sub, float* dc, cudaStream_t stream)
+{
+    if (!valid_sub(sub))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0 || cols % sub != 0 || (cols > 0 && rows > kMaxElems / cols))
+        return FP4Q_ERR_SHAPE;
+    if (w == nullptr || g == nullptr || c == nullptr || dc == nullptr)
+        return FP4Q_ERR_NULL;
+    if (!aligned16(w) || !aligned16(g) || !aligned16(c) || !aligned16(dc))
+        return FP4Q_ERR_ALIGN;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    FocusBwdArgs a;
+    a.w = static_cast<const uint16_t*>(w);
+    a.g = static_cast<const uint16_t*>(g);
+    a.c = static_cast<const uint16_t*>(c);
+    a.n = n;
+    a.dc = dc;
+    return cuda_status(launch_focus_bwd(sub, a, stream));
+}
+
+fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax_out,
+                             cudaStream_t stream)
+{
+    if (!valid_rot(rot))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0 || (rot > 0 && cols % rot != 0) || (cols > 0 && rows > kMaxElems / cols))
+        return FP4Q_ERR_SHAPE;
+    if (x == nullptr || amax_out == nullptr)
+        return FP4Q_ERR_NULL;
+    if (!aligned16(x) || !aligned4(amax_out))
+        return FP4Q_ERR_ALIGN;
+    const int64_t n = rows * cols;
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
+    if (e != cudaSuccess || n == 0)
+        return cuda_status(e);
+    return cuda_status(
+        launch_amax(static_cast<const uint16_t*>(x), n, rot, reinterpret_cast<unsigned*>(amax_out), stream));
+}
+
+fp4q_status fp4q_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t stream)
+{
+    if (n < 0 || n > kMaxElems)
+        return FP4Q_ERR_SHAPE;
+    if (u == nullptr || out == nullptr)
+        return FP4Q_ERR_NULL;
+    if (!aligned16(u) || !aligned16(out))
+        return FP4Q_ERR_ALIGN;
+    if (n == 0)
+        return FP4Q_OK;
+    return cuda_status(launch_e2m1_encode(u, n, out, stream));
+}
+
+fp4q_status fp4q_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t stream)
+{
+    if (n < 0 || n > kMaxElems)
+        return FP4Q_ERR_SHAPE;
+    if (v == nullptr || out == nullptr)
+        return FP4Q_ERR_NULL;
+    if (!aligned16(v) || !aligned16(out))
+        return FP4Q_ERR_ALIGN;
+    if (n == 0)
+        return FP4Q_OK;
+    return cuda_status(launch_e4m3_encode(v, n, out, stream));
+}
+
+const char* fp4q_status_string(fp4q_status s)
+{
+    switch (s) {
+    case FP4Q_OK: return "ok";
+    case FP4Q_ERR_NULL: return "a required pointer is NULL";
+    case FP4Q_ERR_SHAPE: return "invalid shape (negative, or cols not a multiple of block/rot/sub)";
+    case FP4Q_ERR_ALIGN: return "pointer not aligned (16 bytes for arrays, 4 for scalars)";
+    case FP4Q_ERR_UNSUPPORTED: return "unsupported format/block/strategy/rotation/sub/dtype";
+    case FP4Q_ERR_ALIAS: return "global_amax_in and global_scale_out alias";
+    case FP4Q_ERR_CUDA: return "CUDA launch error (see fp4q_last_cuda_error)";
+    default: return "unknown status";
+    }
+}
+
+int fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+
+}  // extern "C"

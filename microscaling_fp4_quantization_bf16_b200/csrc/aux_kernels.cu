@@ -1,0 +1,515 @@
+// aux_kernels.cu -- global abs-max, dequantize, block MSE, FOCUS forward and
+// backward, and the element-wise rounding primitives.
+//
+// Same thread layout as the quantize kernel: one 32-element segment of the
+// flattened tensor per thread, 128-bit loads and stores on full segments.
+#include <cmath>
+
+#include "fp4q_device.cuh"
+#include "internal.h"
+
+namespace fp4q {
+
+constexpr int ATHREADS = 256;
+
+static inline unsigned grid_for(int64_t nseg)
+{
+    return (unsigned)((nseg + ATHREADS - 1) / ATHREADS);
+}
+
+static inline bool grid_ok(int64_t nseg)
+{
+    const int64_t nblk = (nseg + ATHREADS - 1) / ATHREADS;
+    return nblk > 0 && nblk <= 0x7FFFFFFF;
+}
+
+// E8M0 byte -> 2^(b - 127); 255 is NaN.
+__device__ __forceinline__ float e8m0_dec(uint32_t b)
+{
+    if (b == 255u)
+        return __uint_as_float(0x7FC00000u);
+    return b == 0u ? __uint_as_float(0x00200000u) : __uint_as_float(b << 23);
+}
+
+// ------------------------------------------------------------ global abs-max
+
+// Tensor abs-max of the (rotated) tensor, combined across blocks with an
+// unsigned atomicMax on the float bits (non-negative floats order like their
+// bit patterns). *out must hold +0 before the launch.
+template <int ROT>
+__global__ void __launch_bounds__(ATHREADS) amax_kernel(const uint16_t* x, int64_t n, unsigned* out)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = (n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    unsigned m = 0;
+    if (s - lane < nseg) {
+        if constexpr (ROT == 0) {
+            if (s < nseg) {
+                const int64_t base = s * SEG;
+                if (base + SEG <= n) {
+                    const uint4* p = reinterpret_cast<const uint4*>(x + base);
+                    unsigned acc = 0;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        uint4 v = ldg_stream(p + k);
+                        acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
+                        acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
+                        acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
+                        acc = __vmaxu2(acc, v.w & 0x7FFF7FFFu);
+                    }
+                    m = max(acc & 0xFFFFu, acc >> 16) << 16;
+                } else {
+                    for (int64_t i = base; i < n; ++i)
+                        m = max(m, ((unsigned)x[i] & 0x7FFFu) << 16);
+                }
+            }
+        } else {
+            float y[SEG];
+            load_seg_bf16(x, n, s, y);
+            rotate_seg<ROT>(y, lane);
+            if (s < nseg) {
+#pragma unroll
+                for (int i = 0; i < SEG; ++i)
+                    m = max(m, __float_as_uint(fabsf(y[i])));
+            }
+        }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    __shared__ unsigned wm[ATHREADS / 32];
+    if (lane == 0)
+        wm[threadIdx.x / 32] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        unsigned v = lane < ATHREADS / 32 ? wm[lane] : 0u;
+        v = __reduce_max_sync(0xFFFFFFFFu, v);
+        if (lane == 0 && v != 0u)
+            atomicMax(out, v);
+    }
+}
+
+__global__ void finalize_sg_kernel(float* g) { *g = global_scale_of(*g); }
+
+__global__ void set_one_kernel(float* p) { *p = 1.0f; }
+
+cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st)
+{
+    const int64_t nseg = (n + SEG - 1) / SEG;
+    if (!grid_ok(nseg))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    switch (rot) {
+    case 0: amax_kernel<0><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    case 16: amax_kernel<16><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    case 32: amax_kernel<32><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    case 64: amax_kernel<64><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    case 128: amax_kernel<128><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_finalize_sg(float* g, cudaStream_t st)
+{
+    finalize_sg_kernel<<<1, 1, 0, st>>>(g);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_set_one(float* p, cudaStream_t st)
+{
+    set_one_kernel<<<1, 1, 0, st>>>(p);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ small helpers
+
+// Codes of segment s (16 bytes), byte by byte when the segment is partial.
+__device__ __forceinline__ void load_codes(const uint8_t* codes, int64_t s, int nvalid, uint32_t (&q)[4])
+{
+    if (nvalid == SEG) {
+        uint4 c = *reinterpret_cast<const uint4*>(codes + s * (SEG / 2));
+        q[0] = c.x; q[1] = c.y; q[2] = c.z; q[3] = c.w;
+    } else {
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            uint32_t v = 0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (2 * (4 * w + k) < nvalid)
+                    v |= (uint32_t)codes[s * (SEG / 2) + 4 * w + k] << (8 * k);
+            q[w] = v;
+        }
+    }
+}
+
+template <int NB>
+__device__ __forceinline__ void load_scale_bytes(const uint8_t* scales, int64_t s, int nvalid, int B,
+                                                 uint32_t (&sc)[NB])
+{
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        sc[b] = (b * B < nvalid) ? (uint32_t)scales[s * NB + b] : 0u;
+}
+
+template <int NB, bool MX>
+__device__ __forceinline__ void scales_of(const uint32_t (&sc)[NB], float sg, float (&S)[NB])
+{
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        S[b] = MX ? e8m0_dec(sc[b]) : __fmul_rn(e4m3_dec(sc[b]), sg);
+}
+
+// Writes NK floats of segment s (NK = 32 / granularity) to p + s * NK.
+template <int NK>
+__device__ __forceinline__ void store_seg_floats(float* p, int64_t s, int nvalid, int gran,
+                                                 const float (&v)[NK])
+{
+    float* o = p + s * NK;
+    if (nvalid == SEG) {
+        if constexpr (NK >= 4) {
+#pragma unroll
+            for (int k = 0; k < NK / 4; ++k)
+                reinterpret_cast<float4*>(o)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else if constexpr (NK == 2) {
+            *reinterpret_cast<float2*>(o) = make_float2(v[0], v[1]);
+        } else {
+            *o = v[0];
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NK; ++k)
+            if (k * gran < nvalid)
+                o[k] = v[k];
+    }
+}
+
+// ------------------------------------------------------------ dequantize
+
+template <int B, bool MX>
+__global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
+{
+    constexpr int NB = SEG / B;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    uint32_t q[4], sc[NB];
+    load_codes(a.codes, s, nvalid, q);
+    load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+    const float sg = MX ? 1.0f : *a.sg;
+    float S[NB], yh[SEG];
+    scales_of<NB, MX>(sc, sg, S);
+    decode_seg<B>(q, S, yh);
+    store_seg_values(a.out, a.out_kind, s, nvalid, yh);
+}
+
+cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    if (!grid_ok(nseg))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    if (mx) {
+        if (block != 32)
+            return cudaErrorInvalidValue;
+        dequant_kernel<32, true><<<g, ATHREADS, 0, st>>>(a);
+    } else {
+        switch (block) {
+        case 4: dequant_kernel<4, false><<<g, ATHREADS, 0, st>>>(a); break;
+        case 8: dequant_kernel<8, false><<<g, ATHREADS, 0, st>>>(a); break;
+        case 16: dequant_kernel<16, false><<<g, ATHREADS, 0, st>>>(a); break;
+        case 32: dequant_kernel<32, false><<<g, ATHREADS, 0, st>>>(a); break;
+        default: return cudaErrorInvalidValue;
+        }
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ block MSE
+
+template <int B, int ROT, bool MX>
+__global__ void __launch_bounds__(ATHREADS) block_mse_kernel(MseArgs a)
+{
+    constexpr int NB = SEG / B;
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (s - lane >= nseg)
+        return;
+    float y[SEG];
+    load_seg_bf16(a.x, a.n, s, y);
+    rotate_seg<ROT>(y, lane);
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    uint32_t q[4], sc[NB];
+    load_codes(a.codes, s, nvalid, q);
+    load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+    const float sg = MX ? 1.0f : *a.sg;
+    float S[NB], sse[NB], m[NB];
+    scales_of<NB, MX>(sc, sg, S);
+    sse_seg<B>(y, q, S, sse);
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        m[b] = __fmul_rn(sse[b], 1.0f / B);
+    store_seg_floats<NB>(a.mse, s, nvalid, B, m);
+}
+
+template <int B, bool MX>
+static cudaError_t launch_mse_rot(int rot, unsigned g, const MseArgs& a, cudaStream_t st)
+{
+    switch (rot) {
+    case 0: block_mse_kernel<B, 0, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    case 16: block_mse_kernel<B, 16, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    case 32: block_mse_kernel<B, 32, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    case 64: block_mse_kernel<B, 64, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    case 128: block_mse_kernel<B, 128, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    if (!grid_ok(nseg))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    if (mx)
+        return block == 32 ? launch_mse_rot<32, true>(rot, g, a, st) : cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_mse_rot<4, false>(rot, g, a, st);
+    case 8: return launch_mse_rot<8, false>(rot, g, a, st);
+    case 16: return launch_mse_rot<16, false>(rot, g, a, st);
+    case 32: return launch_mse_rot<32, false>(rot, g, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// ------------------------------------------------------------ FOCUS
+
+// fp16 coefficients of segment s: NK = 32 / SUB values at c + s * NK.
+template <int NK>
+__device__ __forceinline__ void load_coeffs(const uint16_t* c, int64_t s, int nvalid, int sub, float (&ck)[NK])
+{
+    const uint16_t* p = c + s * NK;
+    if (nvalid == SEG) {
+        uint32_t w[NK < 2 ? 1 : NK / 2];
+        if constexpr (NK == 1) {
+            w[0] = *p;
+        } else if constexpr (NK == 2) {
+            w[0] = *reinterpret_cast<const uint32_t*>(p);
+        } else if constexpr (NK == 4) {
+            uint2 v = *reinterpret_cast<const uint2*>(p);
+            w[0] = v.x; w[1] = v.y;
+        } else {
+#pragma unroll
+            for (int k = 0; k < NK / 8; ++k) {
+                uint4 v = reinterpret_cast<const uint4*>(p)[k];
+                w[4 * k] = v.x; w[4 * k + 1] = v.y; w[4 * k + 2] = v.z; w[4 * k + 3] = v.w;
+            }
+        }
+        if constexpr (NK == 1) {
+            ck[0] = __half2float(__ushort_as_half((unsigned short)w[0]));
+        } else {
+#pragma unroll
+            for (int k = 0; k < NK / 2; ++k) {
+                float2 f = h2_to_f2(w[k]);
+                ck[2 * k] = f.x;
+                ck[2 * k + 1] = f.y;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NK; ++k)
+            ck[k] = (k * sub < nvalid) ? __half2float(__ushort_as_half(p[k])) : 1.0f;
+    }
+}
+
+// W_hat = S_dq * Q(W / (S_dq * c_k)), S_dq the format's abs-max block scale.
+template <int B, int SUB, bool MX>
+__global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
+{
+    constexpr int NB = SEG / B;
+    constexpr int NK = SEG / SUB;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    float sg = 1.0f;
+    if constexpr (!MX) {
+        sg = global_scale_of(*a.amax);
+        if (a.sg_out != nullptr && s == 0)
+            *a.sg_out = sg;
+    }
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    float y[SEG], ck[NK];
+    load_seg_bf16(a.w, a.n, s, y);
+    load_coeffs<NK>(a.c, s, nvalid, SUB, ck);
+
+    float amax[NB], S[NB];
+    uint32_t sc[NB];
+    bool zb[NB];
+    block_amax<B>(y, amax);
+    const float den6 = __fmul_rn(6.0f, sg);
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        if constexpr (MX) {
+            const int e = e8m0_exp(amax[b]);
+            sc[b] = (uint32_t)(e + 127);
+            S[b] = pow2f(e);
+        } else {
+            sc[b] = e4m3_enc(__fdiv_rn(amax[b], den6));
+            S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
+        }
+        zb[b] = (S[b] == 0.0f);
+    }
+    float r[NK];
+    bool zk[NK];
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+        const int b = (k * SUB) / B;
+        zk[k] = zb[b];
+        r[k] = zb[b] ? 0.0f : guarded_rcp(__fmul_rn(S[b], ck[k]));
+    }
+    uint32_t q[4];
+    encode_seg<SUB>(y, r, zk, q);
+    float yh[SEG];
+    decode_seg<B>(q, S, yh);
+    store_seg_values(a.w_hat, a.out_kind, s, nvalid, yh);
+    if (a.codes != nullptr) {
+        if (nvalid == SEG) {
+            *reinterpret_cast<uint4*>(a.codes + s * (SEG / 2)) = make_uint4(q[0], q[1], q[2], q[3]);
+            store_bytes<NB>(a.scales + s * NB, sc);
+        } else {
+#pragma unroll
+            for (int i = 0; i < SEG / 2; ++i)
+                if (2 * i < nvalid)
+                    a.codes[s * (SEG / 2) + i] = (uint8_t)(q[i / 4] >> (8 * (i % 4)));
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+                if (b * B < nvalid)
+                    a.scales[s * NB + b] = (uint8_t)sc[b];
+        }
+    }
+}
+
+template <int B, int SUB, bool MX>
+static bool try_ffwd(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st)
+{
+    if constexpr (SUB <= B) {
+        if (sub == SUB) {
+            focus_fwd_kernel<B, SUB, MX><<<g, ATHREADS, 0, st>>>(a);
+            return true;
+        }
+    }
+    return false;
+}
+
+template <int B, bool MX>
+static cudaError_t launch_ffwd_sub(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st)
+{
+    if (try_ffwd<B, 2, MX>(sub, g, a, st) || try_ffwd<B, 4, MX>(sub, g, a, st) ||
+        try_ffwd<B, 8, MX>(sub, g, a, st) || try_ffwd<B, 16, MX>(sub, g, a, st) ||
+        try_ffwd<B, 32, MX>(sub, g, a, st))
+        return cudaGetLastError();
+    return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    if (!grid_ok(nseg) || sub > block)
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    if (mx)
+        return block == 32 ? launch_ffwd_sub<32, true>(sub, g, a, st) : cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_ffwd_sub<4, false>(sub, g, a, st);
+    case 8: return launch_ffwd_sub<8, false>(sub, g, a, st);
+    case 16: return launch_ffwd_sub<16, false>(sub, g, a, st);
+    case 32: return launch_ffwd_sub<32, false>(sub, g, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+// dL/dc_k = -(tree_sum over sub-block k of g * W) / (c_k * c_k).
+template <int SUB>
+__global__ void __launch_bounds__(ATHREADS) focus_bwd_kernel(FocusBwdArgs a)
+{
+    constexpr int NK = SEG / SUB;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    float w[SEG], g[SEG], ck[NK], dc[NK];
+    load_seg_bf16(a.w, a.n, s, w);
+    load_seg_bf16(a.g, a.n, s, g);
+    load_coeffs<NK>(a.c, s, nvalid, SUB, ck);
+#pragma unroll
+    for (int i = 0; i < SEG; ++i)
+        w[i] = __fmul_rn(g[i], w[i]);
+#pragma unroll
+    for (int k = 0; k < NK; ++k) {
+        const float acc = tree_sum<SUB>(w + k * SUB);
+        const float cc = __fmul_rn(ck[k], ck[k]);
+        dc[k] = -__fdiv_rn(acc, cc);
+    }
+    store_seg_floats<NK>(a.dc, s, nvalid, SUB, dc);
+}
+
+cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    if (!grid_ok(nseg))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    switch (sub) {
+    case 2: focus_bwd_kernel<2><<<g, ATHREADS, 0, st>>>(a); break;
+    case 4: focus_bwd_kernel<4><<<g, ATHREADS, 0, st>>>(a); break;
+    case 8: focus_bwd_kernel<8><<<g, ATHREADS, 0, st>>>(a); break;
+    case 16: focus_bwd_kernel<16><<<g, ATHREADS, 0, st>>>(a); break;
+    case 32: focus_bwd_kernel<32><<<g, ATHREADS, 0, st>>>(a); break;
+    default: return cudaErrorInvalidValue;
+    }
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ primitives
+
+__global__ void e2m1_encode_kernel(const float* u, int64_t n, uint8_t* out)
+{
+    const int64_t i = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (i >= n)
+        return;
+    float t[4] = {u[i], 0.0f, 0.0f, 0.0f};
+    out[i] = (uint8_t)(e2m1_pack4(t) & 0xFu);
+}
+
+__global__ void e4m3_encode_kernel(const float* v, int64_t n, uint8_t* out)
+{
+    const int64_t i = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (i >= n)
+        return;
+    out[i] = (uint8_t)e4m3_enc(v[i]);
+}
+
+cudaError_t launch_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t st)
+{
+    if (!grid_ok(n))
+        return cudaErrorInvalidValue;
+    e2m1_encode_kernel<<<grid_for(n), ATHREADS, 0, st>>>(u, n, out);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t st)
+{
+    if (!grid_ok(n))
+        return cudaErrorInvalidValue;
+    e4m3_encode_kernel<<<grid_for(n), ATHREADS, 0, st>>>(v, n, out);
+    return cudaGetLastError();
+}
+
+}  // namespace fp4q

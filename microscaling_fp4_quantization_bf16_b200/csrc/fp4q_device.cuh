@@ -1,0 +1,469 @@
+// fp4q_device.cuh -- device primitives shared by the sm_100a kernels.
+//
+// Every floating-point step is an explicit round-to-nearest-even IEEE
+// binary32 operation (__fadd_rn, __fmul_rn, __fdiv_rn, __frcp_rn: never
+// contracted into FMA) or a hardware conversion instruction (cvt with .rn and
+// .satfinite), so a kernel's result is a fixed function of its input:
+//  - E2M1 encode: cvt.rn.satfinite.e2m1x2.f32 (RNE, ties to the even
+//    mantissa, saturating at +-6, sign kept);
+//  - E2M1 decode: cvt.rn.f16x2.e2m1x2 then f16 -> f32 (both exact);
+//  - E4M3 encode: cvt.rn.satfinite.e4m3x2.f32 (RNE, saturating at 448);
+//  - E4M3 decode: cvt.rn.f16x2.e4m3x2 then f16 -> f32 (exact).
+// Formats: OCP E2M1 / E4M3 ("Finer is Better (with the Right Scaling)",
+// 手法 1 and 意義と主張), E8M0 ("Bridging the Gap Between Promise and
+// Performance for Microscaling FP4 Quantization", 技術概要 §1).
+#pragma once
+
+#include <cfloat>
+#include <cstdint>
+#include <type_traits>
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+namespace fp4q {
+
+// Elements owned by one thread: 32 contiguous elements of the flattened
+// tensor (64 bytes of bf16 = four 128-bit loads). Blocks (4..32) and Hadamard
+// chunks (16, 32) lie inside a segment; 64/128-wide chunks span 2/4 lanes.
+constexpr int SEG = 32;
+
+// Calls f(std::integral_constant<int, i>{}) for i = 0 .. N-1, so that i is a
+// compile-time constant inside f (register arrays stay in registers).
+template <int N, int I = 0, class F>
+__device__ __forceinline__ void static_for(F&& f)
+{
+    if constexpr (I < N) {
+        f(std::integral_constant<int, I>{});
+        static_for<N, I + 1>(f);
+    }
+}
+
+// ------------------------------------------------------------------ loads
+
+__device__ __forceinline__ uint4 ldg_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Loads segment s (elements s*32 .. s*32+31) of a bf16 array of n elements,
+// widened to fp32 (exact). Elements at or beyond n read as +0.
+__device__ __forceinline__ void load_seg_bf16(const uint16_t* x, int64_t n, int64_t s, float (&y)[SEG])
+{
+    const int64_t base = s * SEG;
+    if (base + SEG <= n) {
+        const uint4* p = reinterpret_cast<const uint4*>(x + base);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint4 v = ldg_stream(p + k);
+            y[8 * k + 0] = bf_lo(v.x);
+            y[8 * k + 1] = bf_hi(v.x);
+            y[8 * k + 2] = bf_lo(v.y);
+            y[8 * k + 3] = bf_hi(v.y);
+            y[8 * k + 4] = bf_lo(v.z);
+            y[8 * k + 5] = bf_hi(v.z);
+            y[8 * k + 6] = bf_lo(v.w);
+            y[8 * k + 7] = bf_hi(v.w);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < SEG; ++i)
+            y[i] = (base + i < n) ? __uint_as_float((uint32_t)x[base + i] << 16) : 0.0f;
+    }
+}
+
+// ------------------------------------------------------------------ E2M1
+
+// u[0..7] -> eight 4-bit codes; element j in bits 4j..4j+3. In
+// cvt.rn.satfinite.e2m1x2.f32 d, a, b the first source a lands in the upper
+// nibble, so element 2j+1 is passed first.
+__device__ __forceinline__ uint32_t e2m1_pack8(const float* u)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+        "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+        : "=r"(r)
+        : "f"(u[0]), "f"(u[1]), "f"(u[2]), "f"(u[3]), "f"(u[4]), "f"(u[5]), "f"(u[6]), "f"(u[7]));
+    return r;
+}
+
+// u[0..3] -> four 4-bit codes in bits 0..15 (element j in bits 4j..4j+3).
+__device__ __forceinline__ uint32_t e2m1_pack4(const float* u)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q0, q1;\n\t.reg .b16 t;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+        "mov.b16 t, {q0, q1};\n\t"
+        "cvt.u32.u16 %0, t;\n\t}"
+        : "=r"(r)
+        : "f"(u[0]), "f"(u[1]), "f"(u[2]), "f"(u[3]));
+    return r;
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t h)
+{
+    __half2 hh = *reinterpret_cast<__half2*>(&h);
+    return __half22float2(hh);
+}
+
+// Eight 4-bit codes (element j in bits 4j..4j+3) -> their exact values.
+__device__ __forceinline__ void e2m1_unpack8(uint32_t q, float* v)
+{
+    uint32_t h0, h1, h2, h3;
+    asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+        "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+        : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
+        : "r"(q));
+    float2 f;
+    f = h2_to_f2(h0); v[0] = f.x; v[1] = f.y;
+    f = h2_to_f2(h1); v[2] = f.x; v[3] = f.y;
+    f = h2_to_f2(h2); v[4] = f.x; v[5] = f.y;
+    f = h2_to_f2(h3); v[6] = f.x; v[7] = f.y;
+}
+
+// Four 4-bit codes in bits 0..15 -> their exact values.
+__device__ __forceinline__ void e2m1_unpack4(uint32_t q, float* v)
+{
+    uint32_t h0, h1;
+    unsigned short t = (unsigned short)(q & 0xFFFFu);
+    asm("{\n\t.reg .b8 q0, q1;\n\t"
+        "mov.b16 {q0, q1}, %2;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t}"
+        : "=r"(h0), "=r"(h1)
+        : "h"(t));
+    float2 f;
+    f = h2_to_f2(h0); v[0] = f.x; v[1] = f.y;
+    f = h2_to_f2(h1); v[2] = f.x; v[3] = f.y;
+}
+
+// ------------------------------------------------------------------ E4M3
+
+// Two non-negative floats -> two E4M3 bytes: lo in bits 0-7, hi in bits 8-15.
+__device__ __forceinline__ uint32_t e4m3_enc2(float hi, float lo)
+{
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t e4m3_enc(float v) { return e4m3_enc2(0.0f, v) & 0xFFu; }
+
+// E4M3 byte (0..0x7E) -> exact value.
+__device__ __forceinline__ float e4m3_dec(uint32_t code)
+{
+    uint32_t h;
+    unsigned short c = (unsigned short)(code & 0xFFu);
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(c));
+    return h2_to_f2(h).x;
+}
+
+// ------------------------------------------------------------------ scales
+
+// FP32 global scale of hierarchical scaling: amax / (448 * 6); 1 when that is
+// not a positive finite number.
+__device__ __forceinline__ float global_scale_of(float g)
+{
+    float sg = __fdiv_rn(g, 2688.0f);
+    if (!(sg > 0.0f) || !(g <= FLT_MAX))
+        sg = 1.0f;
+    return sg;
+}
+
+// 1 / S, with an overflowing reciprocal replaced by the largest finite float
+// of the same sign.
+__device__ __forceinline__ float guarded_rcp(float S)
+{
+    float r = __frcp_rn(S);
+    if (fabsf(r) > FLT_MAX)
+        r = copysignf(FLT_MAX, r);
+    return r;
+}
+
+// E8M0 exponent of a block abs-max a >= 0: floor(log2 a) - 2 clamped to
+// [-127, 127] (a == 0 -> -127). For a biased fp32 exponent E (0 for zero and
+// subnormals) this is max(E - 129, -127): subnormal a has floor(log2 a) <= -127.
+__device__ __forceinline__ int e8m0_exp(float a)
+{
+    int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);
+    return max(E - 129, -127);
+}
+
+// 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00200000).
+__device__ __forceinline__ float pow2f(int e)
+{
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00200000u);
+}
+
+// ------------------------------------------------------------------ Hadamard
+
+template <int N>
+struct HadK;
+template <> struct HadK<16> { static constexpr float k = 0x1p-2f; };
+template <> struct HadK<32> { static constexpr float k = 0x1.6a09e6p-3f; };
+template <> struct HadK<64> { static constexpr float k = 0x1p-3f; };
+template <> struct HadK<128> { static constexpr float k = 0x1.6a09e6p-4f; };
+
+// Normalised Walsh-Hadamard transform of every ROT-wide chunk, stages in
+// ascending order h = 1, 2, 4, ...: butterflies with h < 32 stay inside the
+// segment; h = 32 and 64 pair lane L with lane L ^ (h / 32) (the lower lane
+// holds index i, the upper lane index i + h). All 32 lanes of the warp must
+// call this together.
+template <int ROT>
+__device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
+{
+    if constexpr (ROT > 0) {
+        constexpr int LOCAL = ROT < SEG ? ROT : SEG;
+#pragma unroll
+        for (int h = 1; h < LOCAL; h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) {
+                if ((i & h) == 0) {
+                    float a = y[i], b = y[i + h];
+                    y[i] = __fadd_rn(a, b);
+                    y[i + h] = __fsub_rn(a, b);
+                }
+            }
+        }
+#pragma unroll
+        for (int h = SEG; h < ROT; h <<= 1) {
+            const int lm = h / SEG;
+            const bool lower = (lane & lm) == 0;
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) {
+                float p = __shfl_xor_sync(0xFFFFFFFFu, y[i], lm);
+                y[i] = lower ? __fadd_rn(y[i], p) : __fsub_rn(p, y[i]);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < SEG; ++i)
+            y[i] = __fmul_rn(y[i], HadK<ROT>::k);
+    }
+}
+
+// ------------------------------------------------------------------ blocks
+
+// Abs-max of each B-wide block of the segment (exact: max is order-free).
+template <int B>
+__device__ __forceinline__ void block_amax(const float (&y)[SEG], float (&a)[SEG / B])
+{
+#pragma unroll
+    for (int b = 0; b < SEG / B; ++b) {
+        float m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < B; ++j)
+            m = fmaxf(m, fabsf(y[b * B + j]));
+        a[b] = m;
+    }
+}
+
+// Adjacent-pair tree sum of e[off .. off+B): for h = 1, 2, .., B/2,
+// e[i] += e[i + h] for i = off, off + 2h, ...
+template <int B>
+__device__ __forceinline__ float tree_sum(float* e)
+{
+#pragma unroll
+    for (int h = 1; h < B; h <<= 1) {
+#pragma unroll
+        for (int i = 0; i + h < B; i += 2 * h)
+            e[i] = __fadd_rn(e[i], e[i + h]);
+    }
+    return e[0];
+}
+
+// Codes of the segment: u = y * r(block), RNE to E2M1, eight per word; the
+// codes of blocks with a zero scale are forced to 0x0.
+template <int B>
+__device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&r)[SEG / B],
+                                           const bool (&zero)[SEG / B], uint32_t (&q)[4])
+{
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        float u[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            u[j] = __fmul_rn(y[8 * w + j], r[(8 * w + j) / B]);
+        uint32_t qw = e2m1_pack8(u);
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (zero[(8 * w + j) / B])
+                m |= 0xFu << (4 * j);
+        q[w] = qw & ~m;
+    }
+}
+
+// Dequantized values of the segment: value(code) * S(block).
+template <int B>
+__device__ __forceinline__ void decode_seg(const uint32_t (&q)[4], const float (&S)[SEG / B],
+                                           float (&yh)[SEG])
+{
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        float v[8];
+        e2m1_unpack8(q[w], v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            yh[8 * w + j] = __fmul_rn(v[j], S[(8 * w + j) / B]);
+    }
+}
+
+// Per-block SSE of y against value(code) * S, tree-summed.
+template <int B>
+__device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&q)[4],
+                                        const float (&S)[SEG / B], float (&sse)[SEG / B])
+{
+    float e[SEG];
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        float v[8];
+        e2m1_unpack8(q[w], v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;
+            float yh = __fmul_rn(v[j], S[i / B]);
+            float d = __fsub_rn(y[i], yh);
+            e[i] = __fmul_rn(d, d);
+        }
+    }
+#pragma unroll
+    for (int b = 0; b < SEG / B; ++b)
+        sse[b] = tree_sum<B>(e + b * B);
+}
+
+// SSE of one B-wide block yb against value(RNE_E2M1(yb * r)) * S. The codes
+// of a zero scale need no masking here: u = y * 0 is a signed zero whose
+// value times S = 0 is a signed zero, and y - (+-0) == y.
+template <int B>
+__device__ __forceinline__ float block_sse(const float* yb, float r, float S)
+{
+    float e[B];
+    if constexpr (B >= 8) {
+#pragma unroll
+        for (int g = 0; g < B / 8; ++g) {
+            float u[8], v[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                u[j] = __fmul_rn(yb[8 * g + j], r);
+            e2m1_unpack8(e2m1_pack8(u), v);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                float d = __fsub_rn(yb[8 * g + j], __fmul_rn(v[j], S));
+                e[8 * g + j] = __fmul_rn(d, d);
+            }
+        }
+    } else {
+        float u[4], v[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            u[j] = __fmul_rn(yb[j], r);
+        e2m1_unpack4(e2m1_pack4(u), v);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            float d = __fsub_rn(yb[j], __fmul_rn(v[j], S));
+            e[j] = __fmul_rn(d, d);
+        }
+    }
+    return tree_sum<B>(e);
+}
+
+// ------------------------------------------------------------------ stores
+
+// NB = SEG / B bytes (one per block) at p (NB-byte aligned).
+template <int NB>
+__device__ __forceinline__ void store_bytes(uint8_t* p, const uint32_t (&v)[NB])
+{
+    if constexpr (NB == 1) {
+        *p = (uint8_t)v[0];
+    } else if constexpr (NB == 2) {
+        *reinterpret_cast<uint16_t*>(p) = (uint16_t)(v[0] | (v[1] << 8));
+    } else if constexpr (NB == 4) {
+        *reinterpret_cast<uint32_t*>(p) = v[0] | (v[1] << 8) | (v[2] << 16) | (v[3] << 24);
+    } else {
+        uint2 w;
+        w.x = v[0] | (v[1] << 8) | (v[2] << 16) | (v[3] << 24);
+        w.y = v[4] | (v[5] << 8) | (v[6] << 16) | (v[7] << 24);
+        *reinterpret_cast<uint2*>(p) = w;
+    }
+}
+
+template <int NB>
+__device__ __forceinline__ void store_floats(float* p, const float (&v)[NB])
+{
+    if constexpr (NB == 1) {
+        *p = v[0];
+    } else if constexpr (NB == 2) {
+        *reinterpret_cast<float2*>(p) = make_float2(v[0], v[1]);
+    } else if constexpr (NB == 4) {
+        *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
+        reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+        reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+    }
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
+{
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);  // RNE, lo in the low half
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// Writes the 32 values of segment s as fp32 (kind 1) or bf16 (kind 2);
+// only the first nvalid elements when the segment is partial.
+__device__ __forceinline__ void store_seg_values(void* out, int kind, int64_t s, int nvalid,
+                                                 const float (&v)[SEG])
+{
+    if (kind == 1) {
+        float* o = reinterpret_cast<float*>(out) + s * SEG;
+        if (nvalid == SEG) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k)
+                reinterpret_cast<float4*>(o)[k] =
+                    make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < SEG; ++i)
+                if (i < nvalid)
+                    o[i] = v[i];
+        }
+    } else if (kind == 2) {
+        uint16_t* o = reinterpret_cast<uint16_t*>(out) + s * SEG;
+        if (nvalid == SEG) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                uint4 w;
+                w.x = pack_bf16x2(v[8 * k + 0], v[8 * k + 1]);
+                w.y = pack_bf16x2(v[8 * k + 2], v[8 * k + 3]);
+                w.z = pack_bf16x2(v[8 * k + 4], v[8 * k + 5]);
+                w.w = pack_bf16x2(v[8 * k + 6], v[8 * k + 7]);
+                reinterpret_cast<uint4*>(o)[k] = w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < SEG; ++i) {
+                if (i < nvalid) {
+                    __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
+                    o[i] = *reinterpret_cast<uint16_t*>(&h);
+                }
+            }
+        }
+    }
+}
+
+}  // namespace fp4q

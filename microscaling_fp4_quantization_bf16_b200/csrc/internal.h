@@ -1,0 +1,82 @@
+// internal.h -- argument blocks and launcher declarations shared between the
+// C-ABI layer (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime_api.h>
+
+namespace fp4q {
+
+// Strategy ids used by the kernels (NVFP4 strategies follow the ABI enum;
+// MXFP4 abs-max is its own kernel family).
+enum KStrat { K_ABSMAX = 0, K_PREVENT_ZERO = 1, K_FOUR_OVER_SIX = 2, K_BRUTE_FORCE = 3, K_MX = 4 };
+
+struct QuantArgs {
+    const uint16_t* x;      // bf16 [n]
+    int64_t n;              // elements (rows * cols)
+    const float* amax;      // NVFP4: device tensor abs-max; NULL for MXFP4
+    float* sg_out;          // NVFP4: receives s_g from thread 0 of block 0, or NULL
+    uint8_t* codes;         // [n / 2]
+    uint8_t* scales;        // [n / B]
+    float* mse;             // [n / B] or NULL
+    void* dq;               // [n] or NULL
+    int dq_kind;            // 0 none, 1 fp32, 2 bf16
+};
+
+struct DequantArgs {
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* sg;        // NVFP4 global scale (device), NULL for MXFP4
+    int64_t n;
+    void* out;
+    int out_kind;           // 1 fp32, 2 bf16
+};
+
+struct MseArgs {
+    const uint16_t* x;
+    const uint8_t* codes;
+    const uint8_t* scales;
+    const float* sg;
+    int64_t n;
+    float* mse;
+};
+
+struct FocusFwdArgs {
+    const uint16_t* w;      // bf16 [n]
+    const uint16_t* c;      // fp16 [n / sub]
+    int64_t n;
+    const float* amax;      // NVFP4 tensor abs-max (device)
+    float* sg_out;
+    void* w_hat;
+    int out_kind;           // 1 fp32, 2 bf16
+    uint8_t* codes;         // optional
+    uint8_t* scales;        // optional
+};
+
+struct FocusBwdArgs {
+    const uint16_t* w;
+    const uint16_t* g;
+    const uint16_t* c;
+    int64_t n;
+    float* dc;
+};
+
+// Each launcher returns cudaErrorInvalidValue for a combination it does not
+// provide (the ABI layer validates before calling), else the launch status.
+cudaError_t launch_quant_b4(int strat, int rot, const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_quant_b8(int strat, int rot, const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_quant_b16(int strat, int rot, const QuantArgs& a, cudaStream_t st);
+cudaError_t launch_quant_b32(int strat, int rot, const QuantArgs& a, cudaStream_t st);
+
+cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st);
+cudaError_t launch_finalize_sg(float* g, cudaStream_t st);
+cudaError_t launch_set_one(float* p, cudaStream_t st);
+cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st);
+cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st);
+cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
+cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);
+cudaError_t launch_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t st);
+cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
+
+}  // namespace fp4q

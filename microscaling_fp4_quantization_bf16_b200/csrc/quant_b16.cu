@@ -1,0 +1,9 @@
+// quant_b16.cu -- instantiations of the quantize kernel for block size 16.
+#include "quant_kernel.cuh"
+
+namespace fp4q {
+cudaError_t launch_quant_b16(int strat, int rot, const QuantArgs& a, cudaStream_t st)
+{
+    return launch_quant_impl<16>(strat, rot, a, st);
+}
+}  // namespace fp4q

@@ -1,0 +1,216 @@
+// quant_kernel.cuh -- the fused rotate -> scale -> encode -> pack kernel.
+//
+// One thread owns one 32-element segment of the flattened tensor (blocks and
+// rotation chunks never straddle rows because cols is a multiple of both).
+// The segment is read once with four 128-bit loads, rotated in registers,
+// scaled, encoded and packed; the 16 code bytes leave in one 128-bit store.
+//
+// Scale selection ("Finer is Better (with the Right Scaling)", 手法 2):
+//   abs-max      c = RNE_E4M3(amax / (6 s_g))
+//   prevent-zero c = max(abs-max code, 0x01)
+//   4-over-6     targets 6 and 4; target 4 is kept only if its block SSE is
+//                strictly lower
+//   brute force  every code 0x01..0x7E, strictly lower SSE wins (ties keep
+//                the lower code)
+// MXFP4 ("Bridging the Gap ...", 技術概要 §1): S = 2^(floor(log2 amax) - 2).
+#pragma once
+
+#include "fp4q_device.cuh"
+#include "internal.h"
+
+namespace fp4q {
+
+constexpr int QTHREADS = 256;
+
+template <int B, int ROT, int STRAT>
+__global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
+{
+    constexpr int NB = SEG / B;
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
+
+    float sg = 1.0f;
+    if constexpr (STRAT != K_MX) {
+        sg = global_scale_of(*a.amax);
+        if (a.sg_out != nullptr && s == 0)
+            *a.sg_out = sg;
+    }
+
+    // Brute force: dequantization scale and reciprocal of every E4M3 code,
+    // shared by the block.
+    __shared__ float tS[STRAT == K_BRUTE_FORCE ? 128 : 1];
+    __shared__ float tR[STRAT == K_BRUTE_FORCE ? 128 : 1];
+    if constexpr (STRAT == K_BRUTE_FORCE) {
+        for (int c = threadIdx.x; c < 128; c += QTHREADS) {
+            float S = (c >= 1 && c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
+            tS[c] = S;
+            tR[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
+        }
+        __syncthreads();
+    }
+
+    if (s - lane >= nseg)
+        return;  // the whole warp is past the end (warp-uniform)
+
+    float y[SEG];
+    load_seg_bf16(a.x, a.n, s, y);  // lanes past the end read zeros
+    rotate_seg<ROT>(y, lane);       // all 32 lanes take part
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+
+    float amax[NB];
+    block_amax<B>(y, amax);
+
+    float S[NB], r[NB], sse[NB];
+    bool zero[NB];
+    uint32_t sc[NB], q[4];
+    bool have_sse = false;
+
+    if constexpr (STRAT == K_MX) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const int e = e8m0_exp(amax[b]);
+            sc[b] = (uint32_t)(e + 127);
+            S[b] = pow2f(e);
+            r[b] = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
+            zero[b] = false;
+        }
+        encode_seg<B>(y, r, zero, q);
+    } else if constexpr (STRAT == K_BRUTE_FORCE) {
+        static_for<NB>([&](auto bi) {
+            constexpr int b = decltype(bi)::value;
+            float best = 0.0f;
+            int bc = 1;
+#pragma unroll 1
+            for (int c = 1; c <= 0x7E; ++c) {
+                const float v = block_sse<B>(y + b * B, tR[c], tS[c]);
+                if (c == 1 || v < best) {
+                    best = v;
+                    bc = c;
+                }
+            }
+            sc[b] = (uint32_t)bc;
+            S[b] = tS[bc];
+            r[b] = tR[bc];
+            zero[b] = (S[b] == 0.0f);
+            sse[b] = best;
+        });
+        encode_seg<B>(y, r, zero, q);
+        have_sse = true;
+    } else {
+        const float den6 = __fmul_rn(6.0f, sg);
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            uint32_t c = e4m3_enc(__fdiv_rn(amax[b], den6));
+            if constexpr (STRAT == K_PREVENT_ZERO)
+                c = max(c, 1u);
+            sc[b] = c;
+            S[b] = __fmul_rn(e4m3_dec(c), sg);
+            zero[b] = (S[b] == 0.0f);
+            r[b] = zero[b] ? 0.0f : guarded_rcp(S[b]);
+        }
+        encode_seg<B>(y, r, zero, q);
+        if constexpr (STRAT == K_FOUR_OVER_SIX) {
+            const float den4 = __fmul_rn(4.0f, sg);
+            float S4[NB], r4[NB], sse4[NB];
+            bool z4[NB];
+            uint32_t c4[NB], q4[4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                c4[b] = e4m3_enc(__fdiv_rn(amax[b], den4));
+                S4[b] = __fmul_rn(e4m3_dec(c4[b]), sg);
+                z4[b] = (S4[b] == 0.0f);
+                r4[b] = z4[b] ? 0.0f : guarded_rcp(S4[b]);
+            }
+            encode_seg<B>(y, r4, z4, q4);
+            sse_seg<B>(y, q, S, sse);
+            sse_seg<B>(y, q4, S4, sse4);
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+                uint32_t m = 0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    if (sse4[(8 * w + j) / B] < sse[(8 * w + j) / B])
+                        m |= 0xFu << (4 * j);
+                q[w] = (q[w] & ~m) | (q4[w] & m);
+            }
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                if (sse4[b] < sse[b]) {
+                    sc[b] = c4[b];
+                    S[b] = S4[b];
+                    sse[b] = sse4[b];
+                }
+            }
+            have_sse = true;
+        }
+    }
+
+    if (a.mse != nullptr && !have_sse)
+        sse_seg<B>(y, q, S, sse);
+
+    float m[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        m[b] = __fmul_rn(sse[b], 1.0f / B);  // exact power-of-two division
+
+    if (nvalid == SEG) {
+        *reinterpret_cast<uint4*>(a.codes + s * (SEG / 2)) = make_uint4(q[0], q[1], q[2], q[3]);
+        store_bytes<NB>(a.scales + s * NB, sc);
+        if (a.mse != nullptr)
+            store_floats<NB>(a.mse + s * NB, m);
+    } else {
+#pragma unroll
+        for (int i = 0; i < SEG / 2; ++i)
+            if (2 * i < nvalid)
+                a.codes[s * (SEG / 2) + i] = (uint8_t)(q[i / 4] >> (8 * (i % 4)));
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            if (b * B < nvalid) {
+                a.scales[s * NB + b] = (uint8_t)sc[b];
+                if (a.mse != nullptr)
+                    a.mse[s * NB + b] = m[b];
+            }
+        }
+    }
+    if (a.dq_kind != 0) {
+        float yh[SEG];
+        decode_seg<B>(q, S, yh);
+        store_seg_values(a.dq, a.dq_kind, s, nvalid, yh);
+    }
+}
+
+template <int B>
+cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t nblk = (nseg + QTHREADS - 1) / QTHREADS;
+    if (nblk <= 0 || nblk > 0x7FFFFFFF)
+        return cudaErrorInvalidValue;
+    const dim3 grid((unsigned)nblk);
+#define FP4Q_QCASE(S_, R_)                                        \
+    if (strat == S_ && rot == R_) {                               \
+        quant_kernel<B, R_, S_><<<grid, QTHREADS, 0, st>>>(a);    \
+        return cudaGetLastError();                                \
+    }
+#define FP4Q_QROTS(S_)      \
+    FP4Q_QCASE(S_, 0)       \
+    FP4Q_QCASE(S_, 16)      \
+    FP4Q_QCASE(S_, 32)      \
+    FP4Q_QCASE(S_, 64)      \
+    FP4Q_QCASE(S_, 128)
+    FP4Q_QROTS(K_ABSMAX)
+    FP4Q_QROTS(K_PREVENT_ZERO)
+    FP4Q_QROTS(K_FOUR_OVER_SIX)
+    FP4Q_QROTS(K_BRUTE_FORCE)
+    if constexpr (B == 32) {
+        FP4Q_QROTS(K_MX)
+    }
+#undef FP4Q_QROTS
+#undef FP4Q_QCASE
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace fp4q

@@ -1,0 +1,142 @@
+"""The C-ABI library loads, exports every entry point declared in
+include/fp4q.h, and rejects invalid arguments on the host before anything is
+launched (so these run without a GPU).
+
+Every call below has at least one invalid argument: the fake addresses are
+never dereferenced because validation fails first.
+"""
+import ctypes as C
+import os
+import re
+
+import pytest
+
+from microscaling_fp4_quantization_bf16_b200 import _abi, build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fp4q.h")
+
+OK, NULL, SHAPE, ALIGN, UNSUP, ALIAS, CUDA = range(7)
+A = 0x100000     # a 16-byte-aligned fake device address
+A2 = 0x200000
+A3 = 0x300000
+MIS = 0x100004   # 4-byte but not 16-byte aligned
+NV, MX = 0, 1
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return _abi.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp4q_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_and_library_agree(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in fp4q.h but not exported"
+        assert n in _abi.SIGNATURES, f"{n} has no ctypes signature"
+    assert sorted(_abi.SIGNATURES) == names
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.fp4q_status_string(s)
+    assert lib.fp4q_status_string(99) == b"unknown status"
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="missing"):
+        _abi._lib_saved = _abi._lib
+        try:
+            _abi._lib = None
+            _abi.load(str(tmp_path / "nope.so"))
+        finally:
+            _abi._lib = _abi._lib_saved
+
+
+def q(lib, x=A, rows=4, cols=64, fmt=NV, block=16, strat=0, rot=0, gin=None, gout=A3 + 64,
+      codes=A2, scales=A3, mse=None, dq=None, dqt=0):
+    return lib.fp4q_quantize(x, rows, cols, fmt, block, strat, rot, gin, gout, codes, scales, mse,
+                             dq, dqt, None)
+
+
+def test_quantize_validation(lib):
+    assert q(lib, x=None) == NULL
+    assert q(lib, codes=None) == NULL
+    assert q(lib, scales=None) == NULL
+    assert q(lib, gout=None) == NULL                  # NVFP4 needs the global scale output
+    assert q(lib, cols=24) == SHAPE                   # 24 % 16
+    assert q(lib, rows=-1) == SHAPE
+    assert q(lib, cols=-16) == SHAPE
+    assert q(lib, rot=32, cols=48) == SHAPE           # 48 % 32
+    assert q(lib, rows=1 << 30, cols=1 << 14) == SHAPE  # beyond 2^40 elements
+    assert q(lib, x=MIS) == ALIGN
+    assert q(lib, codes=MIS) == ALIGN
+    assert q(lib, mse=MIS) == ALIGN
+    assert q(lib, dq=MIS) == ALIGN
+    assert q(lib, gout=A3 + 66) == ALIGN
+    assert q(lib, fmt=MX, block=32, strat=2, gout=None) == UNSUP
+    assert q(lib, fmt=MX, block=16, gout=None) == UNSUP
+    assert q(lib, block=64) == UNSUP
+    assert q(lib, block=2) == UNSUP
+    assert q(lib, rot=8) == UNSUP
+    assert q(lib, strat=4) == UNSUP
+    assert q(lib, fmt=2) == UNSUP
+    assert q(lib, dq=A, dqt=5) == UNSUP
+    assert q(lib, gin=A3 + 64, gout=A3 + 64) == ALIAS
+
+
+def test_other_entry_points_validation(lib):
+    L = lib
+    assert L.fp4q_dequantize(None, A, A, 4, 64, NV, 16, A, 0, None) == NULL
+    assert L.fp4q_dequantize(A, A, None, 4, 64, NV, 16, A, 0, None) == NULL
+    assert L.fp4q_dequantize(A, A, A, 4, 60, NV, 16, A, 0, None) == SHAPE
+    assert L.fp4q_dequantize(A, MIS, A, 4, 64, NV, 16, A, 0, None) == ALIGN
+    assert L.fp4q_dequantize(A, A, A, 4, 64, NV, 16, A, 3, None) == UNSUP
+    assert L.fp4q_block_mse(A, A, A, A, 4, 64, NV, 16, 0, None, None) == NULL
+    assert L.fp4q_block_mse(A, A, A, A, 4, 64, NV, 16, 128, A, None) == SHAPE
+    assert L.fp4q_block_mse(A, A, A, MIS + 2, 4, 64, NV, 16, 0, A, None) == ALIGN
+    # focus forward
+    ff = lambda **k: L.fp4q_focus_fwd(k.get("w", A), k.get("c", A), 4, k.get("cols", 64),
+                                      k.get("fmt", NV), k.get("block", 16), k.get("sub", 8),
+                                      k.get("gin"), k.get("gout", A3), k.get("wh", A2),
+                                      k.get("ot", 1), k.get("codes"), k.get("scales"), None)
+    assert ff(sub=32) == UNSUP      # sub > block
+    assert ff(sub=3) == UNSUP
+    assert ff(sub=1) == UNSUP
+    assert ff(ot=9) == UNSUP
+    assert ff(codes=A) == NULL      # codes without scales
+    assert ff(c=None) == NULL
+    assert ff(w=MIS) == ALIGN
+    assert ff(cols=40) == SHAPE
+    assert ff(gin=A3, gout=A3) == ALIAS
+    # focus backward
+    assert L.fp4q_focus_bwd(A, A, A, 4, 60, 8, A, None) == SHAPE
+    assert L.fp4q_focus_bwd(A, A, A, 4, 64, 6, A, None) == UNSUP
+    assert L.fp4q_focus_bwd(A, None, A, 4, 64, 8, A, None) == NULL
+    assert L.fp4q_focus_bwd(A, A, A, 4, 64, 8, MIS, None) == ALIGN
+    # global amax, primitives
+    assert L.fp4q_global_amax(A, 4, 64, 24, A, None) == UNSUP
+    assert L.fp4q_global_amax(A, 4, 48, 32, A, None) == SHAPE
+    assert L.fp4q_global_amax(A, 4, 64, 0, A + 2, None) == ALIGN
+    assert L.fp4q_global_amax(None, 4, 64, 0, A, None) == NULL
+    assert L.fp4q_e2m1_encode(A, -1, A, None) == SHAPE
+    assert L.fp4q_e2m1_encode(MIS, 8, A, None) == ALIGN
+    assert L.fp4q_e4m3_encode(A, 8, None, None) == NULL
+
+
+def test_python_wrapper_rejects_cpu_tensors():
+    import torch
+    import microscaling_fp4_quantization_bf16_b200 as fp4q
+    with pytest.raises(ValueError, match="CUDA"):
+        fp4q.quantize(torch.zeros(4, 64, dtype=torch.bfloat16))
+    with pytest.raises(ValueError):
+        fp4q.focus_bwd(torch.zeros(4, 64, dtype=torch.bfloat16),
+                       torch.zeros(4, 64, dtype=torch.bfloat16), torch.zeros(4, 8))
