@@ -4,8 +4,9 @@
 Headline workload: MXFP4 (E8M0 scales, block 32) quantization of a
 4096 x 4096 bf16 weight drawn from Laplace(0, 0.02) with 0.1% of entries
 times 50, run without rotation and with a 32-wide blockwise Hadamard; one step
-= both runs. Inputs are resident in HBM; L2 is flushed (a 2 x L2 write)
-before every launch, outside the timed events. ``value`` is quantized
+= both runs. Inputs are resident in HBM and larger than L2: every launch
+reads its own copy of the tensor, rotating through enough copies that each
+is evicted before it is read again. ``value`` is quantized
 elements per second over the whole job (all ranks: independent replicas,
 weak scaling). One JSON line is printed by rank 0.
 
@@ -33,6 +34,13 @@ ROWS, COLS = 4096, 4096
 ROTS = (0, 32)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 SM_COUNT_NOMINAL, FP32_LANES_PER_SM, SM_MAX_MHZ_NOMINAL = 148, 128, 1965.0
+SLEEP_CYCLES = 100_000  # ~50 us of GPU spin before each timed launch (CPU enqueue cover)
+
+
+def copies_for(nbytes: int, l2: int, cap: int = 128) -> int:
+    """Copies of an input needed so that rotating through them moves more
+    than 2 x L2 of data before any copy is read again."""
+    return max(1, min(cap, -(-2 * l2 // max(1, nbytes)) + 1))
 
 
 def bytes_per_elem(block: int, codes=True, scales=True, mse=False, dq=0, extra_in=0.0):
@@ -162,26 +170,33 @@ def run_ours(args, rank, world, local_rank):
     fp4q.load()
     peaks = load_peaks()
     props = torch.cuda.get_device_properties(dev)
-    flush = torch.empty(2 * props.L2_cache_size // 4, dtype=torch.float32, device=dev)
+    l2 = props.L2_cache_size
 
-    x = synth.workload(WORKLOAD)["x"].to(dev)
-    n = x.numel()
-    outs = {r: fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
-                              torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
-                              None, None, None) for r in ROTS}
-    evs = {r: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for r in ROTS}
+    # Inputs larger than L2: every launch reads its own copy of x, and a copy
+    # comes round again only after more than 2 x L2 of other traffic.
+    x0 = synth.workload(WORKLOAD)["x"].to(dev)
+    n = x0.numel()
+    ncopy = copies_for(x0.numel() * 2, l2)
+    xs = [x0.clone() for _ in range(ncopy)]
+    outs = [fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
+                           torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
+                           None, None, None) for _ in range(ncopy)]
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in ROTS]
+    counter = [0]
 
     def step(times):
-        for r in ROTS:
-            flush.zero_()  # keeps the GPU busy while the launch is enqueued
-            s, e = evs[r]
+        for k, r in enumerate(ROTS):
+            j = counter[0] % ncopy
+            counter[0] += 1
+            torch.cuda._sleep(SLEEP_CYCLES)  # the GPU is busy while the launch is enqueued
+            s, e = evs[k]
             s.record()
-            fp4q.quantize(x, "mxfp4", 32, "absmax", r, out=outs[r])
+            fp4q.quantize(xs[j], "mxfp4", 32, "absmax", r, out=outs[j])
             e.record()
         torch.cuda.synchronize()
-        for r in ROTS:
-            times[r].append(evs[r][0].elapsed_time(evs[r][1]))
+        for k, r in enumerate(ROTS):
+            times[r].append(evs[k][0].elapsed_time(evs[k][1]))
 
     sampler = ClockSampler(local_rank)
     with sampler:
@@ -203,6 +218,7 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         t1 = time.perf_counter()
     clocks = sampler.summary(t0, t1)
+    x = xs[0]
 
     total_ms = sum(sum(v) for v in times.values())
     if world > 1:
@@ -270,7 +286,8 @@ def run_ours(args, rank, world, local_rank):
                                    "rot 0 + rot 32 (Hadamard) runs",
                        "rows": ROWS, "cols": COLS, "format": "mxfp4", "block": 32,
                        "rot": list(ROTS), "outputs": "packed codes + scale bytes",
-                       "l2": "flushed before every launch (2 x L2 write, outside the events)",
+                       "l2": f"inputs larger than L2: each launch reads its own copy of x "
+                             f"({ncopy} copies, {ncopy * n * 2 / 2**20:.0f} MiB in rotation)",
                        "parallelism": f"replicas x{world} (independent tensors, no collective)",
                        "soak_s": args.soak},
             "roofline": roofline, "e2e": e2e, "gpu_launches": len(ROTS) * args.steps,
@@ -279,7 +296,7 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
     if rank == 0 and world == 1 and not args.no_breakdown:
-        line["breakdown"] = breakdown(dev, flush, peaks)
+        line["breakdown"] = breakdown(dev, peaks)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -289,24 +306,26 @@ def run_ours(args, rank, world, local_rank):
 
 # ---------------------------------------------------------------- breakdown
 
-def breakdown(dev, flush, peaks, reps: int = 10):
+def breakdown(dev, peaks, reps: int = 10):
     """Every run of every workload, one line each: elements/s, algorithmic
-    GB/s and its fraction of the HBM roofline (FP32 ops for brute force)."""
+    GB/s and its fraction of the HBM roofline (FP32 ops for brute force).
+    Inputs rotate through copies so that every launch reads from HBM."""
     import torch
 
     import microscaling_fp4_quantization_bf16_b200 as fp4q
     from microscaling_fp4_quantization_bf16_b200 import synth
 
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     fp32_peak = SM_COUNT_NOMINAL * FP32_LANES_PER_SM * SM_MAX_MHZ_NOMINAL * 1e6
     rows_out = []
 
-    def timeit(fn, n_launch=1):
+    def timeit(fns):
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         ts = []
         for i in range(reps + 3):
-            flush.zero_()
+            torch.cuda._sleep(SLEEP_CYCLES)
             s.record()
-            fn()
+            fns[i % len(fns)]()
             e.record()
             torch.cuda.synchronize()
             if i >= 3:
@@ -328,33 +347,40 @@ def breakdown(dev, flush, peaks, reps: int = 10):
         rows_out.append(d)
 
     def quant_runs(wl, runs, want_mse=False, dq=None):
-        x = synth.workload(wl)["x"].to(dev)
-        n = x.numel()
-        R, C = x.shape
+        x0 = synth.workload(wl)["x"].to(dev)
+        n = x0.numel()
+        R, C = x0.shape
+        nc = copies_for(2 * n, l2, cap=min(128, reps + 3))
+        xs = [x0] + [x0.clone() for _ in range(nc - 1)]
         for fmt, block, strat, rot in runs:
             nv = fmt == "nvfp4"
-            out = fp4q.Quantized(
+            outs = [fp4q.Quantized(
                 torch.empty(R, C // 2, dtype=torch.uint8, device=dev),
                 torch.empty(R, C // block, dtype=torch.uint8, device=dev),
                 torch.empty(1, device=dev) if nv else None,
                 torch.empty(R, C // block, device=dev) if want_mse else None,
                 torch.empty(R, C, dtype=dq, device=dev) if dq is not None else None)
+                for _ in range(nc)]
             dqb = 0 if dq is None else torch.tensor([], dtype=dq).element_size()
             bpe = bytes_per_elem(block, mse=want_mse, dq=dqb)
             ops = n * 126 * 5 if strat == "brute_force" else None
             tag = f"{wl} {fmt} B{block} {strat} H{rot}"
             if nv:
-                ga = fp4q.global_amax(x, rot)
-                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, global_amax=ga,
-                                                    out=out))
+                ga = fp4q.global_amax(x0, rot)
+                secs = timeit([lambda i=i: fp4q.quantize(xs[i], fmt, block, strat, rot,
+                                                         global_amax=ga, out=outs[i])
+                               for i in range(nc)])
                 add(tag + " (abs-max supplied, 1 pass)", n, secs, bpe, 1, ops)
-                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, out=out))
+                secs = timeit([lambda i=i: fp4q.quantize(xs[i], fmt, block, strat, rot, out=outs[i])
+                               for i in range(nc)])
                 add(tag + " (abs-max computed, 2 passes)", n, secs, bpe, 3, ops,
                     note="memset + amax + quantize + finalize; bytes count one read")
             else:
-                secs = timeit(lambda: fp4q.quantize(x, fmt, block, strat, rot, out=out))
+                secs = timeit([lambda i=i: fp4q.quantize(xs[i], fmt, block, strat, rot, out=outs[i])
+                               for i in range(nc)])
                 add(tag, n, secs, bpe, 1, ops)
-        del x
+            del outs
+        del xs, x0
         torch.cuda.empty_cache()
 
     quant_runs("c1_nvfp4_roundtrip", [("nvfp4", 16, "absmax", 0)], want_mse=True, dq=torch.float32)
@@ -366,16 +392,23 @@ def breakdown(dev, flush, peaks, reps: int = 10):
                                           ("mxfp4", 32, "absmax", 128)])
     # FOCUS
     d = synth.workload("c4_focus")
-    w, c, g = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)
-    n = w.numel()
+    w0, c0, g0 = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)
+    n = w0.numel()
+    nc = copies_for(4 * n, l2, cap=reps + 3)
+    ws = [w0] + [w0.clone() for _ in range(nc - 1)]
+    cs = [c0] + [c0.clone() for _ in range(nc - 1)]
+    gs = [g0] + [g0.clone() for _ in range(nc - 1)]
     for fmt, block in (("nvfp4", 16), ("mxfp4", 32)):
-        fo = fp4q.FocusOut(torch.empty_like(w), torch.empty(1, device=dev) if fmt == "nvfp4" else None,
-                           None, None)
-        ga = fp4q.global_amax(w, 0) if fmt == "nvfp4" else None
-        secs = timeit(lambda: fp4q.focus_fwd(w, c, fmt, block, 8, global_amax=ga, out=fo))
+        fos = [fp4q.FocusOut(torch.empty_like(w0),
+                             torch.empty(1, device=dev) if fmt == "nvfp4" else None, None, None)
+               for _ in range(nc)]
+        ga = fp4q.global_amax(w0, 0) if fmt == "nvfp4" else None
+        secs = timeit([lambda i=i: fp4q.focus_fwd(ws[i], cs[i], fmt, block, 8, global_amax=ga,
+                                                  out=fos[i]) for i in range(nc)])
         add(f"c4_focus fwd {fmt} B{block} sub8 -> bf16", n, secs, 2 + 0.25 + 2, 1)
-    dc = torch.empty(4096, 512, device=dev)
-    secs = timeit(lambda: fp4q.focus_bwd(w, g, c, 8, out=dc))
+    dcs = [torch.empty(4096, 512, device=dev) for _ in range(nc)]
+    secs = timeit([lambda i=i: fp4q.focus_bwd(ws[i], gs[i], cs[i], 8, out=dcs[i])
+                   for i in range(nc)])
     add("c4_focus bwd sub8 -> fp32 dc", n, secs, 2 + 2 + 0.25 + 0.5, 1)
     return rows_out
 

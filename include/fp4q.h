@@ -31,8 +31,9 @@
  *    and the call returns before it completes.
  *  - Arguments are validated on the host before anything is enqueued; on an
  *    error nothing is launched and outputs are untouched.
- *  - rows == 0 or cols == 0 is an empty tensor: nothing is computed except
- *    that NVFP4 global_scale_out receives 1.0.
+ *  - rows == 0 or cols == 0 is an empty tensor: its array pointers may be
+ *    NULL, nothing is read or written except that NVFP4 global_scale_out
+ *    receives 1.0 (and fp4q_global_amax writes 0).
  *  - Inputs must be finite. Outputs must not overlap inputs or each other.
  *  - FP4Q_ERR_CUDA means a launch was rejected by the CUDA runtime; the
  *    runtime's code is available from fp4q_last_cuda_error(). Faults that
@@ -170,7 +171,9 @@ fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot,
  * Element-wise rounding primitives used by every kernel above, exposed so
  * that they can be checked exhaustively: one output byte per input float.
  * fp4q_e2m1_encode: 4-bit E2M1 code (sign kept, RNE, saturating at +-6).
- * fp4q_e4m3_encode: E4M3 code of v >= 0 (RNE, saturating at 448).
+ * fp4q_e4m3_encode: E4M3 code of a non-negative v with a clear sign bit
+ *                   (RNE, saturating at 448); the kernels only round such
+ *                   values (a block abs-max over a positive divisor).
  */
 fp4q_status fp4q_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t stream);
 fp4q_status fp4q_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t stream);

@@ -95,7 +95,10 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
     if (dq != nullptr && dq_dtype != FP4Q_OUT_F32 && dq_dtype != FP4Q_OUT_BF16)
         return FP4Q_ERR_UNSUPPORTED;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
-    if (x == nullptr || codes == nullptr || scales == nullptr || (nv && global_scale_out == nullptr))
+    const int64_t n = rows * cols;
+    if (nv && global_scale_out == nullptr)
+        return FP4Q_ERR_NULL;
+    if (n > 0 && (x == nullptr || codes == nullptr || scales == nullptr))
         return FP4Q_ERR_NULL;
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(block_mse) ||
         !aligned16(dq))
@@ -104,8 +107,6 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
         return FP4Q_ERR_ALIGN;
     if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
         return FP4Q_ERR_ALIAS;
-
-    const int64_t n = rows * cols;
     if (n == 0)
         return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
 
@@ -119,6 +120,7 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
     a.dq_kind = dq == nullptr ? 0 : (dq_dtype == FP4Q_OUT_F32 ? 1 : 2);
     a.amax = nullptr;
     a.sg_out = nullptr;
+    a.keep = 0xFFFFFFFFu;
     int kstrat = nv ? (int)strat : K_MX;
     if (nv) {
         if (global_amax_in != nullptr) {
@@ -150,13 +152,13 @@ fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
     if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
         return FP4Q_ERR_UNSUPPORTED;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
     if (codes == nullptr || scales == nullptr || out == nullptr || (nv && global_scale == nullptr))
         return FP4Q_ERR_NULL;
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
-    const int64_t n = rows * cols;
-    if (n == 0)
-        return FP4Q_OK;
     DequantArgs a;
     a.codes = codes;
     a.scales = scales;
@@ -176,15 +178,15 @@ fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* s
     if (st != FP4Q_OK)
         return st;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
     if (x == nullptr || codes == nullptr || scales == nullptr || block_mse == nullptr ||
         (nv && global_scale == nullptr))
         return FP4Q_ERR_NULL;
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(block_mse) ||
         (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
-    const int64_t n = rows * cols;
-    if (n == 0)
-        return FP4Q_OK;
     MseArgs a;
     a.x = static_cast<const uint16_t*>(x);
     a.codes = codes;
@@ -208,9 +210,12 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
     if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
         return FP4Q_ERR_UNSUPPORTED;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
-    if (w == nullptr || c == nullptr || w_hat == nullptr || (nv && global_scale_out == nullptr))
+    const int64_t n = rows * cols;
+    if (nv && global_scale_out == nullptr)
         return FP4Q_ERR_NULL;
-    if ((codes == nullptr) != (scales == nullptr))
+    if (n > 0 && (w == nullptr || c == nullptr || w_hat == nullptr))
+        return FP4Q_ERR_NULL;
+    if (n > 0 && (codes == nullptr) != (scales == nullptr))
         return FP4Q_ERR_NULL;
     if (!aligned16(w) || !aligned16(c) || !aligned16(w_hat) || !aligned16(codes) || !aligned16(scales))
         return FP4Q_ERR_ALIGN;
@@ -218,7 +223,6 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
         return FP4Q_ERR_ALIGN;
     if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
         return FP4Q_ERR_ALIAS;
-    const int64_t n = rows * cols;
     if (n == 0)
         return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
 
@@ -232,6 +236,7 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
     a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
     a.codes = codes;
     a.scales = scales;
+    a.keep = 0xFFFFFFFFu;
     if (nv) {
         if (global_amax_in != nullptr) {
             a.amax = global_amax_in;
@@ -258,13 +263,13 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
         return FP4Q_ERR_UNSUPPORTED;
     if (rows < 0 || cols < 0 || cols % sub != 0 || (cols > 0 && rows > kMaxElems / cols))
         return FP4Q_ERR_SHAPE;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
     if (w == nullptr || g == nullptr || c == nullptr || dc == nullptr)
         return FP4Q_ERR_NULL;
     if (!aligned16(w) || !aligned16(g) || !aligned16(c) || !aligned16(dc))
         return FP4Q_ERR_ALIGN;
-    const int64_t n = rows * cols;
-    if (n == 0)
-        return FP4Q_OK;
     FocusBwdArgs a;
     a.w = static_cast<const uint16_t*>(w);
     a.g = static_cast<const uint16_t*>(g);
@@ -281,11 +286,11 @@ fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot,
         return FP4Q_ERR_UNSUPPORTED;
     if (rows < 0 || cols < 0 || (rot > 0 && cols % rot != 0) || (cols > 0 && rows > kMaxElems / cols))
         return FP4Q_ERR_SHAPE;
-    if (x == nullptr || amax_out == nullptr)
+    const int64_t n = rows * cols;
+    if (amax_out == nullptr || (n > 0 && x == nullptr))
         return FP4Q_ERR_NULL;
     if (!aligned16(x) || !aligned4(amax_out))
         return FP4Q_ERR_ALIGN;
-    const int64_t n = rows * cols;
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess || n == 0)
         return cuda_status(e);
@@ -297,12 +302,12 @@ fp4q_status fp4q_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream
 {
     if (n < 0 || n > kMaxElems)
         return FP4Q_ERR_SHAPE;
+    if (n == 0)
+        return FP4Q_OK;
     if (u == nullptr || out == nullptr)
         return FP4Q_ERR_NULL;
     if (!aligned16(u) || !aligned16(out))
         return FP4Q_ERR_ALIGN;
-    if (n == 0)
-        return FP4Q_OK;
     return cuda_status(launch_e2m1_encode(u, n, out, stream));
 }
 
@@ -310,12 +315,12 @@ fp4q_status fp4q_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream
 {
     if (n < 0 || n > kMaxElems)
         return FP4Q_ERR_SHAPE;
+    if (n == 0)
+        return FP4Q_OK;
     if (v == nullptr || out == nullptr)
         return FP4Q_ERR_NULL;
     if (!aligned16(v) || !aligned16(out))
         return FP4Q_ERR_ALIGN;
-    if (n == 0)
-        return FP4Q_OK;
     return cuda_status(launch_e4m3_encode(v, n, out, stream));
 }
 

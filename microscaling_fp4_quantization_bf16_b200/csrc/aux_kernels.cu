@@ -23,12 +23,12 @@ static inline bool grid_ok(int64_t nseg)
     return nblk > 0 && nblk <= 0x7FFFFFFF;
 }
 
-// E8M0 byte -> 2^(b - 127); 255 is NaN.
+// E8M0 byte -> 2^(b - 127); 255 is NaN; byte 0 is the subnormal 2^-127.
 __device__ __forceinline__ float e8m0_dec(uint32_t b)
 {
     if (b == 255u)
         return __uint_as_float(0x7FC00000u);
-    return b == 0u ? __uint_as_float(0x00200000u) : __uint_as_float(b << 23);
+    return b == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
 }
 
 // ------------------------------------------------------------ global abs-max
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
         r[k] = zb[b] ? 0.0f : guarded_rcp(__fmul_rn(S[b], ck[k]));
     }
     uint32_t q[4];
-    encode_seg<SUB>(y, r, zk, q);
+    encode_seg<SUB>(y, r, zk, a.keep, q);
     float yh[SEG];
     decode_seg<B>(q, S, yh);
     store_seg_values(a.w_hat, a.out_kind, s, nvalid, yh);

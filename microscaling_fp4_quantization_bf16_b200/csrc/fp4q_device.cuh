@@ -205,10 +205,10 @@ __device__ __forceinline__ int e8m0_exp(float a)
     return max(E - 129, -127);
 }
 
-// 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00200000).
+// 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
 __device__ __forceinline__ float pow2f(int e)
 {
-    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00200000u);
+    return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);
 }
 
 // ------------------------------------------------------------------ Hadamard
@@ -289,9 +289,15 @@ __device__ __forceinline__ float tree_sum(float* e)
 
 // Codes of the segment: u = y * r(block), RNE to E2M1, eight per word; the
 // codes of blocks with a zero scale are forced to 0x0.
+//
+// `keep` must be a run-time all-ones word (a kernel argument). Every encoded
+// word is ANDed with it before anything decodes it again: decoding a word
+// straight out of e2m1_pack8, with no intervening run-time operation, was
+// measured on sm_100a to return 0 for the elements held in bytes 2 and 3.
 template <int B>
 __device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&r)[SEG / B],
-                                           const bool (&zero)[SEG / B], uint32_t (&q)[4])
+                                           const bool (&zero)[SEG / B], uint32_t keep,
+                                           uint32_t (&q)[4])
 {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -305,7 +311,7 @@ __device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&
         for (int j = 0; j < 8; ++j)
             if (zero[(8 * w + j) / B])
                 m |= 0xFu << (4 * j);
-        q[w] = qw & ~m;
+        q[w] = qw & (keep & ~m);
     }
 }
 
@@ -347,11 +353,11 @@ __device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&
         sse[b] = tree_sum<B>(e + b * B);
 }
 
-// SSE of one B-wide block yb against value(RNE_E2M1(yb * r)) * S. The codes
-// of a zero scale need no masking here: u = y * 0 is a signed zero whose
+// SSE of one B-wide block yb against value(RNE_E2M1(yb * r)) * S (`keep` as
+// in encode_seg). The codes of a zero scale need no masking here: u = y * 0 is a signed zero whose
 // value times S = 0 is a signed zero, and y - (+-0) == y.
 template <int B>
-__device__ __forceinline__ float block_sse(const float* yb, float r, float S)
+__device__ __forceinline__ float block_sse(const float* yb, float r, float S, uint32_t keep)
 {
     float e[B];
     if constexpr (B >= 8) {
@@ -361,7 +367,7 @@ __device__ __forceinline__ float block_sse(const float* yb, float r, float S)
 #pragma unroll
             for (int j = 0; j < 8; ++j)
                 u[j] = __fmul_rn(yb[8 * g + j], r);
-            e2m1_unpack8(e2m1_pack8(u), v);
+            e2m1_unpack8(e2m1_pack8(u) & keep, v);  // see encode_seg on `keep`
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
                 float d = __fsub_rn(yb[8 * g + j], __fmul_rn(v[j], S));
@@ -373,7 +379,7 @@ __device__ __forceinline__ float block_sse(const float* yb, float r, float S)
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             u[j] = __fmul_rn(yb[j], r);
-        e2m1_unpack4(e2m1_pack4(u), v);
+        e2m1_unpack4(e2m1_pack4(u) & keep, v);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
             float d = __fsub_rn(yb[j], __fmul_rn(v[j], S));

@@ -22,6 +22,7 @@ struct QuantArgs {
     float* mse;             // [n / B] or NULL
     void* dq;               // [n] or NULL
     int dq_kind;            // 0 none, 1 fp32, 2 bf16
+    uint32_t keep;          // 0xFFFFFFFF, passed at run time (see encode_seg)
 };
 
 struct DequantArgs {
@@ -52,6 +53,7 @@ struct FocusFwdArgs {
     int out_kind;           // 1 fp32, 2 bf16
     uint8_t* codes;         // optional
     uint8_t* scales;        // optional
+    uint32_t keep;          // 0xFFFFFFFF, passed at run time (see encode_seg)
 };
 
 struct FocusBwdArgs {

@@ -77,7 +77,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
             r[b] = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
             zero[b] = false;
         }
-        encode_seg<B>(y, r, zero, q);
+        encode_seg<B>(y, r, zero, a.keep, q);
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
         static_for<NB>([&](auto bi) {
             constexpr int b = decltype(bi)::value;
@@ -85,7 +85,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
             int bc = 1;
 #pragma unroll 1
             for (int c = 1; c <= 0x7E; ++c) {
-                const float v = block_sse<B>(y + b * B, tR[c], tS[c]);
+                const float v = block_sse<B>(y + b * B, tR[c], tS[c], a.keep);
                 if (c == 1 || v < best) {
                     best = v;
                     bc = c;
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
             zero[b] = (S[b] == 0.0f);
             sse[b] = best;
         });
-        encode_seg<B>(y, r, zero, q);
+        encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
     } else {
         const float den6 = __fmul_rn(6.0f, sg);
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
             zero[b] = (S[b] == 0.0f);
             r[b] = zero[b] ? 0.0f : guarded_rcp(S[b]);
         }
-        encode_seg<B>(y, r, zero, q);
+        encode_seg<B>(y, r, zero, a.keep, q);
         if constexpr (STRAT == K_FOUR_OVER_SIX) {
             const float den4 = __fmul_rn(4.0f, sg);
             float S4[NB], r4[NB], sse4[NB];
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
                 z4[b] = (S4[b] == 0.0f);
                 r4[b] = z4[b] ? 0.0f : guarded_rcp(S4[b]);
             }
-            encode_seg<B>(y, r4, z4, q4);
+            encode_seg<B>(y, r4, z4, a.keep, q4);
             sse_seg<B>(y, q, S, sse);
             sse_seg<B>(y, q4, S4, sse4);
 #pragma unroll

@@ -42,9 +42,14 @@ def assert_exact(got, want, what):
 
 
 def assert_mse(got, want, what):
+    """Within 1e-6 relative (equal values, infinities included, count as 0),
+    then also bit-exact, which the pinned operation order gives."""
     got = np.asarray(got, np.float32)
     want = np.asarray(want, np.float32)
-    rel = np.abs(got.astype(np.float64) - want) / np.maximum(np.abs(want.astype(np.float64)), 1e-38)
+    g64, w64 = got.astype(np.float64), want.astype(np.float64)
+    same = (got.view(np.uint32) == want.view(np.uint32))
+    with np.errstate(invalid="ignore"):
+        rel = np.where(same, 0.0, np.abs(g64 - w64) / np.maximum(np.abs(w64), 1e-38))
     assert float(rel.max(initial=0.0)) <= 1e-6, f"{what}: max rel err {rel.max()}"
     assert_exact(got, want, what + " (bit-exact)")
 
