@@ -34,7 +34,8 @@ ROWS, COLS = 4096, 4096
 ROTS = (0, 32)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 SM_COUNT_NOMINAL, FP32_LANES_PER_SM, SM_MAX_MHZ_NOMINAL = 148, 128, 1965.0
-SLEEP_CYCLES = 100_000  # ~50 us of GPU spin before each timed launch (CPU enqueue cover)
+SLEEP_CYCLES_PER_LAUNCH = 100_000  # ~50 us of GPU spin per queued launch (CPU enqueue cover)
+BATCH_STEPS = 10                   # steps queued behind one cover
 
 
 def copies_for(nbytes: int, l2: int, cap: int = 128) -> int:
@@ -181,22 +182,30 @@ def run_ours(args, rank, world, local_rank):
     outs = [fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
                            torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
                            None, None, None) for _ in range(ncopy)]
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in ROTS]
     counter = [0]
 
-    def step(times):
-        for k, r in enumerate(ROTS):
-            j = counter[0] % ncopy
-            counter[0] += 1
-            torch.cuda._sleep(SLEEP_CYCLES)  # the GPU is busy while the launch is enqueued
-            s, e = evs[k]
-            s.record()
-            fp4q.quantize(xs[j], "mxfp4", 32, "absmax", r, out=outs[j])
-            e.record()
+    def batch(nsteps, times):
+        """nsteps steps enqueued behind one sleep (so the GPU never waits for
+        the CPU), with an event after every launch: per-launch durations in a
+        stream of back-to-back launches."""
+        nl = nsteps * len(ROTS)
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)]
+        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nl)
+        ev[0].record()
+        order = []
+        for _ in range(nsteps):
+            for r in ROTS:
+                j = counter[0] % ncopy
+                counter[0] += 1
+                fp4q.quantize(xs[j], "mxfp4", 32, "absmax", r, out=outs[j])
+                ev[len(order) + 1].record()
+                order.append(r)
         torch.cuda.synchronize()
-        for k, r in enumerate(ROTS):
-            times[r].append(evs[k][0].elapsed_time(evs[k][1]))
+        for k, r in enumerate(order):
+            times[r].append(ev[k].elapsed_time(ev[k + 1]))
+
+    def step(times):
+        batch(1, times)
 
     sampler = ClockSampler(local_rank)
     with sampler:
@@ -211,8 +220,8 @@ def run_ours(args, rank, world, local_rank):
         torch.cuda.synchronize()
         t0 = time.perf_counter()
         times = {r: [] for r in ROTS}
-        for _ in range(args.steps):
-            step(times)
+        for i in range(0, args.steps, BATCH_STEPS):
+            batch(min(BATCH_STEPS, args.steps - i), times)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -250,12 +259,14 @@ def run_ours(args, rank, world, local_rank):
     ch = {r: torch.empty(ROWS, COLS // 2, dtype=torch.uint8).pin_memory() for r in ROTS}
     sh = {r: torch.empty(ROWS, COLS // 32, dtype=torch.uint8).pin_memory() for r in ROTS}
 
+    eouts = {r: outs[k] for k, r in enumerate(ROTS)}
+
     def e2e_step():
         xd.copy_(xh, non_blocking=True)
         for r in ROTS:
-            fp4q.quantize(xd, "mxfp4", 32, "absmax", r, out=outs[r])
-            ch[r].copy_(outs[r].codes, non_blocking=True)
-            sh[r].copy_(outs[r].scales, non_blocking=True)
+            fp4q.quantize(xd, "mxfp4", 32, "absmax", r, out=eouts[r])
+            ch[r].copy_(eouts[r].codes, non_blocking=True)
+            sh[r].copy_(eouts[r].scales, non_blocking=True)
         torch.cuda.synchronize()
 
     for _ in range(args.warmup):
@@ -320,17 +331,20 @@ def breakdown(dev, peaks, reps: int = 10):
     rows_out = []
 
     def timeit(fns):
-        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        ts = []
-        for i in range(reps + 3):
-            torch.cuda._sleep(SLEEP_CYCLES)
-            s.record()
+        """Median per-launch time of launches queued back to back (one event
+        after each), cycling through the given closures (one per input copy)
+        so that no launch finds its input in L2."""
+        nrep = max(reps, len(fns))
+        for i in range(3):
             fns[i % len(fns)]()
-            e.record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(s.elapsed_time(e))
-        return statistics.median(ts) / 1e3
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nrep + 1)]
+        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nrep)
+        ev[0].record()
+        for i in range(nrep):
+            fns[(i + 3) % len(fns)]()
+            ev[i + 1].record()
+        torch.cuda.synchronize()
+        return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(nrep)) / 1e3
 
     def add(name, n, secs, bpe, launches, fp32_ops=None, note=None):
         gbs = n * bpe / secs / 1e9
@@ -350,7 +364,7 @@ def breakdown(dev, peaks, reps: int = 10):
         x0 = synth.workload(wl)["x"].to(dev)
         n = x0.numel()
         R, C = x0.shape
-        nc = copies_for(2 * n, l2, cap=min(128, reps + 3))
+        nc = copies_for(2 * n, l2)
         xs = [x0] + [x0.clone() for _ in range(nc - 1)]
         for fmt, block, strat, rot in runs:
             nv = fmt == "nvfp4"
@@ -394,7 +408,7 @@ def breakdown(dev, peaks, reps: int = 10):
     d = synth.workload("c4_focus")
     w0, c0, g0 = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)
     n = w0.numel()
-    nc = copies_for(4 * n, l2, cap=reps + 3)
+    nc = copies_for(4 * n, l2)
     ws = [w0] + [w0.clone() for _ in range(nc - 1)]
     cs = [c0] + [c0.clone() for _ in range(nc - 1)]
     gs = [g0] + [g0.clone() for _ in range(nc - 1)]

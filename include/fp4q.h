@@ -184,6 +184,19 @@ const char* fp4q_status_string(fp4q_status s);
 /* The cudaError_t of the last FP4Q_ERR_CUDA returned on this host thread. */
 int fp4q_last_cuda_error(void);
 
+/*
+ * Pipeline health. The TMA-fed quantize kernel waits on shared-memory
+ * barriers with a bounded number of polls; a wait that runs out (which
+ * correct operation never produces) makes the kernel leave early and adds
+ * one to a per-device counter instead of hanging the GPU. This call
+ * synchronises with the current device, returns the counter and clears it
+ * (-1 if the read failed). Environment: FP4Q_TMA=1 routes quantize calls
+ * whose flattened length is a multiple of 64 (all strategies but brute
+ * force) to the TMA-fed kernel; the default direct-load kernel computes the
+ * same bits.
+ */
+int fp4q_device_errors(void);
+
 #ifdef __cplusplus
 }
 #endif

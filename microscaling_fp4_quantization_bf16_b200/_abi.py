@@ -30,6 +30,7 @@ SIGNATURES = {
     "fp4q_e4m3_encode": (_i32, [_p, _i64, _p, _p]),
     "fp4q_status_string": (C.c_char_p, [_i32]),
     "fp4q_last_cuda_error": (_i32, []),
+    "fp4q_device_errors": (_i32, []),
 }
 
 _lib = None

@@ -3,11 +3,19 @@
 // Host side only: validate every argument, then enqueue kernels on the
 // caller's stream. Nothing is allocated and nothing is synchronised.
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
+
+#include <cuda.h>
 
 #include "fp4q.h"
 #include "internal.h"
 
 using namespace fp4q;
+
+// Count of pipeline waits that ran out (see quant_tma.cuh); one word per
+// device, read and cleared by fp4q_device_errors().
+__device__ unsigned int g_fp4q_device_errors;
 
 namespace {
 
@@ -52,8 +60,78 @@ fp4q_status check_format(int64_t rows, int64_t cols, int fmt, int block, int rot
     return FP4Q_OK;
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// cuTensorMapEncodeTiled from the driver, looked up once (no link to libcuda).
+EncodeTiledFn encode_tiled()
+{
+    static EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+// FP4Q_TMA=1 routes eligible quantize calls (flattened length a multiple of
+// 64, not brute force) to the TMA-fed kernel; both kernels compute the same
+// bits. The direct-load kernel is the default: on B200 it measured faster at
+// every size for unrotated inputs and at all but the largest sizes with a
+// 32-wide rotation.
+bool tma_requested()
+{
+    const char* v = std::getenv("FP4Q_TMA");
+    return v != nullptr && std::strcmp(v, "0") != 0;
+}
+
+// View of x as [n / 64, 64] bf16 rows of 128 bytes, box 64 x 64, 128-byte swizzle.
+bool make_row_map(CUtensorMap* map, const void* x, int64_t n)
+{
+    EncodeTiledFn fn = encode_tiled();
+    if (fn == nullptr)
+        return false;
+    cuuint64_t dims[2] = {64, (cuuint64_t)(n / 64)};
+    cuuint64_t strides[1] = {128};
+    cuuint32_t box[2] = {64, (cuuint32_t)TMA_TILE_ROWS};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(x), dims, strides, box,
+                    estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
 cudaError_t launch_quant(int block, int strat, int rot, const QuantArgs& a, cudaStream_t st)
 {
+    const bool tma_shape = a.n % 64 == 0 && a.n / 64 < ((int64_t)1 << 31);
+    if (strat != K_BRUTE_FORCE && tma_shape && tma_requested()) {
+        CUtensorMap map;
+        if (make_row_map(&map, a.x, a.n)) {
+            int dev = 0, sms = 0;
+            unsigned* err = nullptr;
+            cudaError_t e = cudaGetDevice(&dev);
+            if (e == cudaSuccess)
+                e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+            if (e == cudaSuccess)
+                e = cudaGetSymbolAddress(reinterpret_cast<void**>(&err), g_fp4q_device_errors);
+            if (e != cudaSuccess)
+                return e;
+            const int64_t ntiles = (a.n / 64 + TMA_TILE_ROWS - 1) / TMA_TILE_ROWS;
+            switch (block) {
+            case 4: return launch_quant_tma_b4(strat, rot, a, map, ntiles, err, sms, st);
+            case 8: return launch_quant_tma_b8(strat, rot, a, map, ntiles, err, sms, st);
+            case 16: return launch_quant_tma_b16(strat, rot, a, map, ntiles, err, sms, st);
+            case 32: return launch_quant_tma_b32(strat, rot, a, map, ntiles, err, sms, st);
+            default: return cudaErrorInvalidValue;
+            }
+        }
+    }
     switch (block) {
     case 4: return launch_quant_b4(strat, rot, a, st);
     case 8: return launch_quant_b8(strat, rot, a, st);
@@ -339,5 +417,15 @@ const char* fp4q_status_string(fp4q_status s)
 }
 
 int fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+
+int fp4q_device_errors(void)
+{
+    unsigned v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_fp4q_device_errors, sizeof(v)) != cudaSuccess)
+        return -1;
+    if (v != 0 && cudaMemcpyToSymbol(g_fp4q_device_errors, &zero, sizeof(zero)) != cudaSuccess)
+        return -1;
+    return (int)v;
+}
 
 }  // extern "C"

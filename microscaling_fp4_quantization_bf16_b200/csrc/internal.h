@@ -4,6 +4,7 @@
 
 #include <cstdint>
 
+#include <cuda.h>
 #include <cuda_runtime_api.h>
 
 namespace fp4q {
@@ -70,6 +71,19 @@ cudaError_t launch_quant_b4(int strat, int rot, const QuantArgs& a, cudaStream_t
 cudaError_t launch_quant_b8(int strat, int rot, const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_quant_b16(int strat, int rot, const QuantArgs& a, cudaStream_t st);
 cudaError_t launch_quant_b32(int strat, int rot, const QuantArgs& a, cudaStream_t st);
+
+// TMA-fed quantize kernel (flattened length a multiple of 64; not brute force).
+// The tensor map views x as [n / 64, 64] bf16 with 128-byte swizzle and a box
+// of 64 x 64; ntiles = ceil(n / 64 / 64); err is the device error word.
+constexpr int TMA_TILE_ROWS = 64;
+cudaError_t launch_quant_tma_b4(int strat, int rot, const QuantArgs& a, const CUtensorMap& map,
+                                int64_t ntiles, unsigned* err, int sms, cudaStream_t st);
+cudaError_t launch_quant_tma_b8(int strat, int rot, const QuantArgs& a, const CUtensorMap& map,
+                                int64_t ntiles, unsigned* err, int sms, cudaStream_t st);
+cudaError_t launch_quant_tma_b16(int strat, int rot, const QuantArgs& a, const CUtensorMap& map,
+                                 int64_t ntiles, unsigned* err, int sms, cudaStream_t st);
+cudaError_t launch_quant_tma_b32(int strat, int rot, const QuantArgs& a, const CUtensorMap& map,
+                                 int64_t ntiles, unsigned* err, int sms, cudaStream_t st);
 
 cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st);
 cudaError_t launch_finalize_sg(float* g, cudaStream_t st);

@@ -1,9 +1,15 @@
-// quant_b8.cu -- instantiations of the quantize kernel for block size 8.
-#include "quant_kernel.cuh"
+// quant_b8.cu -- instantiations of the quantize kernels for block size 8.
+#include "quant_tma.cuh"
 
 namespace fp4q {
 cudaError_t launch_quant_b8(int strat, int rot, const QuantArgs& a, cudaStream_t st)
 {
     return launch_quant_impl<8>(strat, rot, a, st);
+}
+
+cudaError_t launch_quant_tma_b8(int strat, int rot, const QuantArgs& a, const CUtensorMap& map,
+                                 int64_t ntiles, unsigned* err, int sms, cudaStream_t st)
+{
+    return launch_quant_tma_impl<8>(strat, rot, a, map, ntiles, err, sms, st);
 }
 }  // namespace fp4q

@@ -22,44 +22,22 @@ namespace fp4q {
 
 constexpr int QTHREADS = 256;
 
-template <int B, int ROT, int STRAT>
-__global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
+// Brute-force candidate tables: dequantization scale and reciprocal of every
+// E4M3 code (index 0 and 0x7F unused), built by each block.
+template <int STRAT>
+struct BruteTables {
+    float S[STRAT == K_BRUTE_FORCE ? 128 : 1];
+    float R[STRAT == K_BRUTE_FORCE ? 128 : 1];
+};
+
+// Scale selection, encoding and stores for one 32-element segment s whose
+// (rotated) values are y. nvalid < 32 only for the last segment.
+template <int B, int STRAT>
+__device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s, int nvalid,
+                                                const QuantArgs& a, float sg,
+                                                const BruteTables<STRAT>& tab)
 {
     constexpr int NB = SEG / B;
-    const int lane = threadIdx.x & 31;
-    const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
-
-    float sg = 1.0f;
-    if constexpr (STRAT != K_MX) {
-        sg = global_scale_of(*a.amax);
-        if (a.sg_out != nullptr && s == 0)
-            *a.sg_out = sg;
-    }
-
-    // Brute force: dequantization scale and reciprocal of every E4M3 code,
-    // shared by the block.
-    __shared__ float tS[STRAT == K_BRUTE_FORCE ? 128 : 1];
-    __shared__ float tR[STRAT == K_BRUTE_FORCE ? 128 : 1];
-    if constexpr (STRAT == K_BRUTE_FORCE) {
-        for (int c = threadIdx.x; c < 128; c += QTHREADS) {
-            float S = (c >= 1 && c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
-            tS[c] = S;
-            tR[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
-        }
-        __syncthreads();
-    }
-
-    if (s - lane >= nseg)
-        return;  // the whole warp is past the end (warp-uniform)
-
-    float y[SEG];
-    load_seg_bf16(a.x, a.n, s, y);  // lanes past the end read zeros
-    rotate_seg<ROT>(y, lane);       // all 32 lanes take part
-    if (s >= nseg)
-        return;
-    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
-
     float amax[NB];
     block_amax<B>(y, amax);
 
@@ -85,15 +63,15 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
             int bc = 1;
 #pragma unroll 1
             for (int c = 1; c <= 0x7E; ++c) {
-                const float v = block_sse<B>(y + b * B, tR[c], tS[c], a.keep);
+                const float v = block_sse<B>(y + b * B, tab.R[c], tab.S[c], a.keep);
                 if (c == 1 || v < best) {
                     best = v;
                     bc = c;
                 }
             }
             sc[b] = (uint32_t)bc;
-            S[b] = tS[bc];
-            r[b] = tR[bc];
+            S[b] = tab.S[bc];
+            r[b] = tab.R[bc];
             zero[b] = (S[b] == 0.0f);
             sse[b] = best;
         });
@@ -180,6 +158,57 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
         decode_seg<B>(q, S, yh);
         store_seg_values(a.dq, a.dq_kind, s, nvalid, yh);
     }
+}
+
+// Global scale s_g for NVFP4 kernels (1 for MXFP4); thread 0 of block 0
+// publishes it when asked.
+template <int STRAT>
+__device__ __forceinline__ float kernel_global_scale(const QuantArgs& a)
+{
+    float sg = 1.0f;
+    if constexpr (STRAT != K_MX) {
+        sg = global_scale_of(*a.amax);
+        if (a.sg_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
+            *a.sg_out = sg;
+    }
+    return sg;
+}
+
+template <int STRAT>
+__device__ __forceinline__ void build_brute_tables(BruteTables<STRAT>& tab, float sg)
+{
+    if constexpr (STRAT == K_BRUTE_FORCE) {
+        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+            float S = (c >= 1 && c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
+            tab.S[c] = S;
+            tab.R[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
+        }
+        __syncthreads();
+    }
+}
+
+// Direct-load kernel: one segment per thread, four 128-bit global loads.
+// Used for the brute-force search (compute bound) and for tensors the TMA
+// kernel does not take (a flattened length that is not a multiple of 64).
+template <int B, int ROT, int STRAT>
+__global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
+{
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
+    const float sg = kernel_global_scale<STRAT>(a);
+    __shared__ BruteTables<STRAT> tab;
+    build_brute_tables<STRAT>(tab, sg);
+
+    if (s - lane >= nseg)
+        return;  // the whole warp is past the end (warp-uniform)
+    float y[SEG];
+    load_seg_bf16(a.x, a.n, s, y);  // lanes past the end read zeros
+    rotate_seg<ROT>(y, lane);       // all 32 lanes take part
+    if (s >= nseg)
+        return;
+    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    process_segment<B, STRAT>(y, s, nvalid, a, sg, tab);
 }
 
 template <int B>

@@ -133,8 +133,13 @@ def shapes_for(block, rot):
     return shapes
 
 
+@pytest.mark.parametrize("loads", ["direct", "tma"])
 @pytest.mark.parametrize("fmt,block,strat,rot", COMBOS)
-def test_quantize_small_shapes(gpu, fmt, block, strat, rot):
+def test_quantize_small_shapes(gpu, monkeypatch, loads, fmt, block, strat, rot):
+    """Every combination through the direct-load kernel and (FP4Q_TMA=1,
+    flattened length a multiple of 64) the TMA-fed kernel."""
+    if loads == "tma":
+        monkeypatch.setenv("FP4Q_TMA", "1")
     for k, (rows, cols) in enumerate(shapes_for(block, rot)):
         x = mixed(rows, cols, seed=1000 * block + rot + k)
         dq = (None, torch.float32, torch.bfloat16)[k % 3]
@@ -336,6 +341,22 @@ def test_focus_small(gpu, fmt, block, sub):
         assert_exact(dc.cpu().numpy(), oracle.focus_bwd(u16(w), u16(gr), u16(c), sub), "focus dc")
 
 
+@pytest.mark.parametrize("loads", ["direct", "tma"])
+def test_multi_tile_tma_tails(gpu, monkeypatch, loads):
+    """Row counts around the 4096-element TMA tile and the persistent grid,
+    including a last tile that is mostly past the end of the tensor."""
+    if loads == "tma":
+        monkeypatch.setenv("FP4Q_TMA", "1")
+    for rows, cols in ((65, 64), (64 * 3 + 1, 128), (4096 * 2 + 64, 64), (1, 4096 * 4)):
+        x = mixed(rows, cols, seed=rows)
+        for fmt, block, strat, rot in (("nvfp4", 16, "four_over_six", 16), ("mxfp4", 32, "absmax", 64),
+                                       ("nvfp4", 4, "absmax", 0)):
+            g = gpu_quantize(gpu, x, fmt, block, strat, rot, dq=torch.bfloat16)
+            o = oracle_quantize(x, fmt, block, strat, rot, dq=torch.bfloat16)
+            compare_quant(g, o, fmt, f"tails {rows}x{cols} {fmt} B{block} {strat} H{rot}")
+    assert gpu._abi.load().fp4q_device_errors() == 0
+
+
 def test_side_stream(gpu):
     x = mixed(64, 256, seed=8).cuda()
     s = torch.cuda.Stream()
@@ -346,3 +367,4 @@ def test_side_stream(gpu):
     torch.cuda.synchronize()
     assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
     assert torch.equal(a.mse.view(torch.int32), b.mse.view(torch.int32))
+    assert gpu._abi.load().fp4q_device_errors() == 0
