@@ -35,7 +35,6 @@ ROTS = (0, 32)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 SM_COUNT_NOMINAL, FP32_LANES_PER_SM, SM_MAX_MHZ_NOMINAL = 148, 128, 1965.0
 SLEEP_CYCLES_PER_LAUNCH = 100_000  # ~50 us of GPU spin per queued launch (CPU enqueue cover)
-BATCH_STEPS = 10                   # steps queued behind one cover
 
 
 def copies_for(nbytes: int, l2: int, cap: int = 128) -> int:
@@ -184,52 +183,44 @@ def run_ours(args, rank, world, local_rank):
                            None, None, None) for _ in range(ncopy)]
     counter = [0]
 
-    def batch(nsteps, times):
-        """nsteps steps enqueued behind one sleep (so the GPU never waits for
-        the CPU), with an event after every launch: per-launch durations in a
-        stream of back-to-back launches."""
-        nl = nsteps * len(ROTS)
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nl + 1)]
-        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nl)
+    def run_steps(nsteps):
+        """nsteps steps' work queued behind one sleep (the GPU never waits for
+        the CPU): nsteps rot-0 launches, then nsteps rot-32 launches, each on
+        its own input copy. Events only at the group boundaries, so launches
+        stream back to back (programmatic dependent launch overlaps each
+        launch with the previous kernel). Returns ms per group."""
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(ROTS) + 1)]
+        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nsteps * len(ROTS))
         ev[0].record()
-        order = []
-        for _ in range(nsteps):
-            for r in ROTS:
+        for k, r in enumerate(ROTS):
+            for _ in range(nsteps):
                 j = counter[0] % ncopy
                 counter[0] += 1
                 fp4q.quantize(xs[j], "mxfp4", 32, "absmax", r, out=outs[j])
-                ev[len(order) + 1].record()
-                order.append(r)
+            ev[k + 1].record()
         torch.cuda.synchronize()
-        for k, r in enumerate(order):
-            times[r].append(ev[k].elapsed_time(ev[k + 1]))
-
-    def step(times):
-        batch(1, times)
+        return [ev[k].elapsed_time(ev[k + 1]) for k in range(len(ROTS))]
 
     sampler = ClockSampler(local_rank)
     with sampler:
         soak_end = time.perf_counter() + args.soak
-        scratch = {r: [] for r in ROTS}
         while time.perf_counter() < soak_end:
-            step(scratch)
-        for _ in range(args.warmup):
-            step(scratch)
+            run_steps(10)
+        run_steps(args.warmup)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         t0 = time.perf_counter()
-        times = {r: [] for r in ROTS}
-        for i in range(0, args.steps, BATCH_STEPS):
-            batch(min(BATCH_STEPS, args.steps - i), times)
+        group_ms = run_steps(args.steps)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         t1 = time.perf_counter()
     clocks = sampler.summary(t0, t1)
     x = xs[0]
+    times = {r: [group_ms[k] / args.steps] for k, r in enumerate(ROTS)}
 
-    total_ms = sum(sum(v) for v in times.values())
+    total_ms = sum(group_ms)
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -243,7 +234,7 @@ def run_ours(args, rank, world, local_rank):
     dom = max(ROTS, key=lambda r: mean[r])
     alg_bytes = bytes_per_elem(32) * n
     achieved = alg_bytes / (mean[dom] / 1e3) / 1e9
-    kname = f"quant_kernel<32,{dom},mx>"
+    kname = f"quant_kernel<B=32, ROT={dom}, MXFP4 abs-max> (direct loads)"
     traffic = recorded_traffic(kname)
     roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -300,8 +291,13 @@ def run_ours(args, rank, world, local_rank):
                        "l2": f"inputs larger than L2: each launch reads its own copy of x "
                              f"({ncopy} copies, {ncopy * n * 2 / 2**20:.0f} MiB in rotation)",
                        "parallelism": f"replicas x{world} (independent tensors, no collective)",
-                       "soak_s": args.soak},
+                       "soak_s": args.soak,
+                       "timing": "steps queued behind one GPU sleep; the timed region runs all rot-0 "
+                                 "launches then all rot-32 launches back to back (one input copy "
+                                 "each), CUDA events at the start, between the groups and at the "
+                                 "end; per-kernel time = group time / launches"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": len(ROTS) * args.steps,
+            "launch_note": "every library kernel uses programmatic dependent launch",
             "clocks": clocks}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -331,20 +327,20 @@ def breakdown(dev, peaks, reps: int = 10):
     rows_out = []
 
     def timeit(fns):
-        """Median per-launch time of launches queued back to back (one event
-        after each), cycling through the given closures (one per input copy)
-        so that no launch finds its input in L2."""
+        """Average per-launch time of launches queued back to back behind one
+        sleep, events only at the ends, cycling through the given closures
+        (one per input copy) so that no launch finds its input in L2."""
         nrep = max(reps, len(fns))
         for i in range(3):
             fns[i % len(fns)]()
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(nrep + 1)]
-        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nrep)
-        ev[0].record()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nrep * 3)
+        ev0.record()
         for i in range(nrep):
             fns[(i + 3) % len(fns)]()
-            ev[i + 1].record()
+        ev1.record()
         torch.cuda.synchronize()
-        return statistics.median(ev[i].elapsed_time(ev[i + 1]) for i in range(nrep)) / 1e3
+        return ev0.elapsed_time(ev1) / nrep / 1e3
 
     def add(name, n, secs, bpe, launches, fp32_ops=None, note=None):
         gbs = n * bpe / secs / 1e9

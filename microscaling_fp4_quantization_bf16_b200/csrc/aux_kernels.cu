@@ -39,6 +39,7 @@ __device__ __forceinline__ float e8m0_dec(uint32_t b)
 template <int ROT>
 __global__ void __launch_bounds__(ATHREADS) amax_kernel(const uint16_t* x, int64_t n, unsigned* out)
 {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
@@ -88,37 +89,48 @@ __global__ void __launch_bounds__(ATHREADS) amax_kernel(const uint16_t* x, int64
     }
 }
 
-__global__ void finalize_sg_kernel(float* g) { *g = global_scale_of(*g); }
+__global__ void finalize_sg_kernel(float* g)
+{
+    pdl_begin();
+    *g = global_scale_of(*g);
+}
 
-__global__ void set_one_kernel(float* p) { *p = 1.0f; }
+__global__ void set_one_kernel(float* p)
+{
+    pdl_begin();
+    *p = 1.0f;
+}
 
 cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     const int64_t nseg = (n + SEG - 1) / SEG;
     if (!grid_ok(nseg))
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nseg);
     switch (rot) {
-    case 0: amax_kernel<0><<<g, ATHREADS, 0, st>>>(x, n, out); break;
-    case 16: amax_kernel<16><<<g, ATHREADS, 0, st>>>(x, n, out); break;
-    case 32: amax_kernel<32><<<g, ATHREADS, 0, st>>>(x, n, out); break;
-    case 64: amax_kernel<64><<<g, ATHREADS, 0, st>>>(x, n, out); break;
-    case 128: amax_kernel<128><<<g, ATHREADS, 0, st>>>(x, n, out); break;
+    case 0: e_ = launch_pdl(amax_kernel<0>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
+    case 16: e_ = launch_pdl(amax_kernel<16>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
+    case 32: e_ = launch_pdl(amax_kernel<32>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
+    case 64: e_ = launch_pdl(amax_kernel<64>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
+    case 128: e_ = launch_pdl(amax_kernel<128>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
+    return e_;
 }
 
 cudaError_t launch_finalize_sg(float* g, cudaStream_t st)
 {
-    finalize_sg_kernel<<<1, 1, 0, st>>>(g);
-    return cudaGetLastError();
+    cudaError_t e_ = cudaSuccess;
+    e_ = launch_pdl(finalize_sg_kernel, dim3(1), dim3(1), 0, st, g);
+    return e_;
 }
 
 cudaError_t launch_set_one(float* p, cudaStream_t st)
 {
-    set_one_kernel<<<1, 1, 0, st>>>(p);
-    return cudaGetLastError();
+    cudaError_t e_ = cudaSuccess;
+    e_ = launch_pdl(set_one_kernel, dim3(1), dim3(1), 0, st, p);
+    return e_;
 }
 
 // ------------------------------------------------------------ small helpers
@@ -188,6 +200,7 @@ __device__ __forceinline__ void store_seg_floats(float* p, int64_t s, int nvalid
 template <int B, bool MX>
 __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 {
+    pdl_begin();
     constexpr int NB = SEG / B;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
@@ -206,6 +219,7 @@ __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 
 cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     if (!grid_ok(nseg))
         return cudaErrorInvalidValue;
@@ -213,17 +227,17 @@ cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t
     if (mx) {
         if (block != 32)
             return cudaErrorInvalidValue;
-        dequant_kernel<32, true><<<g, ATHREADS, 0, st>>>(a);
+        e_ = launch_pdl(dequant_kernel<32, true>, dim3(g), dim3(ATHREADS), 0, st, a);
     } else {
         switch (block) {
-        case 4: dequant_kernel<4, false><<<g, ATHREADS, 0, st>>>(a); break;
-        case 8: dequant_kernel<8, false><<<g, ATHREADS, 0, st>>>(a); break;
-        case 16: dequant_kernel<16, false><<<g, ATHREADS, 0, st>>>(a); break;
-        case 32: dequant_kernel<32, false><<<g, ATHREADS, 0, st>>>(a); break;
+        case 4: e_ = launch_pdl(dequant_kernel<4, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+        case 8: e_ = launch_pdl(dequant_kernel<8, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+        case 16: e_ = launch_pdl(dequant_kernel<16, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+        case 32: e_ = launch_pdl(dequant_kernel<32, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
         default: return cudaErrorInvalidValue;
         }
     }
-    return cudaGetLastError();
+    return e_;
 }
 
 // ------------------------------------------------------------ block MSE
@@ -231,6 +245,7 @@ cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t
 template <int B, int ROT, bool MX>
 __global__ void __launch_bounds__(ATHREADS) block_mse_kernel(MseArgs a)
 {
+    pdl_begin();
     constexpr int NB = SEG / B;
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
@@ -259,15 +274,16 @@ __global__ void __launch_bounds__(ATHREADS) block_mse_kernel(MseArgs a)
 template <int B, bool MX>
 static cudaError_t launch_mse_rot(int rot, unsigned g, const MseArgs& a, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     switch (rot) {
-    case 0: block_mse_kernel<B, 0, MX><<<g, ATHREADS, 0, st>>>(a); break;
-    case 16: block_mse_kernel<B, 16, MX><<<g, ATHREADS, 0, st>>>(a); break;
-    case 32: block_mse_kernel<B, 32, MX><<<g, ATHREADS, 0, st>>>(a); break;
-    case 64: block_mse_kernel<B, 64, MX><<<g, ATHREADS, 0, st>>>(a); break;
-    case 128: block_mse_kernel<B, 128, MX><<<g, ATHREADS, 0, st>>>(a); break;
+    case 0: e_ = launch_pdl(block_mse_kernel<B, 0, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 16: e_ = launch_pdl(block_mse_kernel<B, 16, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 32: e_ = launch_pdl(block_mse_kernel<B, 32, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 64: e_ = launch_pdl(block_mse_kernel<B, 64, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 128: e_ = launch_pdl(block_mse_kernel<B, 128, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
+    return e_;
 }
 
 cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st)
@@ -331,6 +347,7 @@ __device__ __forceinline__ void load_coeffs(const uint16_t* c, int64_t s, int nv
 template <int B, int SUB, bool MX>
 __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
 {
+    pdl_begin();
     constexpr int NB = SEG / B;
     constexpr int NK = SEG / SUB;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
@@ -396,11 +413,11 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
 }
 
 template <int B, int SUB, bool MX>
-static bool try_ffwd(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st)
+static bool try_ffwd(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st, cudaError_t& e)
 {
     if constexpr (SUB <= B) {
         if (sub == SUB) {
-            focus_fwd_kernel<B, SUB, MX><<<g, ATHREADS, 0, st>>>(a);
+            e = launch_pdl(focus_fwd_kernel<B, SUB, MX>, dim3(g), dim3(ATHREADS), 0, st, a);
             return true;
         }
     }
@@ -410,10 +427,11 @@ static bool try_ffwd(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st
 template <int B, bool MX>
 static cudaError_t launch_ffwd_sub(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st)
 {
-    if (try_ffwd<B, 2, MX>(sub, g, a, st) || try_ffwd<B, 4, MX>(sub, g, a, st) ||
-        try_ffwd<B, 8, MX>(sub, g, a, st) || try_ffwd<B, 16, MX>(sub, g, a, st) ||
-        try_ffwd<B, 32, MX>(sub, g, a, st))
-        return cudaGetLastError();
+    cudaError_t e = cudaErrorInvalidValue;
+    if (try_ffwd<B, 2, MX>(sub, g, a, st, e) || try_ffwd<B, 4, MX>(sub, g, a, st, e) ||
+        try_ffwd<B, 8, MX>(sub, g, a, st, e) || try_ffwd<B, 16, MX>(sub, g, a, st, e) ||
+        try_ffwd<B, 32, MX>(sub, g, a, st, e))
+        return e;
     return cudaErrorInvalidValue;
 }
 
@@ -438,6 +456,7 @@ cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, 
 template <int SUB>
 __global__ void __launch_bounds__(ATHREADS) focus_bwd_kernel(FocusBwdArgs a)
 {
+    pdl_begin();
     constexpr int NK = SEG / SUB;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
@@ -462,25 +481,27 @@ __global__ void __launch_bounds__(ATHREADS) focus_bwd_kernel(FocusBwdArgs a)
 
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     if (!grid_ok(nseg))
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nseg);
     switch (sub) {
-    case 2: focus_bwd_kernel<2><<<g, ATHREADS, 0, st>>>(a); break;
-    case 4: focus_bwd_kernel<4><<<g, ATHREADS, 0, st>>>(a); break;
-    case 8: focus_bwd_kernel<8><<<g, ATHREADS, 0, st>>>(a); break;
-    case 16: focus_bwd_kernel<16><<<g, ATHREADS, 0, st>>>(a); break;
-    case 32: focus_bwd_kernel<32><<<g, ATHREADS, 0, st>>>(a); break;
+    case 2: e_ = launch_pdl(focus_bwd_kernel<2>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 4: e_ = launch_pdl(focus_bwd_kernel<4>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 8: e_ = launch_pdl(focus_bwd_kernel<8>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 16: e_ = launch_pdl(focus_bwd_kernel<16>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 32: e_ = launch_pdl(focus_bwd_kernel<32>, dim3(g), dim3(ATHREADS), 0, st, a); break;
     default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
+    return e_;
 }
 
 // ------------------------------------------------------------ primitives
 
 __global__ void e2m1_encode_kernel(const float* u, int64_t n, uint8_t* out)
 {
+    pdl_begin();
     const int64_t i = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
     if (i >= n)
         return;
@@ -490,6 +511,7 @@ __global__ void e2m1_encode_kernel(const float* u, int64_t n, uint8_t* out)
 
 __global__ void e4m3_encode_kernel(const float* v, int64_t n, uint8_t* out)
 {
+    pdl_begin();
     const int64_t i = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
     if (i >= n)
         return;
@@ -498,18 +520,20 @@ __global__ void e4m3_encode_kernel(const float* v, int64_t n, uint8_t* out)
 
 cudaError_t launch_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     if (!grid_ok(n))
         return cudaErrorInvalidValue;
-    e2m1_encode_kernel<<<grid_for(n), ATHREADS, 0, st>>>(u, n, out);
-    return cudaGetLastError();
+    e_ = launch_pdl(e2m1_encode_kernel, dim3(grid_for(n)), dim3(ATHREADS), 0, st, u, n, out);
+    return e_;
 }
 
 cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t st)
 {
+    cudaError_t e_ = cudaSuccess;
     if (!grid_ok(n))
         return cudaErrorInvalidValue;
-    e4m3_encode_kernel<<<grid_for(n), ATHREADS, 0, st>>>(v, n, out);
-    return cudaGetLastError();
+    e_ = launch_pdl(e4m3_encode_kernel, dim3(grid_for(n)), dim3(ATHREADS), 0, st, v, n, out);
+    return e_;
 }
 
 }  // namespace fp4q

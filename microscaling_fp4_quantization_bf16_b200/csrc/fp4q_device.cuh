@@ -39,6 +39,19 @@ __device__ __forceinline__ void static_for(F&& f)
     }
 }
 
+// ------------------------------------------------------------------ launch
+
+// Programmatic dependent launch. Every kernel of the library is launched with
+// programmatic stream serialization and starts with pdl_begin(): it waits
+// until the previous kernel in the stream has completed and its writes are
+// visible (so reading inputs it produced is safe), then lets the next kernel
+// begin launching, which overlaps that launch with this kernel's execution.
+__device__ __forceinline__ void pdl_begin()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ loads
 
 __device__ __forceinline__ uint4 ldg_stream(const uint4* p)

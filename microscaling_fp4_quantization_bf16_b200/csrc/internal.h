@@ -3,11 +3,31 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_runtime_api.h>
 
 namespace fp4q {
+
+// Launch with programmatic stream serialization (see pdl_begin in
+// fp4q_device.cuh); returns the launch status.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                       cudaStream_t st, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 // Strategy ids used by the kernels (NVFP4 strategies follow the ABI enum;
 // MXFP4 abs-max is its own kernel family).

@@ -193,6 +193,7 @@ __device__ __forceinline__ void build_brute_tables(BruteTables<STRAT>& tab, floa
 template <int B, int ROT, int STRAT>
 __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
 {
+    pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
@@ -221,8 +222,7 @@ cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream
     const dim3 grid((unsigned)nblk);
 #define FP4Q_QCASE(S_, R_)                                        \
     if (strat == S_ && rot == R_) {                               \
-        quant_kernel<B, R_, S_><<<grid, QTHREADS, 0, st>>>(a);    \
-        return cudaGetLastError();                                \
+        return launch_pdl(quant_kernel<B, R_, S_>, grid, dim3(QTHREADS), 0, st, a); \
     }
 #define FP4Q_QROTS(S_)      \
     FP4Q_QCASE(S_, 0)       \

@@ -93,6 +93,7 @@ __global__ void __launch_bounds__(TTHREADS)
     const int warp = threadIdx.x / 32;
     const int lane = threadIdx.x & 31;
 
+    pdl_begin();
     const float sg = kernel_global_scale<STRAT>(a);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -180,8 +181,8 @@ cudaError_t launch_tma_one(const CUtensorMap& map, const QuantArgs& a, int64_t n
         return e;
     per_sm = per_sm < 1 ? 1 : per_sm;
     const int64_t grid = ntiles < (int64_t)sms * per_sm ? ntiles : (int64_t)sms * per_sm;
-    kern<<<(unsigned)grid, TTHREADS, TMA_SMEM_BYTES, st>>>(map, a, ntiles, err);
-    return cudaGetLastError();
+    return launch_pdl(kern, dim3((unsigned)grid), dim3(TTHREADS), TMA_SMEM_BYTES, st, map, a, ntiles,
+                      err);
 }
 
 template <int B>
