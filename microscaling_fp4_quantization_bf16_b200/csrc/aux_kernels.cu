@@ -42,38 +42,38 @@ __global__ void __launch_bounds__(ATHREADS) amax_kernel(const uint16_t* x, int64
     pdl_begin();
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (n + SEG - 1) / SEG;
-    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    const int64_t t = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
     unsigned m = 0;
-    if (s - lane < nseg) {
-        if constexpr (ROT == 0) {
-            if (s < nseg) {
-                const int64_t base = s * SEG;
-                if (base + SEG <= n) {
-                    const uint4* p = reinterpret_cast<const uint4*>(x + base);
-                    unsigned acc = 0;
+    if constexpr (ROT == 0) {
+        if (t < nseg) {
+            const int64_t base = t * SEG;
+            if (base + SEG <= n) {
+                const uint4* p = reinterpret_cast<const uint4*>(x + base);
+                unsigned acc = 0;
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        uint4 v = ldg_stream(p + k);
-                        acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
-                        acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
-                        acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
-                        acc = __vmaxu2(acc, v.w & 0x7FFF7FFFu);
-                    }
-                    m = max(acc & 0xFFFFu, acc >> 16) << 16;
-                } else {
-                    for (int64_t i = base; i < n; ++i)
-                        m = max(m, ((unsigned)x[i] & 0x7FFFu) << 16);
+                for (int k = 0; k < 4; ++k) {
+                    uint4 v = ldg_stream(p + k);
+                    acc = __vmaxu2(acc, v.x & 0x7FFF7FFFu);
+                    acc = __vmaxu2(acc, v.y & 0x7FFF7FFFu);
+                    acc = __vmaxu2(acc, v.z & 0x7FFF7FFFu);
+                    acc = __vmaxu2(acc, v.w & 0x7FFF7FFFu);
                 }
+                m = max(acc & 0xFFFFu, acc >> 16) << 16;
+            } else {
+                for (int64_t i = base; i < n; ++i)
+                    m = max(m, ((unsigned)x[i] & 0x7FFFu) << 16);
             }
-        } else {
-            float y[SEG];
-            load_seg_bf16(x, n, s, y);
-            rotate_seg<ROT>(y, lane);
-            if (s < nseg) {
+        }
+    } else {
+        constexpr int SPT = SegsPerThread<ROT>::value;
+        if ((t - lane) * SPT < nseg) {  // warp-uniform
+            float y[SPT][SEG];
+            load_rotate<ROT>(x, n, t, lane, y);  // past the end reads zeros
+#pragma unroll
+            for (int k = 0; k < SPT; ++k)
 #pragma unroll
                 for (int i = 0; i < SEG; ++i)
-                    m = max(m, __float_as_uint(fabsf(y[i])));
-            }
+                    m = max(m, __float_as_uint(fabsf(y[k][i])));
         }
     }
     m = __reduce_max_sync(0xFFFFFFFFu, m);
@@ -103,20 +103,19 @@ __global__ void set_one_kernel(float* p)
 
 cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st)
 {
-    cudaError_t e_ = cudaSuccess;
     const int64_t nseg = (n + SEG - 1) / SEG;
-    if (!grid_ok(nseg))
+    const int64_t nthr = nseg;
+    if (!grid_ok(nthr))
         return cudaErrorInvalidValue;
-    const unsigned g = grid_for(nseg);
+    const unsigned g = grid_for(nthr);
     switch (rot) {
-    case 0: e_ = launch_pdl(amax_kernel<0>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
-    case 16: e_ = launch_pdl(amax_kernel<16>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
-    case 32: e_ = launch_pdl(amax_kernel<32>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
-    case 64: e_ = launch_pdl(amax_kernel<64>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
-    case 128: e_ = launch_pdl(amax_kernel<128>, dim3(g), dim3(ATHREADS), 0, st, x, n, out); break;
+    case 0: return launch_pdl(amax_kernel<0>, dim3(g), dim3(ATHREADS), 0, st, x, n, out);
+    case 16: return launch_pdl(amax_kernel<16>, dim3(g), dim3(ATHREADS), 0, st, x, n, out);
+    case 32: return launch_pdl(amax_kernel<32>, dim3(g), dim3(ATHREADS), 0, st, x, n, out);
+    case 64: return launch_pdl(amax_kernel<64>, dim3(g), dim3(ATHREADS), 0, st, x, n, out);
+    case 128: return launch_pdl(amax_kernel<128>, dim3(g), dim3(ATHREADS), 0, st, x, n, out);
     default: return cudaErrorInvalidValue;
     }
-    return e_;
 }
 
 cudaError_t launch_finalize_sg(float* g, cudaStream_t st)
@@ -247,28 +246,32 @@ __global__ void __launch_bounds__(ATHREADS) block_mse_kernel(MseArgs a)
 {
     pdl_begin();
     constexpr int NB = SEG / B;
+    constexpr int SPT = SegsPerThread<ROT>::value;
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
-    if (s - lane >= nseg)
+    const int64_t t = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if ((t - lane) * SPT >= nseg)
         return;
-    float y[SEG];
-    load_seg_bf16(a.x, a.n, s, y);
-    rotate_seg<ROT>(y, lane);
-    if (s >= nseg)
-        return;
-    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
-    uint32_t q[4], sc[NB];
-    load_codes(a.codes, s, nvalid, q);
-    load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+    float y[SPT][SEG];
+    load_rotate<ROT>(a.x, a.n, t, lane, y);
     const float sg = MX ? 1.0f : *a.sg;
-    float S[NB], sse[NB], m[NB];
-    scales_of<NB, MX>(sc, sg, S);
-    sse_seg<B>(y, q, S, sse);
 #pragma unroll
-    for (int b = 0; b < NB; ++b)
-        m[b] = __fmul_rn(sse[b], 1.0f / B);
-    store_seg_floats<NB>(a.mse, s, nvalid, B, m);
+    for (int k = 0; k < SPT; ++k) {
+        const int64_t s = t * SPT + k;
+        if (s >= nseg)
+            continue;
+        const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+        uint32_t q[4], sc[NB];
+        load_codes(a.codes, s, nvalid, q);
+        load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+        float S[NB], sse[NB], m[NB];
+        scales_of<NB, MX>(sc, sg, S);
+        sse_seg<B>(y[k], q, S, sse);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            m[b] = __fmul_rn(sse[b], 1.0f / B);
+        store_seg_floats<NB>(a.mse, s, nvalid, B, m);
+    }
 }
 
 template <int B, bool MX>
@@ -289,9 +292,10 @@ static cudaError_t launch_mse_rot(int rot, unsigned g, const MseArgs& a, cudaStr
 cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st)
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    if (!grid_ok(nseg))
+    const int64_t nthr = nseg;
+    if (!grid_ok(nthr))
         return cudaErrorInvalidValue;
-    const unsigned g = grid_for(nseg);
+    const unsigned g = grid_for(nthr);
     if (mx)
         return block == 32 ? launch_mse_rot<32, true>(rot, g, a, st) : cudaErrorInvalidValue;
     switch (block) {
@@ -369,7 +373,7 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
     uint32_t sc[NB];
     bool zb[NB];
     block_amax<B>(y, amax);
-    const float den6 = __fmul_rn(6.0f, sg);
+    const NvConsts kc = nv_consts(sg);
 #pragma unroll
     for (int b = 0; b < NB; ++b) {
         if constexpr (MX) {
@@ -377,7 +381,7 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
             sc[b] = (uint32_t)(e + 127);
             S[b] = pow2f(e);
         } else {
-            sc[b] = e4m3_enc(__fdiv_rn(amax[b], den6));
+            sc[b] = e4m3_code_of_quotient(amax[b], kc.den6, kc.rden6, kc.fast);
             S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
         }
         zb[b] = (S[b] == 0.0f);

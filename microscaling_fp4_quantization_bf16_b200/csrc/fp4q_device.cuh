@@ -66,30 +66,55 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p)
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-// Loads segment s (elements s*32 .. s*32+31) of a bf16 array of n elements,
-// widened to fp32 (exact). Elements at or beyond n read as +0.
-__device__ __forceinline__ void load_seg_bf16(const uint16_t* x, int64_t n, int64_t s, float (&y)[SEG])
+// Raw bf16 words of segment s (elements s*32 .. s*32+31) of an array of n
+// elements: element 2i in the low half of word i. Elements at or beyond n
+// read as +0. Issuing these loads early lets a kernel overlap their latency
+// with other start-up work before unpacking.
+__device__ __forceinline__ void load_seg_raw(const uint16_t* x, int64_t n, int64_t s, uint4 (&v)[4])
 {
     const int64_t base = s * SEG;
     if (base + SEG <= n) {
         const uint4* p = reinterpret_cast<const uint4*>(x + base);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            uint4 v = ldg_stream(p + k);
-            y[8 * k + 0] = bf_lo(v.x);
-            y[8 * k + 1] = bf_hi(v.x);
-            y[8 * k + 2] = bf_lo(v.y);
-            y[8 * k + 3] = bf_hi(v.y);
-            y[8 * k + 4] = bf_lo(v.z);
-            y[8 * k + 5] = bf_hi(v.z);
-            y[8 * k + 6] = bf_lo(v.w);
-            y[8 * k + 7] = bf_hi(v.w);
-        }
+        for (int k = 0; k < 4; ++k)
+            v[k] = ldg_stream(p + k);
     } else {
+        uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < SEG; ++i)
-            y[i] = (base + i < n) ? __uint_as_float((uint32_t)x[base + i] << 16) : 0.0f;
+        for (int i = 0; i < 16; ++i) {
+            const uint32_t lo = (base + 2 * i < n) ? (uint32_t)x[base + 2 * i] : 0u;
+            const uint32_t hi = (base + 2 * i + 1 < n) ? (uint32_t)x[base + 2 * i + 1] : 0u;
+            w[i] = lo | (hi << 16);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            v[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     }
+}
+
+// bf16 words -> fp32 values (exact).
+__device__ __forceinline__ void unpack_seg(const uint4 (&v)[4], float (&y)[SEG])
+{
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        y[8 * k + 0] = bf_lo(v[k].x);
+        y[8 * k + 1] = bf_hi(v[k].x);
+        y[8 * k + 2] = bf_lo(v[k].y);
+        y[8 * k + 3] = bf_hi(v[k].y);
+        y[8 * k + 4] = bf_lo(v[k].z);
+        y[8 * k + 5] = bf_hi(v[k].z);
+        y[8 * k + 6] = bf_lo(v[k].w);
+        y[8 * k + 7] = bf_hi(v[k].w);
+    }
+}
+
+// Loads segment s of a bf16 array of n elements, widened to fp32 (exact).
+// Elements at or beyond n read as +0.
+__device__ __forceinline__ void load_seg_bf16(const uint16_t* x, int64_t n, int64_t s, float (&y)[SEG])
+{
+    uint4 v[4];
+    load_seg_raw(x, n, s, v);
+    unpack_seg(v, y);
 }
 
 // ------------------------------------------------------------------ E2M1
@@ -218,6 +243,38 @@ __device__ __forceinline__ int e8m0_exp(float a)
     return max(E - 129, -127);
 }
 
+// Per-thread constants of E4M3 scale selection for target T in {6, 4}:
+// den_T = T * s_g and its correctly rounded reciprocal.
+struct NvConsts {
+    float den6, rden6, den4, rden4;
+    bool fast;  // both reciprocals finite: the quotient shortcut applies
+};
+
+__device__ __forceinline__ NvConsts nv_consts(float sg)
+{
+    NvConsts k;
+    k.den6 = __fmul_rn(6.0f, sg);
+    k.den4 = __fmul_rn(4.0f, sg);
+    k.rden6 = __frcp_rn(k.den6);
+    k.rden4 = __frcp_rn(k.den4);
+    k.fast = k.rden6 <= FLT_MAX && k.rden4 <= FLT_MAX;
+    return k;
+}
+
+// RNE_E4M3_sat(fl(a / den)) for a >= 0 without a division in almost every
+// case. q = fl(a * fl(1/den)) differs from fl(a / den) by at most a few units
+// in the last place, so the two round to different E4M3 codes only if an E4M3
+// rounding boundary (a value or midpoint of the E4M3 grid; every one has the
+// low 19 mantissa bits of its fp32 encoding zero) lies within that distance
+// of q. Those q, and overflowing or zero q, take the exact IEEE division.
+__device__ __forceinline__ uint32_t e4m3_code_of_quotient(float a, float den, float rden, bool fast)
+{
+    float q = __fmul_rn(a, rden);
+    if (!fast || ((__float_as_uint(q) + 8u) & 0x7FFFFu) < 16u)
+        q = __fdiv_rn(a, den);
+    return e4m3_enc(q);
+}
+
 // 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
 __device__ __forceinline__ float pow2f(int e)
 {
@@ -233,25 +290,79 @@ template <> struct HadK<32> { static constexpr float k = 0x1.6a09e6p-3f; };
 template <> struct HadK<64> { static constexpr float k = 0x1p-3f; };
 template <> struct HadK<128> { static constexpr float k = 0x1.6a09e6p-4f; };
 
-// Normalised Walsh-Hadamard transform of every ROT-wide chunk, stages in
-// ascending order h = 1, 2, 4, ...: butterflies with h < 32 stay inside the
-// segment; h = 32 and 64 pair lane L with lane L ^ (h / 32) (the lower lane
-// holds index i, the upper lane index i + h). All 32 lanes of the warp must
-// call this together.
+// Packed pairs of fp32 (sm_100 add/sub/mul.rn.f32x2: two IEEE round-to-
+// nearest-even operations, no flush-to-zero, one instruction).
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pk2(float lo, float hi)
+{
+    f32x2 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+
+__device__ __forceinline__ void upk2(f32x2 v, float& lo, float& hi)
+{
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+
+__device__ __forceinline__ f32x2 add2(f32x2 a, f32x2 b)
+{
+    f32x2 r;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b)
+{
+    f32x2 r;
+    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
+{
+    f32x2 r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+
+// Normalised Walsh-Hadamard transform of every ROT-wide chunk of a segment:
+// stages h = 1, 2, 4, ... in ascending order, (t[i], t[i+h]) <- (t[i]+t[i+h],
+// t[i]-t[i+h]), then one multiply by k_ROT. Stages h < 16 run on packed
+// pairs {y[i], y[i + 16]} (both lanes of one add.f32x2 are butterflies of the
+// same stage, each an IEEE round-to-nearest-even add); stage 16 is scalar;
+// h = 32 and 64 pair lane L with lane L ^ (h / 32) (the lower lane holds index
+// i, the upper lane i + h). All 32 lanes of the warp must call this together.
 template <int ROT>
 __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
 {
     if constexpr (ROT > 0) {
         constexpr int LOCAL = ROT < SEG ? ROT : SEG;
+        f32x2 P[16];
 #pragma unroll
-        for (int h = 1; h < LOCAL; h <<= 1) {
+        for (int i = 0; i < 16; ++i)
+            P[i] = pk2(y[i], y[i + 16]);
 #pragma unroll
-            for (int i = 0; i < SEG; ++i) {
+        for (int h = 1; h < (LOCAL < 16 ? LOCAL : 16); h <<= 1) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
                 if ((i & h) == 0) {
-                    float a = y[i], b = y[i + h];
-                    y[i] = __fadd_rn(a, b);
-                    y[i + h] = __fsub_rn(a, b);
+                    f32x2 a = P[i], b = P[i + h];
+                    P[i] = add2(a, b);
+                    P[i + h] = sub2(a, b);
                 }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+            upk2(P[i], y[i], y[i + 16]);
+        if constexpr (LOCAL == SEG) {  // stage 16: y[i] with y[i + 16]
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float a = y[i], b = y[i + 16];
+                y[i] = __fadd_rn(a, b);
+                y[i + 16] = __fsub_rn(a, b);
             }
         }
 #pragma unroll
@@ -264,10 +375,30 @@ __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
                 y[i] = lower ? __fadd_rn(y[i], p) : __fsub_rn(p, y[i]);
             }
         }
+        const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
 #pragma unroll
-        for (int i = 0; i < SEG; ++i)
-            y[i] = __fmul_rn(y[i], HadK<ROT>::k);
+        for (int i = 0; i < 16; ++i) {
+            f32x2 v = mul2(pk2(y[i], y[i + 16]), kk);
+            upk2(v, y[i], y[i + 16]);
+        }
     }
+}
+
+// Segments per thread (one; kept as a parameter of the kernels' indexing).
+// Two segments per thread for 64/128-wide rotations (all stages up to 32 in
+// registers) measured slower on B200 than one segment with shuffle stages.
+template <int ROT>
+struct SegsPerThread {
+    static constexpr int value = 1;
+};
+
+// Loads the segment(s) of thread t and rotates them.
+template <int ROT>
+__device__ __forceinline__ void load_rotate(const uint16_t* x, int64_t n, int64_t t, int lane,
+                                            float (&y)[SegsPerThread<ROT>::value][SEG])
+{
+    load_seg_bf16(x, n, t, y[0]);
+    rotate_seg<ROT>(y[0], lane);
 }
 
 // ------------------------------------------------------------------ blocks

@@ -22,12 +22,13 @@ namespace fp4q {
 
 constexpr int QTHREADS = 256;
 
-// Brute-force candidate tables: dequantization scale and reciprocal of every
-// E4M3 code (index 0 and 0x7F unused), built by each block.
+// Per-block-scale tables of the NVFP4 kernels, built by every block: the
+// dequantization scale S[c] = E4M3(c) * s_g and its reciprocal R[c] (the
+// zero-scale convention gives R[0] = 0) for every code c; index 0x7F unused.
 template <int STRAT>
-struct BruteTables {
-    float S[STRAT == K_BRUTE_FORCE ? 128 : 1];
-    float R[STRAT == K_BRUTE_FORCE ? 128 : 1];
+struct ScaleTables {
+    float S[STRAT == K_MX ? 1 : 128];
+    float R[STRAT == K_MX ? 1 : 128];
 };
 
 // Scale selection, encoding and stores for one 32-element segment s whose
@@ -35,7 +36,7 @@ struct BruteTables {
 template <int B, int STRAT>
 __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s, int nvalid,
                                                 const QuantArgs& a, float sg,
-                                                const BruteTables<STRAT>& tab)
+                                                const ScaleTables<STRAT>& tab)
 {
     constexpr int NB = SEG / B;
     float amax[NB];
@@ -78,29 +79,28 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
     } else {
-        const float den6 = __fmul_rn(6.0f, sg);
+        const NvConsts k = nv_consts(sg);
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            uint32_t c = e4m3_enc(__fdiv_rn(amax[b], den6));
+            uint32_t c = e4m3_code_of_quotient(amax[b], k.den6, k.rden6, k.fast);
             if constexpr (STRAT == K_PREVENT_ZERO)
                 c = max(c, 1u);
             sc[b] = c;
-            S[b] = __fmul_rn(e4m3_dec(c), sg);
+            S[b] = tab.S[c];
+            r[b] = tab.R[c];
             zero[b] = (S[b] == 0.0f);
-            r[b] = zero[b] ? 0.0f : guarded_rcp(S[b]);
         }
         encode_seg<B>(y, r, zero, a.keep, q);
         if constexpr (STRAT == K_FOUR_OVER_SIX) {
-            const float den4 = __fmul_rn(4.0f, sg);
             float S4[NB], r4[NB], sse4[NB];
             bool z4[NB];
             uint32_t c4[NB], q4[4];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-                c4[b] = e4m3_enc(__fdiv_rn(amax[b], den4));
-                S4[b] = __fmul_rn(e4m3_dec(c4[b]), sg);
+                c4[b] = e4m3_code_of_quotient(amax[b], k.den4, k.rden4, k.fast);
+                S4[b] = tab.S[c4[b]];
+                r4[b] = tab.R[c4[b]];
                 z4[b] = (S4[b] == 0.0f);
-                r4[b] = z4[b] ? 0.0f : guarded_rcp(S4[b]);
             }
             encode_seg<B>(y, r4, z4, a.keep, q4);
             sse_seg<B>(y, q, S, sse);
@@ -175,11 +175,11 @@ __device__ __forceinline__ float kernel_global_scale(const QuantArgs& a)
 }
 
 template <int STRAT>
-__device__ __forceinline__ void build_brute_tables(BruteTables<STRAT>& tab, float sg)
+__device__ __forceinline__ void build_scale_tables(ScaleTables<STRAT>& tab, float sg)
 {
-    if constexpr (STRAT == K_BRUTE_FORCE) {
+    if constexpr (STRAT != K_MX) {
         for (int c = threadIdx.x; c < 128; c += blockDim.x) {
-            float S = (c >= 1 && c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
+            float S = (c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
             tab.S[c] = S;
             tab.R[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
         }
@@ -187,9 +187,9 @@ __device__ __forceinline__ void build_brute_tables(BruteTables<STRAT>& tab, floa
     }
 }
 
-// Direct-load kernel: one segment per thread, four 128-bit global loads.
-// Used for the brute-force search (compute bound) and for tensors the TMA
-// kernel does not take (a flattened length that is not a multiple of 64).
+// Direct-load kernel: one segment per thread (two for 64/128-wide
+// rotations), 128-bit global loads. Used by default, and for the brute-force
+// search (compute bound) and flattened lengths that are not a multiple of 64.
 template <int B, int ROT, int STRAT>
 __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
 {
@@ -197,32 +197,35 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
-    const float sg = kernel_global_scale<STRAT>(a);
-    __shared__ BruteTables<STRAT> tab;
-    build_brute_tables<STRAT>(tab, sg);
+    const bool warp_active = s - lane < nseg;  // warp-uniform
 
-    if (s - lane >= nseg)
-        return;  // the whole warp is past the end (warp-uniform)
-    float y[SEG];
-    load_seg_bf16(a.x, a.n, s, y);  // lanes past the end read zeros
-    rotate_seg<ROT>(y, lane);       // all 32 lanes take part
-    if (s >= nseg)
+    uint4 raw[4];
+    if (warp_active)
+        load_seg_raw(a.x, a.n, s, raw);  // in flight while the tables are built
+    const float sg = kernel_global_scale<STRAT>(a);
+    __shared__ ScaleTables<STRAT> tab;
+    build_scale_tables<STRAT>(tab, sg);
+    if (!warp_active)
         return;
-    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
-    process_segment<B, STRAT>(y, s, nvalid, a, sg, tab);
+
+    float y[SEG];
+    unpack_seg(raw, y);
+    rotate_seg<ROT>(y, lane);  // all 32 lanes take part; past the end holds zeros
+    if (s < nseg)
+        process_segment<B, STRAT>(y, s, (int)min((int64_t)SEG, a.n - s * SEG), a, sg, tab);
 }
 
 template <int B>
 cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream_t st)
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t nblk = (nseg + QTHREADS - 1) / QTHREADS;
-    if (nblk <= 0 || nblk > 0x7FFFFFFF)
-        return cudaErrorInvalidValue;
-    const dim3 grid((unsigned)nblk);
-#define FP4Q_QCASE(S_, R_)                                        \
-    if (strat == S_ && rot == R_) {                               \
-        return launch_pdl(quant_kernel<B, R_, S_>, grid, dim3(QTHREADS), 0, st, a); \
+#define FP4Q_QCASE(S_, R_)                                                              \
+    if (strat == S_ && rot == R_) {                                                     \
+        constexpr int64_t per_block = (int64_t)QTHREADS;                                \
+        const int64_t nblk = (nseg + per_block - 1) / per_block;                        \
+        if (nblk <= 0 || nblk > 0x7FFFFFFF)                                             \
+            return cudaErrorInvalidValue;                                               \
+        return launch_pdl(quant_kernel<B, R_, S_>, dim3((unsigned)nblk), dim3(QTHREADS), 0, st, a); \
     }
 #define FP4Q_QROTS(S_)      \
     FP4Q_QCASE(S_, 0)       \

@@ -95,6 +95,8 @@ __global__ void __launch_bounds__(TTHREADS)
 
     pdl_begin();
     const float sg = kernel_global_scale<STRAT>(a);
+    __shared__ ScaleTables<STRAT> tab;
+    build_scale_tables<STRAT>(tab, sg);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_addr(full + s), 1);
@@ -130,7 +132,6 @@ __global__ void __launch_bounds__(TTHREADS)
     const int row = c >> 1;
     const int half = c & 1;
     const int64_t nseg = a.n / SEG;
-    BruteTables<STRAT> no_tables;
     int it = 0;
     for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
         const int stage = it % STAGES;
@@ -164,7 +165,7 @@ __global__ void __launch_bounds__(TTHREADS)
         rotate_seg<ROT>(y, lane);  // 64/128-wide chunks: neighbouring lanes of this warp
         const int64_t s = tile * TILE_SEGS + c;
         if (s < nseg)  // rows past the end were zero-filled by TMA
-            process_segment<B, STRAT>(y, s, SEG, a, sg, no_tables);
+            process_segment<B, STRAT>(y, s, SEG, a, sg, tab);
     }
 }
 
