@@ -439,9 +439,101 @@ __device__ __forceinline__ float tree_sum(float* e)
 // straight out of e2m1_pack8, with no intervening run-time operation, was
 // measured on sm_100a to return 0 for the elements held in bytes 2 and 3.
 template <int B>
-__device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&r)[SEG / B],
+__device__ __forceinline__ void encode_seg_packed(const float (&y)[SEG], const float (&r)[SEG / B],
                                            const bool (&zero)[SEG / B], uint32_t keep,
                                            uint32_t (&q)[4])
+{
+    // u = y * r on packed pairs {i, i + 16}
+    float u[SEG];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        f32x2 U = mul2(pk2(y[i], y[i + 16]), pk2(r[i / B], r[(i + 16) / B]));
+        upk2(U, u[i], u[i + 16]);
+    }
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t qw = e2m1_pack8(u + 8 * w);
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (zero[(8 * w + j) / B])
+                m |= 0xFu << (4 * j);
+        q[w] = qw & (keep & ~m);
+    }
+}
+
+// Dequantized values of the segment: value(code) * S(block).
+template <int B>
+__device__ __forceinline__ void decode_seg(const uint32_t (&q)[4], const float (&S)[SEG / B],
+                                           float (&yh)[SEG])
+{
+    float v[SEG];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+        e2m1_unpack8(q[w], v + 8 * w);
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        f32x2 Y = mul2(pk2(v[i], v[i + 16]), pk2(S[i / B], S[(i + 16) / B]));
+        upk2(Y, yh[i], yh[i + 16]);
+    }
+}
+
+// Per-block SSE of y against value(code) * S, tree-summed. Values are formed
+// on packed pairs {i, i + 16}: for B <= 16 the two lanes of E[g*B .. g*B + B)
+// hold two whole blocks (g and g + 16/B) whose adjacent-pair trees run in
+// lockstep; for B = 32 the packed tree yields the two half sums and the last
+// level adds them, which is the same tree.
+//
+// ptxas fuses a packed multiply (mul.rn.f32x2, and even fma.rn.f32x2 with a
+// -0 addend) into a following packed add/sub although .rn and -fmad=false
+// forbid contraction; measured on sm_100a it changed low bits. A packed
+// product is therefore always consumed first by a scalar __fsub_rn /
+// __fadd_rn, which are never contracted: d = y - yhat and the first tree level.
+template <int B>
+__device__ __forceinline__ void sse_seg_packed(const float (&y)[SEG], const uint32_t (&q)[4],
+                                        const float (&S)[SEG / B], float (&sse)[SEG / B])
+{
+    float v[SEG];
+#pragma unroll
+    for (int w = 0; w < 4; ++w)
+        e2m1_unpack8(q[w], v + 8 * w);
+    float e[SEG];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        float h0, h1, d0, d1;
+        upk2(mul2(pk2(v[i], v[i + 16]), pk2(S[i / B], S[(i + 16) / B])), h0, h1);
+        d0 = __fsub_rn(y[i], h0);
+        d1 = __fsub_rn(y[i + 16], h1);
+        upk2(mul2(pk2(d0, d1), pk2(d0, d1)), e[i], e[i + 16]);
+    }
+    f32x2 E[8];  // tree level h = 1, scalar: E[j] = {e[2j] + e[2j+1], e[2j+16] + e[2j+17]}
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        E[j] = pk2(__fadd_rn(e[2 * j], e[2 * j + 1]), __fadd_rn(e[2 * j + 16], e[2 * j + 17]));
+    constexpr int G = B < 16 ? B : 16;  // packed tree width (elements)
+#pragma unroll
+    for (int h = 1; h < G / 2; h <<= 1) {  // levels 2 .. G/2 on the half-length array
+#pragma unroll
+        for (int j = 0; j + h < 8; j += 2 * h)
+            E[j] = add2(E[j], E[j + h]);
+    }
+    if constexpr (B == 32) {
+        float lo, hi;
+        upk2(E[0], lo, hi);
+        sse[0] = __fadd_rn(lo, hi);
+    } else {
+#pragma unroll
+        for (int g = 0; g < 16 / B; ++g)
+            upk2(E[g * B / 2], sse[g], sse[g + 16 / B]);
+    }
+}
+
+// Scalar forms of encode_seg and sse_seg (one IEEE operation per element
+// and step); the packed forms above compute the same bits.
+template <int B>
+__device__ __forceinline__ void encode_seg_scalar(const float (&y)[SEG], const float (&r)[SEG / B],
+                                                  const bool (&zero)[SEG / B], uint32_t keep,
+                                                  uint32_t (&q)[4])
 {
 #pragma unroll
     for (int w = 0; w < 4; ++w) {
@@ -459,25 +551,9 @@ __device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&
     }
 }
 
-// Dequantized values of the segment: value(code) * S(block).
 template <int B>
-__device__ __forceinline__ void decode_seg(const uint32_t (&q)[4], const float (&S)[SEG / B],
-                                           float (&yh)[SEG])
-{
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        float v[8];
-        e2m1_unpack8(q[w], v);
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            yh[8 * w + j] = __fmul_rn(v[j], S[(8 * w + j) / B]);
-    }
-}
-
-// Per-block SSE of y against value(code) * S, tree-summed.
-template <int B>
-__device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&q)[4],
-                                        const float (&S)[SEG / B], float (&sse)[SEG / B])
+__device__ __forceinline__ void sse_seg_scalar(const float (&y)[SEG], const uint32_t (&q)[4],
+                                               const float (&S)[SEG / B], float (&sse)[SEG / B])
 {
     float e[SEG];
 #pragma unroll
@@ -487,14 +563,42 @@ __device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const int i = 8 * w + j;
-            float yh = __fmul_rn(v[j], S[i / B]);
-            float d = __fsub_rn(y[i], yh);
+            float d = __fsub_rn(y[i], __fmul_rn(v[j], S[i / B]));
             e[i] = __fmul_rn(d, d);
         }
     }
 #pragma unroll
     for (int b = 0; b < SEG / B; ++b)
         sse[b] = tree_sum<B>(e + b * B);
+}
+
+// Selected forms (both compute the same bits).
+#ifndef FP4Q_PACKED_ENCODE
+#define FP4Q_PACKED_ENCODE 0
+#endif
+#ifndef FP4Q_PACKED_SSE
+#define FP4Q_PACKED_SSE 1
+#endif
+
+template <int B>
+__device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&r)[SEG / B],
+                                           const bool (&zero)[SEG / B], uint32_t keep,
+                                           uint32_t (&q)[4])
+{
+    if constexpr (FP4Q_PACKED_ENCODE)
+        encode_seg_packed<B>(y, r, zero, keep, q);
+    else
+        encode_seg_scalar<B>(y, r, zero, keep, q);
+}
+
+template <int B>
+__device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&q)[4],
+                                        const float (&S)[SEG / B], float (&sse)[SEG / B])
+{
+    if constexpr (FP4Q_PACKED_SSE)
+        sse_seg_packed<B>(y, q, S, sse);
+    else
+        sse_seg_scalar<B>(y, q, S, sse);
 }
 
 // SSE of one B-wide block yb against value(RNE_E2M1(yb * r)) * S (`keep` as
