@@ -365,14 +365,17 @@ __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
                 y[i + 16] = __fsub_rn(a, b);
             }
         }
+        // Cross-lane stages: the lower lane needs p + v, the upper p - v (p the
+        // partner's value, v its own). fma(s, v, p) with s = +1 / -1 forms s*v
+        // exactly and rounds once, so it equals that add / subtract bit for bit.
 #pragma unroll
         for (int h = SEG; h < ROT; h <<= 1) {
             const int lm = h / SEG;
-            const bool lower = (lane & lm) == 0;
+            const float sgn = (lane & lm) == 0 ? 1.0f : -1.0f;
 #pragma unroll
             for (int i = 0; i < SEG; ++i) {
                 float p = __shfl_xor_sync(0xFFFFFFFFu, y[i], lm);
-                y[i] = lower ? __fadd_rn(y[i], p) : __fsub_rn(p, y[i]);
+                y[i] = __fmaf_rn(sgn, y[i], p);
             }
         }
         const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
