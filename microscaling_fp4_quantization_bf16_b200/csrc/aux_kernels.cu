@@ -196,47 +196,83 @@ __device__ __forceinline__ void store_seg_floats(float* p, int64_t s, int nvalid
 
 // ------------------------------------------------------------ dequantize
 
-template <int B, bool MX>
+// One thread per EPT consecutive elements (EPT = 8 for bf16 output, 4 for
+// fp32): its 16 output bytes are one store, and a warp's stores cover 512
+// contiguous bytes. A thread's elements lie in one block unless B = 4 < EPT.
+template <int B, bool MX, int EPT>
 __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 {
     pdl_begin();
-    constexpr int NB = SEG / B;
-    const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
-    if (s >= nseg)
+    constexpr int NS = EPT > B ? EPT / B : 1;  // scale bytes per thread
+    const int64_t t = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    const int64_t e0 = t * EPT;
+    if (e0 >= a.n)
         return;
-    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
-    uint32_t q[4], sc[NB];
-    load_codes(a.codes, s, nvalid, q);
-    load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+    const int nvalid = (int)min((int64_t)EPT, a.n - e0);  // a multiple of 4
+    uint32_t q;
+    if (EPT == 8 && nvalid == 8)
+        q = *reinterpret_cast<const uint32_t*>(a.codes + e0 / 2);
+    else
+        q = *reinterpret_cast<const uint16_t*>(a.codes + e0 / 2);
+    uint32_t sc[NS];
+#pragma unroll
+    for (int k = 0; k < NS; ++k)
+        sc[k] = (k * B < nvalid) ? (uint32_t)a.scales[e0 / B + k] : 0u;
     const float sg = MX ? 1.0f : *a.sg;
-    float S[NB], yh[SEG];
-    scales_of<NB, MX>(sc, sg, S);
-    decode_seg<B>(q, S, yh);
-    store_seg_values(a.out, a.out_kind, s, nvalid, yh);
+    float S[NS];
+    scales_of<NS, MX>(sc, sg, S);
+    float v[EPT];
+    if constexpr (EPT == 8)
+        e2m1_unpack8(q, v);
+    else
+        e2m1_unpack4(q, v);
+    float yh[EPT];
+#pragma unroll
+    for (int j = 0; j < EPT / 2; ++j) {
+        const f32x2 Y = mul2(pk2(v[2 * j], v[2 * j + 1]), pk2(S[(2 * j) / B], S[(2 * j + 1) / B]));
+        upk2(Y, yh[2 * j], yh[2 * j + 1]);
+    }
+    if constexpr (EPT == 8) {  // bf16
+        uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + e0;
+        uint4 w;
+        w.x = pack_bf16x2(yh[0], yh[1]);
+        w.y = pack_bf16x2(yh[2], yh[3]);
+        w.z = pack_bf16x2(yh[4], yh[5]);
+        w.w = pack_bf16x2(yh[6], yh[7]);
+        if (nvalid == 8)
+            *reinterpret_cast<uint4*>(o) = w;
+        else
+            *reinterpret_cast<uint2*>(o) = make_uint2(w.x, w.y);
+    } else {  // fp32
+        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + e0) =
+            make_float4(yh[0], yh[1], yh[2], yh[3]);
+    }
+}
+
+template <int B, bool MX>
+static cudaError_t launch_dequant_b(const DequantArgs& a, cudaStream_t st)
+{
+    const int ept = a.out_kind == 2 ? 8 : 4;
+    const int64_t nthr = (a.n + ept - 1) / ept;
+    if (!grid_ok(nthr))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nthr);
+    if (ept == 8)
+        return launch_pdl(dequant_kernel<B, MX, 8>, dim3(g), dim3(ATHREADS), 0, st, a);
+    return launch_pdl(dequant_kernel<B, MX, 4>, dim3(g), dim3(ATHREADS), 0, st, a);
 }
 
 cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st)
 {
-    cudaError_t e_ = cudaSuccess;
-    const int64_t nseg = (a.n + SEG - 1) / SEG;
-    if (!grid_ok(nseg))
-        return cudaErrorInvalidValue;
-    const unsigned g = grid_for(nseg);
-    if (mx) {
-        if (block != 32)
-            return cudaErrorInvalidValue;
-        e_ = launch_pdl(dequant_kernel<32, true>, dim3(g), dim3(ATHREADS), 0, st, a);
-    } else {
-        switch (block) {
-        case 4: e_ = launch_pdl(dequant_kernel<4, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-        case 8: e_ = launch_pdl(dequant_kernel<8, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-        case 16: e_ = launch_pdl(dequant_kernel<16, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-        case 32: e_ = launch_pdl(dequant_kernel<32, false>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-        default: return cudaErrorInvalidValue;
-        }
+    if (mx)
+        return block == 32 ? launch_dequant_b<32, true>(a, st) : cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_dequant_b<4, false>(a, st);
+    case 8: return launch_dequant_b<8, false>(a, st);
+    case 16: return launch_dequant_b<16, false>(a, st);
+    case 32: return launch_dequant_b<32, false>(a, st);
+    default: return cudaErrorInvalidValue;
     }
-    return e_;
 }
 
 // ------------------------------------------------------------ block MSE
@@ -348,6 +384,8 @@ __device__ __forceinline__ void load_coeffs(const uint16_t* c, int64_t s, int nv
 }
 
 // W_hat = S_dq * Q(W / (S_dq * c_k)), S_dq the format's abs-max block scale.
+// (Every thread derives s_g itself: a per-CTA table and barrier, as in the
+// quantize kernel, measured slower for this one-segment-per-thread kernel.)
 template <int B, int SUB, bool MX>
 __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
 {
@@ -373,19 +411,23 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
     uint32_t sc[NB];
     bool zb[NB];
     block_amax<B>(y, amax);
-    const NvConsts kc = nv_consts(sg);
+    if constexpr (MX) {
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        if constexpr (MX) {
+        for (int b = 0; b < NB; ++b) {
             const int e = e8m0_exp(amax[b]);
             sc[b] = (uint32_t)(e + 127);
             S[b] = pow2f(e);
-        } else {
-            sc[b] = e4m3_code_of_quotient(amax[b], kc.den6, kc.rden6, kc.fast);
-            S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
         }
-        zb[b] = (S[b] == 0.0f);
+    } else {
+        const NvConsts kc = nv_consts(sg);
+        e4m3_codes_of_quotients<NB>(amax, kc.den6, kc.rden6, kc.fast, sc);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
     }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        zb[b] = (S[b] == 0.0f);
     float r[NK];
     bool zk[NK];
 #pragma unroll

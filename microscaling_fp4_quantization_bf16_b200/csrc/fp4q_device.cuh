@@ -261,18 +261,40 @@ __device__ __forceinline__ NvConsts nv_consts(float sg)
     return k;
 }
 
-// RNE_E4M3_sat(fl(a / den)) for a >= 0 without a division in almost every
-// case. q = fl(a * fl(1/den)) differs from fl(a / den) by at most a few units
-// in the last place, so the two round to different E4M3 codes only if an E4M3
+// Scale codes RNE_E4M3_sat(fl(a / den)), a >= 0, mostly without a division:
+// q = fl(a * fl(1/den)) differs from fl(a / den) by at most a few units in
+// the last place, so the two round to different E4M3 codes only if an E4M3
 // rounding boundary (a value or midpoint of the E4M3 grid; every one has the
 // low 19 mantissa bits of its fp32 encoding zero) lies within that distance
-// of q. Those q, and overflowing or zero q, take the exact IEEE division.
-__device__ __forceinline__ uint32_t e4m3_code_of_quotient(float a, float den, float rden, bool fast)
+// of q. quotient_flagged marks those q, and overflowing or zero q, for the
+// exact IEEE division -- except q = +0 from a = +0, which the division also
+// gives (den > 0).
+__device__ __forceinline__ bool quotient_flagged(float q, float a)
 {
-    float q = __fmul_rn(a, rden);
-    if (!fast || ((__float_as_uint(q) + 8u) & 0x7FFFFu) < 16u)
-        q = __fdiv_rn(a, den);
-    return e4m3_enc(q);
+    return ((__float_as_uint(q) + 8u) & 0x7FFFFu) < 16u && a != 0.0f;
+}
+
+// The codes of NB quotients a[b] / den at once: one exact division pass for
+// all of them if any shortcut quotient is flagged.
+template <int NB>
+__device__ __forceinline__ void e4m3_codes_of_quotients(const float (&a)[NB], float den, float rden,
+                                                        bool fast, uint32_t (&c)[NB])
+{
+    float q[NB];
+    bool slow = !fast;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        q[b] = __fmul_rn(a[b], rden);
+        slow |= quotient_flagged(q[b], a[b]);
+    }
+    if (slow) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            q[b] = __fdiv_rn(a[b], den);
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        c[b] = e4m3_enc(q[b]);
 }
 
 // 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
@@ -327,13 +349,26 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
     return r;
 }
 
+__device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
+{
+    f32x2 r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+
 // Normalised Walsh-Hadamard transform of every ROT-wide chunk of a segment:
 // stages h = 1, 2, 4, ... in ascending order, (t[i], t[i+h]) <- (t[i]+t[i+h],
-// t[i]-t[i+h]), then one multiply by k_ROT. Stages h < 16 run on packed
-// pairs {y[i], y[i + 16]} (both lanes of one add.f32x2 are butterflies of the
-// same stage, each an IEEE round-to-nearest-even add); stage 16 is scalar;
-// h = 32 and 64 pair lane L with lane L ^ (h / 32) (the lower lane holds index
-// i, the upper lane i + h). All 32 lanes of the warp must call this together.
+// t[i]-t[i+h]), then one multiply by k_ROT. All stages run on packed pairs
+// P[i] = {y[i], y[i + 16]}:
+//  - h < 16: both lanes of one add.f32x2 / sub.f32x2 are butterflies of the
+//    same stage;
+//  - h = 16 pairs the two lanes of P[i]: fma(P, {1, -1}, {y[i+16], y[i]})
+//    gives {y[i] + y[i+16], y[i] - y[i+16]}, each product exact and the sum
+//    rounded once, so bit for bit the add and the subtract;
+//  - h = 32, 64 pair lane L with lane L ^ (h / 32): the lower lane needs
+//    p + v, the upper p - v (p the partner's value, v its own), again one
+//    exact product and one rounding: fma(+-1, v, p).
+// All 32 lanes of the warp must call this together.
 template <int ROT>
 __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
 {
@@ -354,36 +389,33 @@ __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
                 }
             }
         }
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-            upk2(P[i], y[i], y[i + 16]);
-        if constexpr (LOCAL == SEG) {  // stage 16: y[i] with y[i + 16]
+        if constexpr (LOCAL == SEG) {  // stage 16
+            const f32x2 pm = pk2(1.0f, -1.0f);
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                float a = y[i], b = y[i + 16];
-                y[i] = __fadd_rn(a, b);
-                y[i + 16] = __fsub_rn(a, b);
+                float lo, hi;
+                upk2(P[i], lo, hi);
+                P[i] = fma2(P[i], pm, pk2(hi, lo));
             }
         }
-        // Cross-lane stages: the lower lane needs p + v, the upper p - v (p the
-        // partner's value, v its own). fma(s, v, p) with s = +1 / -1 forms s*v
-        // exactly and rounds once, so it equals that add / subtract bit for bit.
 #pragma unroll
         for (int h = SEG; h < ROT; h <<= 1) {
             const int lm = h / SEG;
             const float sgn = (lane & lm) == 0 ? 1.0f : -1.0f;
+            const f32x2 ss = pk2(sgn, sgn);
 #pragma unroll
-            for (int i = 0; i < SEG; ++i) {
-                float p = __shfl_xor_sync(0xFFFFFFFFu, y[i], lm);
-                y[i] = __fmaf_rn(sgn, y[i], p);
+            for (int i = 0; i < 16; ++i) {
+                float lo, hi;
+                upk2(P[i], lo, hi);
+                const float plo = __shfl_xor_sync(0xFFFFFFFFu, lo, lm);
+                const float phi = __shfl_xor_sync(0xFFFFFFFFu, hi, lm);
+                P[i] = fma2(ss, P[i], pk2(plo, phi));
             }
         }
         const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            f32x2 v = mul2(pk2(y[i], y[i + 16]), kk);
-            upk2(v, y[i], y[i + 16]);
-        }
+        for (int i = 0; i < 16; ++i)
+            upk2(mul2(P[i], kk), y[i], y[i + 16]);
     }
 }
 
@@ -446,22 +478,26 @@ __device__ __forceinline__ void encode_seg_packed(const float (&y)[SEG], const f
                                            const bool (&zero)[SEG / B], uint32_t keep,
                                            uint32_t (&q)[4])
 {
-    // u = y * r on packed pairs {i, i + 16}
-    float u[SEG];
+    // u = y * r on packed pairs {i, i + 16}: words w and w + 2 together
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-        f32x2 U = mul2(pk2(y[i], y[i + 16]), pk2(r[i / B], r[(i + 16) / B]));
-        upk2(U, u[i], u[i + 16]);
-    }
+    for (int w = 0; w < 2; ++w) {
+        float u[8], v[8];
 #pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t qw = e2m1_pack8(u + 8 * w);
-        uint32_t m = 0;
+        for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;
+            f32x2 U = mul2(pk2(y[i], y[i + 16]), pk2(r[i / B], r[(i + 16) / B]));
+            upk2(U, u[j], v[j]);
+        }
+        uint32_t m0 = 0, m1 = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
+        for (int j = 0; j < 8; ++j) {
             if (zero[(8 * w + j) / B])
-                m |= 0xFu << (4 * j);
-        q[w] = qw & (keep & ~m);
+                m0 |= 0xFu << (4 * j);
+            if (zero[(8 * w + 16 + j) / B])
+                m1 |= 0xFu << (4 * j);
+        }
+        q[w] = e2m1_pack8(u) & (keep & ~m0);
+        q[w + 2] = e2m1_pack8(v) & (keep & ~m1);
     }
 }
 
@@ -575,7 +611,9 @@ __device__ __forceinline__ void sse_seg_scalar(const float (&y)[SEG], const uint
         sse[b] = tree_sum<B>(e + b * B);
 }
 
-// Selected forms (both compute the same bits).
+// Selected forms (both compute the same bits). The packed encode measured
+// faster in the MXFP4 kernel and slower in the NVFP4 ones (register
+// pressure), so the quantize kernel picks it per format.
 #ifndef FP4Q_PACKED_ENCODE
 #define FP4Q_PACKED_ENCODE 0
 #endif
@@ -583,12 +621,12 @@ __device__ __forceinline__ void sse_seg_scalar(const float (&y)[SEG], const uint
 #define FP4Q_PACKED_SSE 1
 #endif
 
-template <int B>
+template <int B, bool PACKED = FP4Q_PACKED_ENCODE>
 __device__ __forceinline__ void encode_seg(const float (&y)[SEG], const float (&r)[SEG / B],
                                            const bool (&zero)[SEG / B], uint32_t keep,
                                            uint32_t (&q)[4])
 {
-    if constexpr (FP4Q_PACKED_ENCODE)
+    if constexpr (PACKED)
         encode_seg_packed<B>(y, r, zero, keep, q);
     else
         encode_seg_scalar<B>(y, r, zero, keep, q);

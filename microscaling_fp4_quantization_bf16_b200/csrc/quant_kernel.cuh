@@ -22,21 +22,22 @@ namespace fp4q {
 
 constexpr int QTHREADS = 256;
 
-// Per-block-scale tables of the NVFP4 kernels, built by every block: the
+// Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
 // dequantization scale S[c] = E4M3(c) * s_g and its reciprocal R[c] (the
-// zero-scale convention gives R[0] = 0) for every code c; index 0x7F unused.
+// zero-scale convention gives R[0] = 0) for every code c (index 0x7F unused),
+// and the scale-selection constants of s_g.
 template <int STRAT>
 struct ScaleTables {
     float S[STRAT == K_MX ? 1 : 128];
     float R[STRAT == K_MX ? 1 : 128];
+    NvConsts k;
 };
 
 // Scale selection, encoding and stores for one 32-element segment s whose
 // (rotated) values are y. nvalid < 32 only for the last segment.
 template <int B, int STRAT>
 __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s, int nvalid,
-                                                const QuantArgs& a, float sg,
-                                                const ScaleTables<STRAT>& tab)
+                                                const QuantArgs& a, const ScaleTables<STRAT>& tab)
 {
     constexpr int NB = SEG / B;
     float amax[NB];
@@ -56,7 +57,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             r[b] = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
             zero[b] = false;
         }
-        encode_seg<B>(y, r, zero, a.keep, q);
+        encode_seg<B, true>(y, r, zero, a.keep, q);  // packed: measured faster here
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
         static_for<NB>([&](auto bi) {
             constexpr int b = decltype(bi)::value;
@@ -79,10 +80,32 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
     } else {
-        const NvConsts k = nv_consts(sg);
+        // Quotients a_b / (T s_g) for the targets T in use, by the reciprocal
+        // shortcut; one exact division pass if any of them is flagged.
+        const NvConsts k = tab.k;
+        constexpr bool FOUR = STRAT == K_FOUR_OVER_SIX;
+        float q6[NB], q4[NB];
+        bool slow = !k.fast;
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            uint32_t c = e4m3_code_of_quotient(amax[b], k.den6, k.rden6, k.fast);
+            q6[b] = __fmul_rn(amax[b], k.rden6);
+            slow |= quotient_flagged(q6[b], amax[b]);
+            if constexpr (FOUR) {
+                q4[b] = __fmul_rn(amax[b], k.rden4);
+                slow |= quotient_flagged(q4[b], amax[b]);
+            }
+        }
+        if (slow) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                q6[b] = __fdiv_rn(amax[b], k.den6);
+                if constexpr (FOUR)
+                    q4[b] = __fdiv_rn(amax[b], k.den4);
+            }
+        }
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            uint32_t c = e4m3_enc(q6[b]);
             if constexpr (STRAT == K_PREVENT_ZERO)
                 c = max(c, 1u);
             sc[b] = c;
@@ -91,20 +114,20 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             zero[b] = (S[b] == 0.0f);
         }
         encode_seg<B>(y, r, zero, a.keep, q);
-        if constexpr (STRAT == K_FOUR_OVER_SIX) {
+        if constexpr (FOUR) {
             float S4[NB], r4[NB], sse4[NB];
             bool z4[NB];
-            uint32_t c4[NB], q4[4];
+            uint32_t c4[NB], q4w[4];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-                c4[b] = e4m3_code_of_quotient(amax[b], k.den4, k.rden4, k.fast);
+                c4[b] = e4m3_enc(q4[b]);
                 S4[b] = tab.S[c4[b]];
                 r4[b] = tab.R[c4[b]];
                 z4[b] = (S4[b] == 0.0f);
             }
-            encode_seg<B>(y, r4, z4, a.keep, q4);
+            encode_seg<B>(y, r4, z4, a.keep, q4w);
             sse_seg<B>(y, q, S, sse);
-            sse_seg<B>(y, q4, S4, sse4);
+            sse_seg<B>(y, q4w, S4, sse4);
 #pragma unroll
             for (int w = 0; w < 4; ++w) {
                 uint32_t m = 0;
@@ -112,7 +135,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
                 for (int j = 0; j < 8; ++j)
                     if (sse4[(8 * w + j) / B] < sse[(8 * w + j) / B])
                         m |= 0xFu << (4 * j);
-                q[w] = (q[w] & ~m) | (q4[w] & m);
+                q[w] = (q[w] & ~m) | (q4w[w] & m);
             }
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
@@ -160,28 +183,26 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
     }
 }
 
-// Global scale s_g for NVFP4 kernels (1 for MXFP4); thread 0 of block 0
-// publishes it when asked.
+// Builds the CTA's scale tables (NVFP4 kernels; nothing for MXFP4): threads
+// 0..127 each compute s_g from the global abs-max and one table entry; thread
+// 0 also the scale-selection constants and, in CTA 0, publishes s_g when
+// asked. Ends with a CTA barrier.
 template <int STRAT>
-__device__ __forceinline__ float kernel_global_scale(const QuantArgs& a)
-{
-    float sg = 1.0f;
-    if constexpr (STRAT != K_MX) {
-        sg = global_scale_of(*a.amax);
-        if (a.sg_out != nullptr && blockIdx.x == 0 && threadIdx.x == 0)
-            *a.sg_out = sg;
-    }
-    return sg;
-}
-
-template <int STRAT>
-__device__ __forceinline__ void build_scale_tables(ScaleTables<STRAT>& tab, float sg)
+__device__ __forceinline__ void build_scale_tables(ScaleTables<STRAT>& tab, const QuantArgs& a)
 {
     if constexpr (STRAT != K_MX) {
-        for (int c = threadIdx.x; c < 128; c += blockDim.x) {
-            float S = (c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
-            tab.S[c] = S;
-            tab.R[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
+        if (threadIdx.x < 128) {
+            const float sg = global_scale_of(*a.amax);
+            for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+                const float S = (c <= 0x7E) ? __fmul_rn(e4m3_dec((uint32_t)c), sg) : 0.0f;
+                tab.S[c] = S;
+                tab.R[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
+            }
+            if (threadIdx.x == 0) {
+                tab.k = nv_consts(sg);
+                if (a.sg_out != nullptr && blockIdx.x == 0)
+                    *a.sg_out = sg;
+            }
         }
         __syncthreads();
     }
@@ -202,9 +223,8 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
     uint4 raw[4];
     if (warp_active)
         load_seg_raw(a.x, a.n, s, raw);  // in flight while the tables are built
-    const float sg = kernel_global_scale<STRAT>(a);
     __shared__ ScaleTables<STRAT> tab;
-    build_scale_tables<STRAT>(tab, sg);
+    build_scale_tables<STRAT>(tab, a);
     if (!warp_active)
         return;
 
@@ -212,7 +232,7 @@ __global__ void __launch_bounds__(QTHREADS) quant_kernel(QuantArgs a)
     unpack_seg(raw, y);
     rotate_seg<ROT>(y, lane);  // all 32 lanes take part; past the end holds zeros
     if (s < nseg)
-        process_segment<B, STRAT>(y, s, (int)min((int64_t)SEG, a.n - s * SEG), a, sg, tab);
+        process_segment<B, STRAT>(y, s, (int)min((int64_t)SEG, a.n - s * SEG), a, tab);
 }
 
 template <int B>

@@ -94,9 +94,8 @@ __global__ void __launch_bounds__(TTHREADS)
     const int lane = threadIdx.x & 31;
 
     pdl_begin();
-    const float sg = kernel_global_scale<STRAT>(a);
     __shared__ ScaleTables<STRAT> tab;
-    build_scale_tables<STRAT>(tab, sg);
+    build_scale_tables<STRAT>(tab, a);
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_addr(full + s), 1);
@@ -165,7 +164,7 @@ __global__ void __launch_bounds__(TTHREADS)
         rotate_seg<ROT>(y, lane);  // 64/128-wide chunks: neighbouring lanes of this warp
         const int64_t s = tile * TILE_SEGS + c;
         if (s < nseg)  // rows past the end were zero-filled by TMA
-            process_segment<B, STRAT>(y, s, SEG, a, sg, tab);
+            process_segment<B, STRAT>(y, s, SEG, a, tab);
     }
 }
 
