@@ -420,7 +420,13 @@ __global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
         }
     } else {
         const NvConsts kc = nv_consts(sg);
-        e4m3_codes_of_quotients<NB>(amax, kc.den6, kc.rden6, kc.fast, sc);
+        float qd[NB], qr[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            qd[b] = kc.den6;
+            qr[b] = kc.rden6;
+        }
+        e4m3_quotient_codes<NB>(amax, qd, qr, kc.fast, sc);
 #pragma unroll
         for (int b = 0; b < NB; ++b)
             S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);

@@ -261,42 +261,6 @@ __device__ __forceinline__ NvConsts nv_consts(float sg)
     return k;
 }
 
-// Scale codes RNE_E4M3_sat(fl(a / den)), a >= 0, mostly without a division:
-// q = fl(a * fl(1/den)) differs from fl(a / den) by at most a few units in
-// the last place, so the two round to different E4M3 codes only if an E4M3
-// rounding boundary (a value or midpoint of the E4M3 grid; every one has the
-// low 19 mantissa bits of its fp32 encoding zero) lies within that distance
-// of q. quotient_flagged marks those q, and overflowing or zero q, for the
-// exact IEEE division -- except q = +0 from a = +0, which the division also
-// gives (den > 0).
-__device__ __forceinline__ bool quotient_flagged(float q, float a)
-{
-    return ((__float_as_uint(q) + 8u) & 0x7FFFFu) < 16u && a != 0.0f;
-}
-
-// The codes of NB quotients a[b] / den at once: one exact division pass for
-// all of them if any shortcut quotient is flagged.
-template <int NB>
-__device__ __forceinline__ void e4m3_codes_of_quotients(const float (&a)[NB], float den, float rden,
-                                                        bool fast, uint32_t (&c)[NB])
-{
-    float q[NB];
-    bool slow = !fast;
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        q[b] = __fmul_rn(a[b], rden);
-        slow |= quotient_flagged(q[b], a[b]);
-    }
-    if (slow) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-            q[b] = __fdiv_rn(a[b], den);
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b)
-        c[b] = e4m3_enc(q[b]);
-}
-
 // 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
 __device__ __forceinline__ float pow2f(int e)
 {
@@ -347,6 +311,48 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
     f32x2 r;
     asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
     return r;
+}
+
+// Scale codes c[i] = RNE_E4M3_sat(fl(a[i] / den[i])), a[i] >= 0, mostly
+// without a division. q = fl(a * fl(1/den)) is within a few units in the last
+// place of fl(a / den) (two roundings of relative size <= 2^-24 each), so the
+// two round to different E4M3 codes only if an E4M3 rounding boundary (a
+// midpoint between adjacent E4M3 values) lies within that distance of q. The
+// check rounds q * (1 - 2^-18) and q * (1 + 2^-18), which bracket both q and
+// fl(a / den) by a wide margin: if their codes agree, no midpoint lies between
+// them and code(q) is the code of fl(a / den) (E4M3 rounding is monotone). If
+// any pair disagrees, every code is recomputed from the IEEE division. q = 0
+// and q = inf (saturating like any q > 448) need no special case. Quotients
+// are formed and checked two at a time (packed multiplies, one conversion of
+// two values).
+template <int N>
+__device__ __forceinline__ void e4m3_quotient_codes(const float (&a)[N], const float (&den)[N],
+                                                    const float (&rden)[N], bool fast,
+                                                    uint32_t (&c)[N])
+{
+    constexpr int NP = (N + 1) / 2;
+    const f32x2 up = pk2(1.0f + 0x1p-18f, 1.0f + 0x1p-18f);
+    const f32x2 dn = pk2(1.0f - 0x1p-18f, 1.0f - 0x1p-18f);
+    bool slow = !fast;
+#pragma unroll
+    for (int p = 0; p < NP; ++p) {
+        const int i = 2 * p, j = 2 * p + 1 < N ? 2 * p + 1 : 2 * p;
+        const f32x2 Q = mul2(pk2(a[i], a[j]), pk2(rden[i], rden[j]));
+        float q0, q1, p0, p1, m0, m1;
+        upk2(Q, q0, q1);
+        upk2(mul2(Q, up), p0, p1);
+        upk2(mul2(Q, dn), m0, m1);
+        const uint32_t cq = e4m3_enc2(q1, q0);
+        slow |= e4m3_enc2(p1, p0) != e4m3_enc2(m1, m0);
+        c[i] = cq & 0xFFu;
+        if (2 * p + 1 < N)
+            c[j] = cq >> 8;
+    }
+    if (slow) {
+#pragma unroll
+        for (int i = 0; i < N; ++i)
+            c[i] = e4m3_enc(__fdiv_rn(a[i], den[i]));
+    }
 }
 
 __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)

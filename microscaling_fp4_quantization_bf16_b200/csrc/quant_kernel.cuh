@@ -80,32 +80,27 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
     } else {
-        // Quotients a_b / (T s_g) for the targets T in use, by the reciprocal
-        // shortcut; one exact division pass if any of them is flagged.
+        // Scale codes of the targets in use: 6, and 4 for 4-over-6.
         const NvConsts k = tab.k;
         constexpr bool FOUR = STRAT == K_FOUR_OVER_SIX;
-        float q6[NB], q4[NB];
-        bool slow = !k.fast;
+        constexpr int NQ = FOUR ? 2 * NB : NB;
+        float qa[NQ], qd[NQ], qr[NQ];
+        uint32_t qc[NQ];
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            q6[b] = __fmul_rn(amax[b], k.rden6);
-            slow |= quotient_flagged(q6[b], amax[b]);
+            qa[b] = amax[b];
+            qd[b] = k.den6;
+            qr[b] = k.rden6;
             if constexpr (FOUR) {
-                q4[b] = __fmul_rn(amax[b], k.rden4);
-                slow |= quotient_flagged(q4[b], amax[b]);
+                qa[NB + b] = amax[b];
+                qd[NB + b] = k.den4;
+                qr[NB + b] = k.rden4;
             }
         }
-        if (slow) {
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                q6[b] = __fdiv_rn(amax[b], k.den6);
-                if constexpr (FOUR)
-                    q4[b] = __fdiv_rn(amax[b], k.den4);
-            }
-        }
+        e4m3_quotient_codes<NQ>(qa, qd, qr, k.fast, qc);
 #pragma unroll
         for (int b = 0; b < NB; ++b) {
-            uint32_t c = e4m3_enc(q6[b]);
+            uint32_t c = qc[b];
             if constexpr (STRAT == K_PREVENT_ZERO)
                 c = max(c, 1u);
             sc[b] = c;
@@ -120,7 +115,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             uint32_t c4[NB], q4w[4];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-                c4[b] = e4m3_enc(q4[b]);
+                c4[b] = qc[NB + b];
                 S4[b] = tab.S[c4[b]];
                 r4[b] = tab.R[c4[b]];
                 z4[b] = (S4[b] == 0.0f);
