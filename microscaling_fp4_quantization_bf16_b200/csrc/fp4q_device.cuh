@@ -684,6 +684,38 @@ __device__ __forceinline__ float block_sse(const float* yb, float r, float S, ui
     return tree_sum<B>(e);
 }
 
+// Lower bound on the block SSE of every scale whose reciprocal is <= r: the
+// tree sum of fl(y^2) over the elements with fl(|y| * r) <= 0.25 (those
+// round to code 0 and contribute exactly fl(y^2)), zeros elsewhere. A larger
+// scale has a smaller reciprocal, rounds a superset of elements to zero and,
+// since the tree sum of non-negative terms is monotone in every term, has an
+// SSE at least this large.
+template <int B>
+__device__ __forceinline__ float block_zero_lb(const float* yb, float r)
+{
+    float e[B];
+#pragma unroll
+    for (int j = 0; j < B; ++j) {
+        const float u = __fmul_rn(fabsf(yb[j]), r);
+        e[j] = u <= 0.25f ? __fmul_rn(yb[j], yb[j]) : 0.0f;
+    }
+    return tree_sum<B>(e);
+}
+
+// Lower bound on the block SSE of every scale S' <= S (code <= c) when the
+// block maximum a saturates at S: if fl(a * r) > 5 it rounds to 6 and its
+// error term is fl((a - fl(6 S))^2) <= SSE; a smaller scale also saturates and
+// moves fl(6 S') further below a (provided fl(6 S) <= a). Returns -1 when
+// these conditions do not hold (no bound).
+__device__ __forceinline__ float saturation_lb(float a, float r, float S)
+{
+    const float y6 = __fmul_rn(6.0f, S);
+    if (!(__fmul_rn(a, r) > 5.0f) || !(y6 <= a))
+        return -1.0f;
+    const float d = __fsub_rn(a, y6);
+    return __fmul_rn(d, d);
+}
+
 // ------------------------------------------------------------------ stores
 
 // NB = SEG / B bytes (one per block) at p (NB-byte aligned).

@@ -59,16 +59,54 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         }
         encode_seg<B, true>(y, r, zero, a.keep, q);  // packed: measured faster here
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
+        // Exact search with pruning. The candidates from the abs-max code c6 - 4
+        // upward are evaluated in ascending order (strictly lower SSE wins, so
+        // ties keep the lower code); from c6 + 5 on, every third code checks
+        // block_zero_lb, and once it exceeds the best SSE no larger code can win.
+        // Codes below c6 - 4 are skipped when saturation_lb at c6 - 5 exceeds the
+        // best SSE, else searched as well (ties then go to the lower code).
+        // Non-finite blocks search every code in order, as the definition does.
+        const NvConsts k = tab.k;
+        float qd[NB], qr[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            qd[b] = k.den6;
+            qr[b] = k.rden6;
+        }
+        uint32_t c6[NB];
+        e4m3_quotient_codes<NB>(amax, qd, qr, k.fast, c6);
         static_for<NB>([&](auto bi) {
             constexpr int b = decltype(bi)::value;
+            const float* yb = y + b * B;
+            const bool finite = amax[b] <= FLT_MAX;
+            const int lo = finite ? max(1, (int)c6[b] - 4) : 1;
             float best = 0.0f;
-            int bc = 1;
+            int bc = lo;
 #pragma unroll 1
-            for (int c = 1; c <= 0x7E; ++c) {
-                const float v = block_sse<B>(y + b * B, tab.R[c], tab.S[c], a.keep);
-                if (c == 1 || v < best) {
+            for (int c = lo; c <= 0x7E; ++c) {
+                if (finite && c >= (int)c6[b] + 5 && (c - (int)c6[b] - 5) % 3 == 0 &&
+                    block_zero_lb<B>(yb, tab.R[c]) > best)
+                    break;
+                const float v = block_sse<B>(yb, tab.R[c], tab.S[c], a.keep);
+                if (c == lo || v < best) {
                     best = v;
                     bc = c;
+                }
+            }
+            if (lo > 1 && !(saturation_lb(amax[b], tab.R[lo - 1], tab.S[lo - 1]) > best)) {
+                float bl = 0.0f;
+                int cl = 1;
+#pragma unroll 1
+                for (int c = 1; c < lo; ++c) {
+                    const float v = block_sse<B>(yb, tab.R[c], tab.S[c], a.keep);
+                    if (c == 1 || v < bl) {
+                        bl = v;
+                        cl = c;
+                    }
+                }
+                if (bl <= best) {
+                    best = bl;
+                    bc = cl;
                 }
             }
             sc[b] = (uint32_t)bc;
