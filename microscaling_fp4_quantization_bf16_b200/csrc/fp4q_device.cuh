@@ -617,6 +617,58 @@ __device__ __forceinline__ void sse_seg_scalar(const float (&y)[SEG], const uint
         sse[b] = tree_sum<B>(e + b * B);
 }
 
+// Word-pair forms for blocks of B <= 8 elements: words w and w + 2 of a
+// segment (elements 8w .. 8w+7 and 8w+16 .. 8w+23) hold 8 / B whole blocks
+// each, so a segment can be processed in two halves. Element j of the half is
+// packed with element j of the other word (the pairs {i, i + 16} of the
+// segment forms above), and every result equals the segment forms' bits.
+template <int B>
+__device__ __forceinline__ void encode_word_pair(const float (&y)[SEG], int w, const float (&rl)[8 / B],
+                                                 const float (&rh)[8 / B], uint32_t zl, uint32_t zh,
+                                                 uint32_t keep, uint32_t& ql, uint32_t& qh)
+{
+    float u[8], v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int i = 8 * w + j;
+        upk2(mul2(pk2(y[i], y[i + 16]), pk2(rl[j / B], rh[j / B])), u[j], v[j]);
+    }
+    ql = e2m1_pack8(u) & (keep & ~zl);
+    qh = e2m1_pack8(v) & (keep & ~zh);
+}
+
+template <int B>
+__device__ __forceinline__ void sse_word_pair(const float (&y)[SEG], int w, uint32_t ql, uint32_t qh,
+                                              const float (&Sl)[8 / B], const float (&Sh)[8 / B],
+                                              float (&el)[8 / B], float (&eh)[8 / B])
+{
+    static_assert(B == 4 || B == 8, "word pairs hold whole blocks of 4 or 8");
+    float va[8], vb[8], e[16];
+    e2m1_unpack8(ql, va);
+    e2m1_unpack8(qh, vb);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int i = 8 * w + j;
+        float h0, h1;
+        upk2(mul2(pk2(va[j], vb[j]), pk2(Sl[j / B], Sh[j / B])), h0, h1);
+        const float d0 = __fsub_rn(y[i], h0);
+        const float d1 = __fsub_rn(y[i + 16], h1);
+        upk2(mul2(pk2(d0, d1), pk2(d0, d1)), e[j], e[8 + j]);
+    }
+    f32x2 E[4];  // first tree level, scalar: {e[2k] + e[2k+1] of word w, same of word w + 2}
+#pragma unroll
+    for (int k = 0; k < 4; ++k)
+        E[k] = pk2(__fadd_rn(e[2 * k], e[2 * k + 1]), __fadd_rn(e[8 + 2 * k], e[8 + 2 * k + 1]));
+    E[0] = add2(E[0], E[1]);
+    E[2] = add2(E[2], E[3]);
+    if constexpr (B == 4) {
+        upk2(E[0], el[0], eh[0]);
+        upk2(E[2], el[1], eh[1]);
+    } else {
+        upk2(add2(E[0], E[2]), el[0], eh[0]);
+    }
+}
+
 // Selected forms (both compute the same bits). The packed encode measured
 // faster in the MXFP4 kernel and slower in the NVFP4 ones (register
 // pressure), so the quantize kernel picks it per format.

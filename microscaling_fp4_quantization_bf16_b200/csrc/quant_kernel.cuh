@@ -117,6 +117,68 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         });
         encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
+    } else if constexpr (STRAT == K_FOUR_OVER_SIX && B <= 8) {
+        // 4-over-6 for blocks of 4 or 8, one half segment (words w and w + 2)
+        // at a time, so the candidates' temporaries of only half the blocks
+        // are live at once. Same operations as the segment form below.
+        const NvConsts k = tab.k;
+        float qa[2 * NB], qd[2 * NB], qr[2 * NB];
+        uint32_t qc[2 * NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            qa[b] = amax[b];
+            qd[b] = k.den6;
+            qr[b] = k.rden6;
+            qa[NB + b] = amax[b];
+            qd[NB + b] = k.den4;
+            qr[NB + b] = k.rden4;
+        }
+        e4m3_quotient_codes<2 * NB>(qa, qd, qr, k.fast, qc);
+        constexpr int KB = 8 / B;  // blocks per word
+        static_for<2>([&](auto wi) {
+            constexpr int w = decltype(wi)::value;
+            constexpr int bl = 8 * w / B, bh = (8 * w + 16) / B;  // first block of each word
+            float S6l[KB], S6h[KB], S4l[KB], S4h[KB], r6l[KB], r6h[KB], r4l[KB], r4h[KB];
+            uint32_t z6l = 0, z6h = 0, z4l = 0, z4h = 0;
+            constexpr uint32_t BM = B == 4 ? 0xFFFFu : 0xFFFFFFFFu;  // nibbles of one block
+#pragma unroll
+            for (int t = 0; t < KB; ++t) {
+                S6l[t] = tab.S[qc[bl + t]];
+                r6l[t] = tab.R[qc[bl + t]];
+                S6h[t] = tab.S[qc[bh + t]];
+                r6h[t] = tab.R[qc[bh + t]];
+                S4l[t] = tab.S[qc[NB + bl + t]];
+                r4l[t] = tab.R[qc[NB + bl + t]];
+                S4h[t] = tab.S[qc[NB + bh + t]];
+                r4h[t] = tab.R[qc[NB + bh + t]];
+                z6l |= S6l[t] == 0.0f ? BM << (4 * B * t) : 0u;
+                z6h |= S6h[t] == 0.0f ? BM << (4 * B * t) : 0u;
+                z4l |= S4l[t] == 0.0f ? BM << (4 * B * t) : 0u;
+                z4h |= S4h[t] == 0.0f ? BM << (4 * B * t) : 0u;
+            }
+            uint32_t q6l, q6h, q4l, q4h;
+            encode_word_pair<B>(y, w, r6l, r6h, z6l, z6h, a.keep, q6l, q6h);
+            encode_word_pair<B>(y, w, r4l, r4h, z4l, z4h, a.keep, q4l, q4h);
+            float e6l[KB], e6h[KB], e4l[KB], e4h[KB];
+            sse_word_pair<B>(y, w, q6l, q6h, S6l, S6h, e6l, e6h);
+            sse_word_pair<B>(y, w, q4l, q4h, S4l, S4h, e4l, e4h);
+            uint32_t ml = 0, mh = 0;
+#pragma unroll
+            for (int t = 0; t < KB; ++t) {
+                const bool fl = e4l[t] < e6l[t], fh = e4h[t] < e6h[t];
+                ml |= fl ? BM << (4 * B * t) : 0u;
+                mh |= fh ? BM << (4 * B * t) : 0u;
+                sc[bl + t] = fl ? qc[NB + bl + t] : qc[bl + t];
+                S[bl + t] = fl ? S4l[t] : S6l[t];
+                sse[bl + t] = fl ? e4l[t] : e6l[t];
+                sc[bh + t] = fh ? qc[NB + bh + t] : qc[bh + t];
+                S[bh + t] = fh ? S4h[t] : S6h[t];
+                sse[bh + t] = fh ? e4h[t] : e6h[t];
+            }
+            q[w] = (q6l & ~ml) | (q4l & ml);
+            q[w + 2] = (q6h & ~mh) | (q4h & mh);
+        });
+        have_sse = true;
     } else {
         // Scale codes of the targets in use: 6, and 4 for 4-over-6.
         const NvConsts k = tab.k;
