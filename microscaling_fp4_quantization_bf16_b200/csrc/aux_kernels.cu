@@ -11,15 +11,17 @@
 namespace fp4q {
 
 constexpr int ATHREADS = 256;
+// block MSE and FOCUS forward: 128-thread CTAs measured faster on B200
+constexpr int STHREADS = 128;
 
-static inline unsigned grid_for(int64_t nseg)
+static inline unsigned grid_for(int64_t nseg, int threads = ATHREADS)
 {
-    return (unsigned)((nseg + ATHREADS - 1) / ATHREADS);
+    return (unsigned)((nseg + threads - 1) / threads);
 }
 
-static inline bool grid_ok(int64_t nseg)
+static inline bool grid_ok(int64_t nseg, int threads = ATHREADS)
 {
-    const int64_t nblk = (nseg + ATHREADS - 1) / ATHREADS;
+    const int64_t nblk = (nseg + threads - 1) / threads;
     return nblk > 0 && nblk <= 0x7FFFFFFF;
 }
 
@@ -278,14 +280,14 @@ cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t
 // ------------------------------------------------------------ block MSE
 
 template <int B, int ROT, bool MX>
-__global__ void __launch_bounds__(ATHREADS) block_mse_kernel(MseArgs a)
+__global__ void __launch_bounds__(STHREADS) block_mse_kernel(MseArgs a)
 {
     pdl_begin();
     constexpr int NB = SEG / B;
     constexpr int SPT = SegsPerThread<ROT>::value;
     const int lane = threadIdx.x & 31;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t t = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    const int64_t t = (int64_t)blockIdx.x * STHREADS + threadIdx.x;
     if ((t - lane) * SPT >= nseg)
         return;
     float y[SPT][SEG];
@@ -315,11 +317,11 @@ static cudaError_t launch_mse_rot(int rot, unsigned g, const MseArgs& a, cudaStr
 {
     cudaError_t e_ = cudaSuccess;
     switch (rot) {
-    case 0: e_ = launch_pdl(block_mse_kernel<B, 0, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-    case 16: e_ = launch_pdl(block_mse_kernel<B, 16, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-    case 32: e_ = launch_pdl(block_mse_kernel<B, 32, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-    case 64: e_ = launch_pdl(block_mse_kernel<B, 64, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
-    case 128: e_ = launch_pdl(block_mse_kernel<B, 128, MX>, dim3(g), dim3(ATHREADS), 0, st, a); break;
+    case 0: e_ = launch_pdl(block_mse_kernel<B, 0, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 16: e_ = launch_pdl(block_mse_kernel<B, 16, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 32: e_ = launch_pdl(block_mse_kernel<B, 32, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 64: e_ = launch_pdl(block_mse_kernel<B, 64, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 128: e_ = launch_pdl(block_mse_kernel<B, 128, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
     default: return cudaErrorInvalidValue;
     }
     return e_;
@@ -329,9 +331,9 @@ cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaS
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t nthr = nseg;
-    if (!grid_ok(nthr))
+    if (!grid_ok(nthr, STHREADS))
         return cudaErrorInvalidValue;
-    const unsigned g = grid_for(nthr);
+    const unsigned g = grid_for(nthr, STHREADS);
     if (mx)
         return block == 32 ? launch_mse_rot<32, true>(rot, g, a, st) : cudaErrorInvalidValue;
     switch (block) {
@@ -387,13 +389,13 @@ __device__ __forceinline__ void load_coeffs(const uint16_t* c, int64_t s, int nv
 // (Every thread derives s_g itself: a per-CTA table and barrier, as in the
 // quantize kernel, measured slower for this one-segment-per-thread kernel.)
 template <int B, int SUB, bool MX>
-__global__ void __launch_bounds__(ATHREADS) focus_fwd_kernel(FocusFwdArgs a)
+__global__ void __launch_bounds__(STHREADS) focus_fwd_kernel(FocusFwdArgs a)
 {
     pdl_begin();
     constexpr int NB = SEG / B;
     constexpr int NK = SEG / SUB;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    const int64_t s = (int64_t)blockIdx.x * STHREADS + threadIdx.x;
     float sg = 1.0f;
     if constexpr (!MX) {
         sg = global_scale_of(*a.amax);
@@ -469,7 +471,7 @@ static bool try_ffwd(int sub, unsigned g, const FocusFwdArgs& a, cudaStream_t st
 {
     if constexpr (SUB <= B) {
         if (sub == SUB) {
-            e = launch_pdl(focus_fwd_kernel<B, SUB, MX>, dim3(g), dim3(ATHREADS), 0, st, a);
+            e = launch_pdl(focus_fwd_kernel<B, SUB, MX>, dim3(g), dim3(STHREADS), 0, st, a);
             return true;
         }
     }
@@ -490,9 +492,9 @@ static cudaError_t launch_ffwd_sub(int sub, unsigned g, const FocusFwdArgs& a, c
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st)
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
-    if (!grid_ok(nseg) || sub > block)
+    if (!grid_ok(nseg, STHREADS) || sub > block)
         return cudaErrorInvalidValue;
-    const unsigned g = grid_for(nseg);
+    const unsigned g = grid_for(nseg, STHREADS);
     if (mx)
         return block == 32 ? launch_ffwd_sub<32, true>(sub, g, a, st) : cudaErrorInvalidValue;
     switch (block) {
