@@ -154,6 +154,19 @@ class ClockSampler:
 
 # ---------------------------------------------------------------- our arm
 
+def reduce_max(value: float, world: int, dev) -> float:
+    """The maximum of value over all ranks (the job's time is its slowest
+    rank's); value itself when there is one rank."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -220,11 +233,7 @@ def run_ours(args, rank, world, local_rank):
     x = xs[0]
     times = {r: [group_ms[k] / args.steps] for k, r in enumerate(ROTS)}
 
-    total_ms = sum(group_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(sum(group_ms), world, dev)
     elems = n * len(ROTS) * args.steps * world
     value = elems / (total_ms / 1e3)
     ms_per_step = total_ms / args.steps
@@ -291,11 +300,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     te0 = time.perf_counter()
     e2e_steps(args.steps)
-    te = time.perf_counter() - te0
-    if world > 1:
-        t = torch.tensor([te], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        te = float(t.item())
+    te = reduce_max(time.perf_counter() - te0, world, dev)
     h2d = xh.numel() * xh.element_size()
     d2h = sum(ch[0][r].numel() + sh[0][r].numel() for r in ROTS)
     e2e = {"value": elems / te, "unit": "elements/s", "h2d_bytes_per_step": h2d,

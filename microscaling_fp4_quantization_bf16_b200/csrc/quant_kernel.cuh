@@ -216,7 +216,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             r[b] = tab.R[c];
             zero[b] = (S[b] == 0.0f);
         }
-        encode_seg<B>(y, r, zero, a.keep, q);
+        encode_seg<B, B == 32>(y, r, zero, a.keep, q);  // packed measured faster for B = 32 only
         if constexpr (FOUR) {
             float S4[NB], r4[NB], sse4[NB];
             bool z4[NB];
@@ -228,7 +228,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
                 r4[b] = tab.R[c4[b]];
                 z4[b] = (S4[b] == 0.0f);
             }
-            encode_seg<B>(y, r4, z4, a.keep, q4w);
+            encode_seg<B, B == 32>(y, r4, z4, a.keep, q4w);
             sse_seg<B>(y, q, S, sse);
             sse_seg<B>(y, q4w, S4, sse4);
 #pragma unroll

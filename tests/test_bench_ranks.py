@@ -1,0 +1,65 @@
+"""Host logic of bench.py's multi-rank path on CPU: two gloo ranks, the job
+time is the maximum over ranks, and the reference arm runs on rank 0 only."""
+import os
+import socket
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, out):
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.reduce_max(1.5 + rank, world, torch.device("cpu"))
+        out[rank] = got
+    finally:
+        dist.destroy_process_group()
+
+
+def test_reduce_max_two_ranks():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    out = ctx.Manager().dict()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert dict(out) == {0: 2.5, 1: 2.5}
+
+
+def test_reduce_max_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    assert bench.reduce_max(3.25, 1, None) == 3.25
+
+
+def test_reference_arm_other_ranks_do_nothing(capsys):
+    sys.path.insert(0, ROOT)
+    import bench
+
+    class A:
+        steps, warmup, ref_seconds = 3, 3, 1.0
+
+    bench.run_reference(A(), rank=1, world=2)
+    assert capsys.readouterr().out == ""
