@@ -22,12 +22,13 @@ namespace fp4q {
 
 // CTA shape of the direct-load kernel: 128 threads (one segment each). The
 // MXFP4 kernels are also asked to fit 10 CTAs (40 warps) per SM, which caps
-// them at 48 registers; both measured faster on B200 than 256-thread CTAs
-// at the registers the compiler picks unconstrained.
+// them at 48 registers, the NVFP4 ones (brute force aside) 7 CTAs (72
+// registers); all measured faster on B200 than 256-thread CTAs at the
+// registers the compiler picks unconstrained.
 constexpr int QTHREADS = 128;
 template <int STRAT>
 struct QMinBlocks {
-    static constexpr int value = STRAT == K_MX ? 10 : 1;
+    static constexpr int value = STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE ? 1 : 7);
 };
 
 // Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
