@@ -60,6 +60,10 @@
  *  R9  FOCUS backward: dQ/du := 1 everywhere (no clipping), S_dq receives no
  *      gradient, dc_k = -(tsum_k(g * W) / (c_k * c_k)); the CRS per-block c_i
  *      is the special case sub-block == block.
+ *  R11 MXFP4 "brute force" is the MSE-optimised grid of [BRIDGE] 技術概要
+ *      §2.2 item 1 (per group, the scale minimising the MSE) over the
+ *      format's own scales: every E8M0 byte 0..254, scanned upward, a strictly
+ *      smaller SSE wins, a tie keeps the lower byte.
  */
 #include <float.h>
 #include <math.h>
@@ -457,9 +461,28 @@ static float nv_block(const float* y, int B, int strat, float sg, uint8_t* scale
     return quant_block(y, B, S, q, yhat);
 }
 
-/* MXFP4 block: S = 2^e with e the E8M0 exponent of the block abs-max. */
-static float mx_block(const float* y, int B, uint8_t* scale, uint8_t* q, float* yhat)
+/* MXFP4 block. abs-max: S = 2^e with e the E8M0 exponent of the block
+ * abs-max ([BRIDGE] 技術概要 §1). brute force (reading R11): the
+ * MSE-optimised grid of [BRIDGE] 技術概要 §2.2 item 1 restricted to the
+ * format's own scales -- every E8M0 byte 0..254 (S = 2^(byte - 127)) scanned
+ * upward, a strictly smaller SSE wins (a tie keeps the lower byte). */
+static float mx_block(const float* y, int B, int strat, uint8_t* scale, uint8_t* q, float* yhat)
 {
+    if (strat == REF_BRUTE_FORCE) {
+        uint8_t qt[128];
+        float yht[128];
+        int best_b = -1;
+        float best = 0.0f;
+        for (int b = 0; b <= 254; b++) {
+            float sse = quant_block(y, B, (float)ref_e8m0_value(b), qt, yht);
+            if (best_b < 0 || sse < best) {
+                best = sse;
+                best_b = b;
+            }
+        }
+        *scale = (uint8_t)best_b;
+        return quant_block(y, B, (float)ref_e8m0_value(best_b), q, yhat);
+    }
     float amax = 0.0f;
     for (int i = 0; i < B; i++) {
         float a = fabsf(y[i]);
@@ -504,7 +527,7 @@ int ref_quantize(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int blo
 {
     if (!valid_common(rows, cols, fmt, block, rot))
         return REF_ERR_ARG;
-    if (fmt == REF_FMT_MXFP4 && strat != REF_ABSMAX)
+    if (fmt == REF_FMT_MXFP4 && strat != REF_ABSMAX && strat != REF_BRUTE_FORCE)
         return REF_ERR_ARG;
     if (strat < REF_ABSMAX || strat > REF_BRUTE_FORCE)
         return REF_ERR_ARG;
@@ -524,7 +547,7 @@ int ref_quantize(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int blo
         for (int64_t b = 0; b < nb; b++) {
             const float* yb = y + b * block;
             uint8_t sc;
-            float sse = (fmt == REF_FMT_MXFP4) ? mx_block(yb, block, &sc, q, yhat)
+            float sse = (fmt == REF_FMT_MXFP4) ? mx_block(yb, block, strat, &sc, q, yhat)
                                                : nv_block(yb, block, strat, sg, &sc, q, yhat);
             int64_t base = i * cols + b * block;
             scales[i * nb + b] = sc;

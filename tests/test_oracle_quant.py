@@ -288,3 +288,83 @@ def test_focus_bwd_closed_form_and_ste(ref, sub):
     L = lambda cc: (G * W / cc[..., None]).sum(axis=2)
     fd = (L(C + h) - L(C - h)) / (2 * h)
     assert np.allclose(dc, fd, rtol=1e-4, atol=1e-6 * np.abs(fd).max())
+
+
+# ----------------------------------------- MXFP4 MSE-optimised E8M0 scale
+
+def test_mxfp4_mse_grid_hand_examples(ref):
+    # [5, -0.25, 0.75, 2.5]: SSE 1.375 at S = 1 (byte 127, the abs-max byte) and
+    # again at S = 2 (5/2 -> 2 -> 4, -0.125 -> 0, 0.375 -> 0.5 -> 1, 1.25 -> 1 -> 2);
+    # S = 4 gives 1.875, S = 1/2 saturates: the tie keeps the lower byte.
+    y = [5.0, -0.25, 0.75, 2.5] + [0.0] * 28
+    out = ref.quantize(bf16_bits([y]), "mxfp4", 32, "brute_force", 0, dq="f32")
+    assert out["scales"].tolist() == [[127]]
+    assert out["mse"][0, 0] == np.float32(1.375 / 32)
+    # 7.90625 alone: the abs-max byte 127 (S = 1) saturates it to 6; S = 2, 4, 8
+    # and 16 all give 8 (error 0.09375^2); the lowest of them, byte 128, wins.
+    z = [7.90625] + [0.0] * 31
+    am = ref.quantize(bf16_bits([z]), "mxfp4", 32, "absmax", 0)
+    bf = ref.quantize(bf16_bits([z]), "mxfp4", 32, "brute_force", 0, dq="f32")
+    assert am["scales"].tolist() == [[127]] and am["mse"][0, 0] == np.float32(1.90625 ** 2 / 32)
+    assert bf["scales"].tolist() == [[128]]
+    assert bf["dq"][0, 0] == 8.0
+    assert bf["mse"][0, 0] == np.float32(0.09375 ** 2 / 32)
+
+
+def test_mxfp4_mse_grid_never_worse_than_absmax(ref):
+    x = synth.bits16(synth.laplace_outliers(64, 256, seed=9))
+    for rot in (0, 32, 128):
+        am = ref.quantize(x, "mxfp4", 32, "absmax", rot, want_mse=True)
+        bf = ref.quantize(x, "mxfp4", 32, "brute_force", rot, want_mse=True)
+        assert np.all(bf["mse"] <= am["mse"])
+        moved = bf["scales"] != am["scales"]
+        assert np.all((bf["mse"] < am["mse"]) | (bf["scales"] < am["scales"]) | ~moved)
+        assert moved.any()
+
+
+def _sse64(y, S):
+    """Block SSE in float64 with the E2M1 grid (nearest, ties to the even
+    mantissa, saturating); S is a power of two, so y / S is exact."""
+    u = y / S
+    a = np.abs(u)
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    idx = np.argmin(np.abs(a[:, None] - grid[None, :]), axis=1)
+    # exact ties between two grid points go to the even index (even mantissa)
+    d = np.abs(a[:, None] - grid[None, :])
+    for i in range(a.size):
+        cand = np.nonzero(d[i] == d[i].min())[0]
+        idx[i] = cand[0] if len(cand) == 1 else [c for c in cand if c % 2 == 0][0]
+    v = np.where(a >= 6, 6.0, grid[idx]) * np.sign(u)
+    return float(np.sum((y - v * S) ** 2))
+
+
+def test_mxfp4_mse_grid_minimum_in_double(ref):
+    rng = np.random.default_rng(21)
+    x = bf16_bits(rng.laplace(0, 1, (16, 32)) * np.where(rng.random((16, 32)) < 0.05, 30, 1))
+    out = ref.quantize(x, "mxfp4", 32, "brute_force", 0, want_mse=True)
+    y = f32_of_bf16(x).astype(np.float64)
+    for i in range(16):
+        all64 = [_sse64(y[i], 2.0 ** (b - 127)) for b in range(255)]
+        chosen = _sse64(y[i], 2.0 ** (int(out["scales"][i, 0]) - 127))
+        assert chosen <= min(all64) * (1 + 1e-5) + 1e-30
+
+
+def test_mxfp4_mse_grid_exact_blocks(ref):
+    # blocks exactly on the E2M1 grid times 2^e: some scale gives SSE 0; the
+    # chosen byte is the lowest such byte (found here by exact rational checks)
+    from fractions import Fraction
+    rng = np.random.default_rng(5)
+    grid = [Fraction(v) for v in (0, 0.5, 1, 1.5, 2, 3, 4, 6)]
+    rows = []
+    for _ in range(24):
+        e = int(rng.integers(-20, 20))
+        v = rng.choice([0, 0.5, 1, 1.5, 2, 3, 4, 6], 32) * rng.choice([-1, 1], 32)
+        rows.append(v * 2.0 ** e)
+    x = bf16_bits(rows)
+    out = ref.quantize(x, "mxfp4", 32, "brute_force", 0, want_mse=True)
+    y = f32_of_bf16(x).astype(np.float64)
+    for i in range(24):
+        want = next(b for b in range(255)
+                    if all(abs(Fraction(float(t)) / Fraction(2) ** (b - 127)) in grid for t in y[i]))
+        assert out["scales"][i, 0] == want
+        assert out["mse"][i, 0] == 0.0
