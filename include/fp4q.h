@@ -64,7 +64,10 @@ typedef enum {
 typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1 } fp4q_format;
 
 /* Block-scale selection ("Finer is Better (with the Right Scaling)", 手法 2).
- * MXFP4 offers FP4Q_ABSMAX only. */
+ * MXFP4 offers FP4Q_ABSMAX (E8M0 byte floor(log2 amax) - 2 + 127) and
+ * FP4Q_BRUTE_FORCE: the MSE-optimised scale of "Bridging the Gap Between
+ * Promise and Performance for Microscaling FP4 Quantization" (技術概要 §2.2
+ * item 1) over every E8M0 byte 0..254, ties -> lower byte. */
 typedef enum {
     FP4Q_ABSMAX = 0,        /* code = RNE_E4M3(amax / (6 s_g)) */
     FP4Q_PREVENT_ZERO = 1,  /* abs-max code clipped below at 0x01 (2^-9) */
@@ -97,7 +100,7 @@ typedef enum { FP4Q_OUT_F32 = 0, FP4Q_OUT_BF16 = 1 } fp4q_dtype;
  * block_mse        float [rows, cols/block] or NULL.
  * dq               [rows, cols] of dq_dtype, or NULL.
  * Errors: NULL, SHAPE (cols % block, cols % rot), ALIGN, UNSUPPORTED
- * (MXFP4 with a strategy other than ABSMAX, unknown enum values), ALIAS, CUDA.
+ * (MXFP4 with PREVENT_ZERO or FOUR_OVER_SIX, unknown enum values), ALIAS, CUDA.
  */
 fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
                           fp4q_strategy strat, int rot, const float* global_amax_in,

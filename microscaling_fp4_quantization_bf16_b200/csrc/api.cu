@@ -110,7 +110,7 @@ bool make_row_map(CUtensorMap* map, const void* x, int64_t n)
 cudaError_t launch_quant(int block, int strat, int rot, const QuantArgs& a, cudaStream_t st)
 {
     const bool tma_shape = a.n % 64 == 0 && a.n / 64 < ((int64_t)1 << 31);
-    if (strat != K_BRUTE_FORCE && tma_shape && tma_requested()) {
+    if (strat != K_BRUTE_FORCE && strat != K_MX_BRUTE && tma_shape && tma_requested()) {
         CUtensorMap map;
         if (make_row_map(&map, a.x, a.n)) {
             int dev = 0, sms = 0;
@@ -168,7 +168,7 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
         return st;
     if (strat < FP4Q_ABSMAX || strat > FP4Q_BRUTE_FORCE)
         return FP4Q_ERR_UNSUPPORTED;
-    if (fmt == FP4Q_FMT_MXFP4 && strat != FP4Q_ABSMAX)
+    if (fmt == FP4Q_FMT_MXFP4 && strat != FP4Q_ABSMAX && strat != FP4Q_BRUTE_FORCE)
         return FP4Q_ERR_UNSUPPORTED;
     if (dq != nullptr && dq_dtype != FP4Q_OUT_F32 && dq_dtype != FP4Q_OUT_BF16)
         return FP4Q_ERR_UNSUPPORTED;
@@ -199,7 +199,7 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
     a.amax = nullptr;
     a.sg_out = nullptr;
     a.keep = 0xFFFFFFFFu;
-    int kstrat = nv ? (int)strat : K_MX;
+    int kstrat = nv ? (int)strat : (strat == FP4Q_BRUTE_FORCE ? K_MX_BRUTE : K_MX);
     if (nv) {
         if (global_amax_in != nullptr) {
             a.amax = global_amax_in;

@@ -261,7 +261,7 @@ __device__ __forceinline__ NvConsts nv_consts(float sg)
     return k;
 }
 
-// 2^e for e in [-127, 125] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
+// 2^e for e in [-127, 127] (2^-127 is the subnormal 0x00400000 = 2^22 * 2^-149).
 __device__ __forceinline__ float pow2f(int e)
 {
     return e >= -126 ? __uint_as_float((uint32_t)(e + 127) << 23) : __uint_as_float(0x00400000u);

@@ -31,7 +31,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 
 // Strategy ids used by the kernels (NVFP4 strategies follow the ABI enum;
 // MXFP4 abs-max is its own kernel family).
-enum KStrat { K_ABSMAX = 0, K_PREVENT_ZERO = 1, K_FOUR_OVER_SIX = 2, K_BRUTE_FORCE = 3, K_MX = 4 };
+enum KStrat { K_ABSMAX = 0, K_PREVENT_ZERO = 1, K_FOUR_OVER_SIX = 2, K_BRUTE_FORCE = 3, K_MX = 4,
+              K_MX_BRUTE = 5 };
 
 struct QuantArgs {
     const uint16_t* x;      // bf16 [n]

@@ -28,7 +28,7 @@ namespace fp4q {
 constexpr int QTHREADS = 128;
 template <int STRAT>
 struct QMinBlocks {
-    static constexpr int value = STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE ? 1 : 7);
+    static constexpr int value = STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE ? 1 : 7);
 };
 
 // Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
@@ -37,8 +37,8 @@ struct QMinBlocks {
 // and the scale-selection constants of s_g.
 template <int STRAT>
 struct ScaleTables {
-    float S[STRAT == K_MX ? 1 : 128];
-    float R[STRAT == K_MX ? 1 : 128];
+    float S[STRAT == K_MX || STRAT == K_MX_BRUTE ? 1 : 128];
+    float R[STRAT == K_MX || STRAT == K_MX_BRUTE ? 1 : 128];
     NvConsts k;
 };
 
@@ -67,6 +67,52 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             zero[b] = false;
         }
         encode_seg<B, true>(y, r, zero, a.keep, q);  // packed: measured faster here
+    } else if constexpr (STRAT == K_MX_BRUTE) {
+        // MXFP4 MSE-optimised scale: every E8M0 byte 0..254 (S = 2^(byte -
+        // 127)), searched like the NVFP4 brute force below -- upward from the
+        // abs-max byte - 4, stopped by block_zero_lb (checked from abs-max + 2),
+        // lower bytes skipped under saturation_lb; ties keep the lower byte.
+        static_assert(B == 32, "MXFP4 blocks are 32 wide");
+        const float am = amax[0];
+        const bool finite = am <= FLT_MAX;
+        const int babs = e8m0_exp(am) + 127;
+        const int lo = finite ? max(0, babs - 4) : 0;
+        float best = 0.0f;
+        int bb = lo;
+#pragma unroll 1
+        for (int bt = lo; bt <= 254; ++bt) {
+            const float rb = pow2f(127 - bt);
+            if (finite && bt >= babs + 2 && block_zero_lb<32>(y, rb) > best)
+                break;
+            const float v = block_sse<32>(y, rb, pow2f(bt - 127), a.keep);
+            if (bt == lo || v < best) {
+                best = v;
+                bb = bt;
+            }
+        }
+        if (lo > 0 && !(saturation_lb(am, pow2f(128 - lo), pow2f(lo - 128)) > best)) {
+            float bl = 0.0f;
+            int cl = 0;
+#pragma unroll 1
+            for (int bt = 0; bt < lo; ++bt) {
+                const float v = block_sse<32>(y, pow2f(127 - bt), pow2f(bt - 127), a.keep);
+                if (bt == 0 || v < bl) {
+                    bl = v;
+                    cl = bt;
+                }
+            }
+            if (bl <= best) {
+                best = bl;
+                bb = cl;
+            }
+        }
+        sc[0] = (uint32_t)bb;
+        S[0] = pow2f(bb - 127);
+        r[0] = pow2f(127 - bb);
+        zero[0] = false;
+        sse[0] = best;
+        encode_seg<B, true>(y, r, zero, a.keep, q);
+        have_sse = true;
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
         // Exact search with pruning. The candidates from the abs-max code c6 - 4
         // upward are evaluated in ascending order (strictly lower SSE wins, so
@@ -294,7 +340,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
 template <int STRAT>
 __device__ __forceinline__ void build_scale_tables(ScaleTables<STRAT>& tab, const QuantArgs& a)
 {
-    if constexpr (STRAT != K_MX) {
+    if constexpr (STRAT != K_MX && STRAT != K_MX_BRUTE) {
         if (threadIdx.x < 128) {
             const float sg = global_scale_of(*a.amax);
             for (int c = threadIdx.x; c < 128; c += blockDim.x) {
@@ -363,6 +409,7 @@ cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream
     FP4Q_QROTS(K_BRUTE_FORCE)
     if constexpr (B == 32) {
         FP4Q_QROTS(K_MX)
+        FP4Q_QROTS(K_MX_BRUTE)
     }
 #undef FP4Q_QROTS
 #undef FP4Q_QCASE

@@ -83,6 +83,7 @@ def test_quantize_validation(lib):
     assert q(lib, dq=MIS) == ALIGN
     assert q(lib, gout=A3 + 66) == ALIGN
     assert q(lib, fmt=MX, block=32, strat=2, gout=None) == UNSUP
+    assert q(lib, fmt=MX, block=32, strat=1, gout=None) == UNSUP
     assert q(lib, fmt=MX, block=16, gout=None) == UNSUP
     assert q(lib, block=64) == UNSUP
     assert q(lib, block=2) == UNSUP

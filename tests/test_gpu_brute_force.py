@@ -53,3 +53,28 @@ def test_brute_force_stress(gpu, block, rot, gamax):
     g = gpu_quantize(gpu, x, "nvfp4", block, "brute_force", rot, gamax=gamax, mse=True)
     o = oracle_quantize(x, "nvfp4", block, "brute_force", rot, gamax=gamax, mse=True)
     compare_quant(g, o, "nvfp4", f"brute B{block} H{rot} gamax={gamax}")
+
+
+@pytest.mark.parametrize("rot", [0, 32, 128])
+def test_mxfp4_mse_grid_stress(gpu, rot):
+    """The MXFP4 MSE-optimised E8M0 scale ("Bridging the Gap ...", 技術概要
+    §2.2 item 1) on the same stress rows: GPU vs the oracle's scan of all
+    255 bytes."""
+    x = stress_rows(2048, 128, seed=300 + rot)
+    g = gpu_quantize(gpu, x, "mxfp4", 32, "brute_force", rot, mse=True)
+    o = oracle_quantize(x, "mxfp4", 32, "brute_force", rot, mse=True)
+    compare_quant(g, o, "mxfp4", f"mxfp4 mse grid H{rot}")
+
+
+def test_mxfp4_mse_grid_full_size_sampled(gpu):
+    """C2 (4096x4096 Laplace + outliers) with the MSE-optimised E8M0 scale, rot
+    0 and 32: every element of 64 sampled rows (MXFP4 needs no tensor-wide
+    value, so a row's result depends on that row only)."""
+    x = synth.workload("c2_mxfp4_laplace_outliers")["x"]
+    rows = np.random.default_rng(3).choice(x.shape[0], 64, replace=False)
+    for rot in (0, 32):
+        g = gpu_quantize(gpu, x, "mxfp4", 32, "brute_force", rot, mse=True)
+        o = oracle_quantize(x[rows], "mxfp4", 32, "brute_force", rot, mse=True)
+        for k in ("codes", "scales", "mse"):
+            g[k] = g[k][rows]
+        compare_quant(g, o, "mxfp4", f"C2 mse grid H{rot}")

@@ -122,7 +122,8 @@ def mixed(rows, cols, seed):
 
 COMBOS = [("nvfp4", b, s, r) for b in (4, 8, 16, 32)
           for s in ("absmax", "prevent_zero", "four_over_six", "brute_force")
-          for r in (0, 16, 32, 64, 128)] + [("mxfp4", 32, "absmax", r) for r in (0, 16, 32, 64, 128)]
+          for r in (0, 16, 32, 64, 128)] + [("mxfp4", 32, s, r) for s in ("absmax", "brute_force")
+                                            for r in (0, 16, 32, 64, 128)]
 
 
 def shapes_for(block, rot):
