@@ -70,13 +70,15 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
     } else if constexpr (STRAT == K_MX_BRUTE) {
         // MXFP4 MSE-optimised scale: every E8M0 byte 0..254 (S = 2^(byte -
         // 127)), searched like the NVFP4 brute force below -- upward from the
-        // abs-max byte - 4, stopped by block_zero_lb (checked from abs-max + 2),
+        // abs-max byte - 1, stopped by block_zero_lb (checked from abs-max + 2),
         // lower bytes skipped under saturation_lb; ties keep the lower byte.
+        // (At abs-max - 2 the block maximum is 16 to 32 times the scale, so
+        // the saturation bound almost always excludes every lower byte.)
         static_assert(B == 32, "MXFP4 blocks are 32 wide");
         const float am = amax[0];
         const bool finite = am <= FLT_MAX;
         const int babs = e8m0_exp(am) + 127;
-        const int lo = finite ? max(0, babs - 4) : 0;
+        const int lo = finite ? max(0, babs - 1) : 0;
         float best = 0.0f;
         int bb = lo;
 #pragma unroll 1
