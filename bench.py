@@ -408,8 +408,9 @@ def breakdown(dev, peaks, reps: int = 10):
                 for _ in range(nc)]
             dqb = 0 if dq is None else torch.tensor([], dtype=dq).element_size()
             bpe = bytes_per_elem(block, mse=want_mse, dq=dqb)
-            ops = n * 126 * 5 if strat == "brute_force" else None
-            tag = f"{wl} {fmt} B{block} {strat} H{rot}"
+            ops = n * (126 if nv else 255) * 5 if strat == "brute_force" else None
+            label = "mse_grid (E8M0 brute force)" if (strat == "brute_force" and not nv) else strat
+            tag = f"{wl} {fmt} B{block} {label} H{rot}"
             if nv:
                 ga = fp4q.global_amax(x0, rot)
                 secs = timeit([lambda i=i: fp4q.quantize(xs[i], fmt, block, strat, rot,
@@ -429,7 +430,8 @@ def breakdown(dev, peaks, reps: int = 10):
         torch.cuda.empty_cache()
 
     quant_runs("c1_nvfp4_roundtrip", [("nvfp4", 16, "absmax", 0)], want_mse=True, dq=torch.float32)
-    quant_runs("c2_mxfp4_laplace_outliers", [("mxfp4", 32, "absmax", 0), ("mxfp4", 32, "absmax", 32)])
+    quant_runs("c2_mxfp4_laplace_outliers", [("mxfp4", 32, s, r) for s in ("absmax", "brute_force")
+                                             for r in (0, 32)])
     quant_runs("c3_strategy_sweep_t3", [("nvfp4", b, s, 0) for b in (4, 8, 16, 32)
                                         for s in ("absmax", "prevent_zero", "four_over_six",
                                                   "brute_force")], want_mse=True)
