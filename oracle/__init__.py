@@ -75,6 +75,8 @@ def lib():
         L.ref_focus_fwd.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         L.ref_focus_bwd.restype = i32
         L.ref_focus_bwd.argtypes = [p, p, p, i64, i64, i32, p]
+        L.ref_dequantize_unrotate.restype = i32
+        L.ref_dequantize_unrotate.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p]
         for name in ("ref_rne_e2m1_array", "ref_rne_e4m3_array"):
             getattr(L, name).restype = None
             getattr(L, name).argtypes = [p, i64, p]
@@ -227,6 +229,20 @@ def dequantize(codes, scales, global_scale, rows, cols, fmt="nvfp4", block=16, o
     ob = np.zeros((rows, cols), np.uint16) if out == "bf16" else None
     rc = lib().ref_dequantize(_ptr(codes), _ptr(scales), _ptr(gs), rows, cols, _fmt(fmt), block,
                               _ptr(of), _ptr(ob))
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return of if out == "f32" else ob
+
+
+def dequantize_unrotate(codes, scales, global_scale, rows, cols, fmt="nvfp4", block=16, rot=0,
+                        out="f32"):
+    codes = np.ascontiguousarray(codes, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    gs = np.array([1.0 if global_scale is None else global_scale], np.float32)
+    of = np.zeros((rows, cols), np.float32) if out == "f32" else None
+    ob = np.zeros((rows, cols), np.uint16) if out == "bf16" else None
+    rc = lib().ref_dequantize_unrotate(_ptr(codes), _ptr(scales), _ptr(gs), rows, cols,
+                                       _fmt(fmt), block, rot, _ptr(of), _ptr(ob))
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")
     return of if out == "f32" else ob

@@ -60,6 +60,9 @@
  *  R9  FOCUS backward: dQ/du := 1 everywhere (no clipping), S_dq receives no
  *      gradient, dc_k = -(tsum_k(g * W) / (c_k * c_k)); the CRS per-block c_i
  *      is the special case sub-block == block.
+ *  R13 Dequantization back to the original domain applies the normalised
+ *      rotation again (same stages and k_n): H_n is symmetric and
+ *      H_n H_n = n I, so it is its own inverse up to the rounding of k_n.
  *  R11 MXFP4 "brute force" is the MSE-optimised grid of [BRIDGE] 技術概要
  *      §2.2 item 1 (per group, the scale minimising the MSE) over the
  *      format's own scales: every E8M0 byte 0..254, scanned upward, a strictly
@@ -593,6 +596,42 @@ int ref_dequantize(const uint8_t* codes, const uint8_t* scales, const float* glo
         if (out_bf16)
             out_bf16[k] = ref_float_to_bf16(v);
     }
+    return REF_OK;
+}
+
+/* Dequantize, then return to the original domain: yhat = value(q) * S as in
+ * ref_dequantize, then every rot-wide chunk of a row through the normalised
+ * transform once more (reading R13: the Sylvester H_n is symmetric with
+ * H_n H_n = n I, so the normalised rotation is its own inverse, exactly for
+ * n = 16 and 64 where k_n^2 n = 1, up to the rounding of k_n otherwise).
+ * [BRIDGE] 技術概要 §2.2 item 3 (blockwise rotations). rot == 0 is plain
+ * dequantization. */
+int ref_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales, const float* global_scale,
+                            int64_t rows, int64_t cols, int fmt, int block, int rot,
+                            float* out_f32, uint16_t* out_bf16)
+{
+    if (!valid_common(rows, cols, fmt, block, rot))
+        return REF_ERR_ARG;
+    float sg = (fmt == REF_FMT_NVFP4) ? *global_scale : 1.0f;
+    float* y = (float*)malloc(sizeof(float) * (size_t)cols);
+    for (int64_t i = 0; i < rows; i++) {
+        for (int64_t j = 0; j < cols; j++) {
+            int64_t k = i * cols + j;
+            uint8_t byte = codes[k / 2];
+            int q = (k & 1) ? (byte >> 4) : (byte & 15);
+            y[j] = (float)ref_e2m1_value(q) * block_scale(fmt, scales[k / block], sg);
+        }
+        if (rot > 0)
+            for (int64_t j = 0; j < cols; j += rot)
+                ref_fwht(y + j, rot);
+        for (int64_t j = 0; j < cols; j++) {
+            if (out_f32)
+                out_f32[i * cols + j] = y[j];
+            if (out_bf16)
+                out_bf16[i * cols + j] = ref_float_to_bf16(y[j]);
+        }
+    }
+    free(y);
     return REF_OK;
 }
 

@@ -368,3 +368,51 @@ def test_mxfp4_mse_grid_exact_blocks(ref):
                     if all(abs(Fraction(float(t)) / Fraction(2) ** (b - 127)) in grid for t in y[i]))
         assert out["scales"][i, 0] == want
         assert out["mse"][i, 0] == 0.0
+
+
+# ------------------------------------------- dequantization back to the original domain
+
+def _h(n):
+    from scipy.linalg import hadamard
+    return hadamard(n).astype(np.float64) / math.sqrt(n)
+
+
+@pytest.mark.parametrize("rot", [16, 32, 64, 128])
+def test_dequantize_unrotate_matches_float64_rotation(ref, rot):
+    # MXFP4 codes with E8M0 scales 2^-3 .. 2^3: the dequantized values are short
+    # dyadic numbers, so for rot 16 and 64 (k_n = 1/4, 1/8) the fp32 transform is
+    # exact and must equal the float64 product with the normalised Sylvester matrix
+    rng = np.random.default_rng(rot)
+    rows, cols = 6, 256
+    codes = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+    scales = rng.integers(124, 131, (rows, cols // 32), dtype=np.uint8)
+    plain = ref.dequantize(codes, scales, None, rows, cols, "mxfp4", 32)
+    got = ref.dequantize_unrotate(codes, scales, None, rows, cols, "mxfp4", 32, rot)
+    want = (plain.astype(np.float64).reshape(rows, cols // rot, rot) @ _h(rot).T).reshape(rows, cols)
+    if rot in (16, 64):
+        assert np.array_equal(got.astype(np.float64), want)
+    else:
+        assert np.max(np.abs(got - want)) <= 1e-6 * np.max(np.abs(want))
+
+
+def test_dequantize_unrotate_rot0_is_dequantize(ref):
+    rng = np.random.default_rng(1)
+    codes = rng.integers(0, 256, (4, 32), dtype=np.uint8)
+    scales = rng.integers(0, 127, (4, 4), dtype=np.uint8)
+    a = ref.dequantize(codes, scales, 0.5, 4, 64, "nvfp4", 16)
+    b = ref.dequantize_unrotate(codes, scales, 0.5, 4, 64, "nvfp4", 16, 0)
+    assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+@pytest.mark.parametrize("fmt,block,rot", [("mxfp4", 32, 32), ("mxfp4", 32, 128), ("nvfp4", 16, 16)])
+def test_rotated_round_trip_error_equals_block_sse(ref, fmt, block, rot):
+    # the rotation is orthonormal (up to the rounding of k_n): the squared error of
+    # quantize -> dequantize -> undo the rotation equals the sum of the block SSEs
+    # measured in the rotated domain
+    x = synth.bits16(synth.laplace_outliers(32, 512, seed=4))
+    q = ref.quantize(x, fmt, block, "absmax", rot, want_mse=True)
+    back = ref.dequantize_unrotate(q["codes"], q["scales"], q["global_scale"] if fmt == "nvfp4" else None,
+                                   32, 512, fmt, block, rot)
+    err = np.sum((f32_of_bf16(x).astype(np.float64) - back.astype(np.float64)) ** 2)
+    sse = np.sum(q["mse"].astype(np.float64) * block)
+    assert abs(err - sse) <= 1e-4 * sse
