@@ -121,6 +121,23 @@ fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
                             cudaStream_t stream);
 
 /*
+ * fp4q_dequantize_unrotate -- fp4q_dequantize, then every rot-wide chunk of a
+ * row taken back to the original domain by the normalised Walsh-Hadamard
+ * transform (the blockwise rotation of "Bridging the Gap Between Promise and
+ * Performance for Microscaling FP4 Quantization", 技術概要 §2.2 item 3; the
+ * Sylvester matrix is symmetric with H H = n I, so the normalised transform
+ * is its own inverse -- exactly for rot 16 and 64, up to the rounding of
+ * 1/sqrt(rot) for 32 and 128). Same stage order and constant as the rotation
+ * applied by fp4q_quantize. rot in {0, 16, 32, 64, 128}; 0 is plain
+ * dequantization. Arguments, ownership and errors as fp4q_dequantize, plus
+ * SHAPE when cols % rot != 0 and UNSUPPORTED for another rot.
+ */
+fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales,
+                                     const float* global_scale, int64_t rows, int64_t cols,
+                                     fp4q_format fmt, int block, int rot, void* out,
+                                     fp4q_dtype out_dtype, cudaStream_t stream);
+
+/*
  * fp4q_block_mse -- per-block mean squared error of x (rotated by rot first)
  * against dequantize(codes, scales): tree sum of (y - yhat)^2 divided by
  * block ("Finer is Better (with the Right Scaling)", 手法 1: MSE per block

@@ -87,13 +87,20 @@ def quantize(x: torch.Tensor, fmt="nvfp4", block: int = 16, strategy="absmax", r
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, global_scale: Optional[torch.Tensor],
                fmt="nvfp4", block: int = 16, dtype: torch.dtype = torch.float32,
-               out: Optional[torch.Tensor] = None) -> torch.Tensor:
+               out: Optional[torch.Tensor] = None, rot: int = 0) -> torch.Tensor:
+    """value(code) * S; with rot > 0 the values are also taken back from the
+    rotated domain (fp4q_dequantize_unrotate)."""
     rows, half = codes.shape
     cols = 2 * half
     if out is None:
         out = torch.empty(rows, cols, dtype=dtype, device=codes.device)
-    _abi.call("fp4q_dequantize", codes.data_ptr(), scales.data_ptr(), _ptr(global_scale), rows,
-              cols, _fmt(fmt), block, out.data_ptr(), DTYPES[out.dtype], _stream())
+    if rot:
+        _abi.call("fp4q_dequantize_unrotate", codes.data_ptr(), scales.data_ptr(),
+                  _ptr(global_scale), rows, cols, _fmt(fmt), block, rot, out.data_ptr(),
+                  DTYPES[out.dtype], _stream())
+    else:
+        _abi.call("fp4q_dequantize", codes.data_ptr(), scales.data_ptr(), _ptr(global_scale),
+                  rows, cols, _fmt(fmt), block, out.data_ptr(), DTYPES[out.dtype], _stream())
     return out
 
 

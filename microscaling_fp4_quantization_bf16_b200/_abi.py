@@ -21,6 +21,7 @@ SIGNATURES = {
     "fp4q_quantize": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
                              _i32, _p]),
     "fp4q_dequantize": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _p, _i32, _p]),
+    "fp4q_dequantize_unrotate": (_i32, [_p, _p, _p, _i64, _i64, _i32, _i32, _i32, _p, _i32, _p]),
     "fp4q_block_mse": (_i32, [_p, _p, _p, _p, _i64, _i64, _i32, _i32, _i32, _p, _p]),
     "fp4q_focus_fwd": (_i32, [_p, _p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _i32, _p, _p,
                               _p]),

@@ -244,7 +244,37 @@ fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
     a.n = n;
     a.out = out;
     a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
+    a.keep = 0xFFFFFFFFu;
     return cuda_status(launch_dequant(nv ? 0 : 1, block, a, stream));
+}
+
+fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales,
+                                     const float* global_scale, int64_t rows, int64_t cols,
+                                     fp4q_format fmt, int block, int rot, void* out,
+                                     fp4q_dtype out_dtype, cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, rot);
+    if (st != FP4Q_OK)
+        return st;
+    if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    if (codes == nullptr || scales == nullptr || out == nullptr || (nv && global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (nv && !aligned4(global_scale)))
+        return FP4Q_ERR_ALIGN;
+    DequantArgs a;
+    a.codes = codes;
+    a.scales = scales;
+    a.sg = nv ? global_scale : nullptr;
+    a.n = n;
+    a.out = out;
+    a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
+    a.keep = 0xFFFFFFFFu;
+    return cuda_status(launch_dequant_rot(nv ? 0 : 1, block, rot, a, stream));
 }
 
 fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,

@@ -277,6 +277,76 @@ cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t
     }
 }
 
+// Dequantize and undo the blockwise rotation: one segment per thread, the
+// segment's values decoded, then rotated again by the normalised transform
+// (its own inverse; 64/128-wide chunks span neighbouring lanes, so whole warps
+// take part). Each decoded product is masked with the run-time all-ones
+// `keep` before the butterflies: ptxas would otherwise fuse the packed
+// multiply of the decode into the first packed add of the rotation, which
+// changes the rounding.
+template <int B, bool MX, int ROT>
+__global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
+{
+    pdl_begin();
+    constexpr int NB = SEG / B;
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    const int64_t s = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
+    if (s - lane >= nseg)  // warp-uniform
+        return;
+    const bool active = s < nseg;
+    const int nvalid = active ? (int)min((int64_t)SEG, a.n - s * SEG) : 0;
+    uint32_t q[4] = {0u, 0u, 0u, 0u}, sc[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b)
+        sc[b] = 0u;
+    if (active) {
+        load_codes(a.codes, s, nvalid, q);
+        load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
+    }
+    const float sg = MX ? 1.0f : *a.sg;
+    float S[NB], yh[SEG];
+    scales_of<NB, MX>(sc, sg, S);
+    decode_seg<B>(q, S, yh);
+#pragma unroll
+    for (int i = 0; i < SEG; ++i)
+        yh[i] = __uint_as_float(__float_as_uint(yh[i]) & a.keep);
+    rotate_seg<ROT>(yh, lane);
+    if (active)
+        store_seg_values(a.out, a.out_kind, s, nvalid, yh);
+}
+
+template <int B, bool MX>
+static cudaError_t launch_dequant_rot_b(int rot, const DequantArgs& a, cudaStream_t st)
+{
+    const int64_t nseg = (a.n + SEG - 1) / SEG;
+    if (!grid_ok(nseg))
+        return cudaErrorInvalidValue;
+    const unsigned g = grid_for(nseg);
+    switch (rot) {
+    case 16: return launch_pdl(dequant_rot_kernel<B, MX, 16>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 32: return launch_pdl(dequant_rot_kernel<B, MX, 32>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 64: return launch_pdl(dequant_rot_kernel<B, MX, 64>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 128: return launch_pdl(dequant_rot_kernel<B, MX, 128>, dim3(g), dim3(ATHREADS), 0, st, a);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a, cudaStream_t st)
+{
+    if (rot == 0)
+        return launch_dequant(mx, block, a, st);
+    if (mx)
+        return block == 32 ? launch_dequant_rot_b<32, true>(rot, a, st) : cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_dequant_rot_b<4, false>(rot, a, st);
+    case 8: return launch_dequant_rot_b<8, false>(rot, a, st);
+    case 16: return launch_dequant_rot_b<16, false>(rot, a, st);
+    case 32: return launch_dequant_rot_b<32, false>(rot, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
 // ------------------------------------------------------------ block MSE
 
 template <int B, int ROT, bool MX>

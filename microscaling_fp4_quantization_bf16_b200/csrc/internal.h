@@ -54,6 +54,7 @@ struct DequantArgs {
     int64_t n;
     void* out;
     int out_kind;           // 1 fp32, 2 bf16
+    uint32_t keep;          // 0xFFFFFFFF, passed at run time (see dequant_rot_kernel)
 };
 
 struct MseArgs {
@@ -110,6 +111,7 @@ cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cu
 cudaError_t launch_finalize_sg(float* g, cudaStream_t st);
 cudaError_t launch_set_one(float* p, cudaStream_t st);
 cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st);
+cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a, cudaStream_t st);
 cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st);
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);

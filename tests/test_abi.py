@@ -101,6 +101,15 @@ def test_other_entry_points_validation(lib):
     assert L.fp4q_dequantize(A, A, A, 4, 60, NV, 16, A, 0, None) == SHAPE
     assert L.fp4q_dequantize(A, MIS, A, 4, 64, NV, 16, A, 0, None) == ALIGN
     assert L.fp4q_dequantize(A, A, A, 4, 64, NV, 16, A, 3, None) == UNSUP
+    du = lambda **k: L.fp4q_dequantize_unrotate(k.get("codes", A), A, k.get("gs", A), 4,
+                                                k.get("cols", 128), NV, 16, k.get("rot", 32),
+                                                k.get("out", A), k.get("ot", 0), None)
+    assert du(rot=24) == UNSUP
+    assert du(cols=96, rot=64) == SHAPE
+    assert du(ot=4) == UNSUP
+    assert du(codes=None) == NULL
+    assert du(gs=None) == NULL
+    assert du(out=MIS) == ALIGN
     assert L.fp4q_block_mse(A, A, A, A, 4, 64, NV, 16, 0, None, None) == NULL
     assert L.fp4q_block_mse(A, A, A, A, 4, 64, NV, 16, 128, A, None) == SHAPE
     assert L.fp4q_block_mse(A, A, A, MIS + 2, 4, 64, NV, 16, 0, A, None) == ALIGN

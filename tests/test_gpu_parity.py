@@ -302,6 +302,37 @@ def test_dequantize_and_block_mse_any_bytes(gpu, fmt, block):
         assert_exact(m.cpu().numpy(), q["mse"], "block_mse == quantize mse")
 
 
+@pytest.mark.parametrize("fmt,block", [("nvfp4", 4), ("nvfp4", 8), ("nvfp4", 16), ("nvfp4", 32),
+                                       ("mxfp4", 32)])
+@pytest.mark.parametrize("rot", [16, 32, 64, 128])
+def test_dequantize_unrotate(gpu, fmt, block, rot):
+    """Dequantization back to the original domain (the normalised rotation
+    applied again) on real codes of real data and on arbitrary code and scale
+    bytes."""
+    # a flattened length that is not a multiple of 32 where the shape allows it
+    rows, cols = 9, 2 * max(rot, block, 32) + (16 if rot == 16 and block <= 16 else 0)
+    x = mixed(rows, cols, seed=rot + block)
+    q = gpu_quantize(gpu, x, fmt, block, "absmax", rot)
+    rng = np.random.default_rng(rot * block)
+    raw_codes = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
+    # scale bytes whose values stay finite through the butterflies (an infinity
+    # would turn into NaN, whose bit pattern is not part of the contract)
+    raw_scales = rng.integers(0, 127 if fmt == "nvfp4" else 201, size=(rows, cols // block),
+                              dtype=np.uint8)
+    for codes, scales, sg, what in ((q["codes"], q["scales"], q["gs"], "quantized"),
+                                    (raw_codes, raw_scales, np.float32(3.1e-3), "raw bytes")):
+        gs = torch.tensor([sg], device="cuda") if fmt == "nvfp4" else None
+        for dt, name in ((torch.float32, "f32"), (torch.bfloat16, "bf16")):
+            out = gpu.dequantize(torch.from_numpy(np.ascontiguousarray(codes)).cuda(),
+                                 torch.from_numpy(np.ascontiguousarray(scales)).cuda(), gs, fmt,
+                                 block, dt, rot=rot)
+            torch.cuda.synchronize()
+            got = out.cpu().numpy() if dt == torch.float32 else u16(out)
+            want = oracle.dequantize_unrotate(codes, scales, sg if fmt == "nvfp4" else None, rows,
+                                              cols, fmt, block, rot, name)
+            assert_exact(got, want, f"dequant-unrotate {fmt} B{block} H{rot} {name} {what}")
+
+
 def test_global_amax(gpu):
     x = mixed(9, 256, seed=5)
     for rot in (0, 16, 32, 64, 128):
