@@ -432,6 +432,21 @@ def breakdown(dev, peaks, reps: int = 10):
     quant_runs("c1_nvfp4_roundtrip", [("nvfp4", 16, "absmax", 0)], want_mse=True, dq=torch.float32)
     quant_runs("c2_mxfp4_laplace_outliers", [("mxfp4", 32, s, r) for s in ("absmax", "brute_force")
                                              for r in (0, 32)])
+    # dequantize (and back to the original domain) of C2's rot-32 codes, bf16 out
+    x0 = synth.workload("c2_mxfp4_laplace_outliers")["x"].to(dev)
+    n = x0.numel()
+    q0 = fp4q.quantize(x0, "mxfp4", 32, "absmax", 32)
+    nc = copies_for(n // 2, l2)
+    qs = [(q0.codes.clone(), q0.scales.clone()) for _ in range(nc)]
+    dos = [torch.empty_like(x0) for _ in range(nc)]
+    for rot in (0, 32):
+        secs = timeit([lambda i=i: fp4q.dequantize(qs[i][0], qs[i][1], None, "mxfp4", 32,
+                                                   torch.bfloat16, out=dos[i], rot=rot)
+                       for i in range(nc)])
+        add(f"c2_mxfp4_laplace_outliers dequantize{' + undo H32' if rot else ''} -> bf16", n, secs,
+            0.5 + 1 / 32 + 2, 1)
+    del x0, q0, qs, dos
+    torch.cuda.empty_cache()
     quant_runs("c3_strategy_sweep_t3", [("nvfp4", b, s, 0) for b in (4, 8, 16, 32)
                                         for s in ("absmax", "prevent_zero", "four_over_six",
                                                   "brute_force")], want_mse=True)
