@@ -595,7 +595,8 @@ SUITE = ["quant MXFP4 B32 rot0", "quant MXFP4 B32 rot32", "quant MXFP4 B32 rot12
          "quant NVFP4 B16 abs-max (+MSE)", "quant NVFP4 B16 4-over-6 rot16",
          "quant NVFP4 B4 4-over-6 (+MSE)", "quant NVFP4 B16 brute force (1024 rows, +MSE)",
          "global abs-max rot16", "dequantize NVFP4 B16 -> bf16", "block MSE NVFP4 B16",
-         "FOCUS fwd NVFP4 B16 sub8 -> bf16", "FOCUS bwd sub8"]
+         "FOCUS fwd NVFP4 B16 sub8 -> bf16", "FOCUS bwd sub8", "quant NVFP4 B16 4-over-6 (+MSE)",
+         "quant MXFP4 B32 MSE-optimised E8M0 scale", "dequantize MXFP4 B32 + undo 128-wide Hadamard -> bf16"]
 
 
 def run_suite(rounds: int = 2):
@@ -634,6 +635,10 @@ def run_suite(rounds: int = 2):
         outs[9] = fp4q.block_mse(x, q16.codes, q16.scales, q16.global_scale, "nvfp4", 16, 0)
         outs[10] = fp4q.focus_fwd(w, c, "nvfp4", 16, 8, global_amax=gw)
         outs[11] = fp4q.focus_bwd(w, g, c, 8)
+        outs[12] = fp4q.quantize(x, "nvfp4", 16, "four_over_six", 0, global_amax=ga, want_mse=True)
+        outs[13] = fp4q.quantize(x, "mxfp4", 32, "brute_force", 0)
+        outs[14] = fp4q.dequantize(outs[2].codes, outs[2].scales, None, "mxfp4", 32, torch.bfloat16,
+                                   rot=128)
         torch.cuda.synchronize()
     print(json.dumps({"suite": SUITE, "rounds": rounds, "shape": [R, C],
                       "device_errors": fp4q._abi.load().fp4q_device_errors()}))

@@ -321,7 +321,7 @@ __device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b)
 // check rounds q * (1 - 2^-18) and q * (1 + 2^-18), which bracket both q and
 // fl(a / den) by a wide margin: if their codes agree, no midpoint lies between
 // them and code(q) is the code of fl(a / den) (E4M3 rounding is monotone). If
-// any pair disagrees, every code is recomputed from the IEEE division. q = 0
+// they disagree, that pair's codes are recomputed from the IEEE division. q = 0
 // and q = inf (saturating like any q > 448) need no special case. Quotients
 // are formed and checked two at a time (packed multiplies, one conversion of
 // two values).
@@ -333,7 +333,6 @@ __device__ __forceinline__ void e4m3_quotient_codes(const float (&a)[N], const f
     constexpr int NP = (N + 1) / 2;
     const f32x2 up = pk2(1.0f + 0x1p-18f, 1.0f + 0x1p-18f);
     const f32x2 dn = pk2(1.0f - 0x1p-18f, 1.0f - 0x1p-18f);
-    bool slow = !fast;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
         const int i = 2 * p, j = 2 * p + 1 < N ? 2 * p + 1 : 2 * p;
@@ -342,16 +341,15 @@ __device__ __forceinline__ void e4m3_quotient_codes(const float (&a)[N], const f
         upk2(Q, q0, q1);
         upk2(mul2(Q, up), p0, p1);
         upk2(mul2(Q, dn), m0, m1);
-        const uint32_t cq = e4m3_enc2(q1, q0);
-        slow |= e4m3_enc2(p1, p0) != e4m3_enc2(m1, m0);
+        uint32_t cq = e4m3_enc2(q1, q0);
+        // a midpoint between the brackets (or no fast path at all): this pair
+        // takes the IEEE division. Quotients that share a segment rarely need
+        // it together, so each pair branches on its own.
+        if (!fast || e4m3_enc2(p1, p0) != e4m3_enc2(m1, m0))
+            cq = e4m3_enc2(__fdiv_rn(a[j], den[j]), __fdiv_rn(a[i], den[i]));
         c[i] = cq & 0xFFu;
         if (2 * p + 1 < N)
             c[j] = cq >> 8;
-    }
-    if (slow) {
-#pragma unroll
-        for (int i = 0; i < N; ++i)
-            c[i] = e4m3_enc(__fdiv_rn(a[i], den[i]));
     }
 }
 
