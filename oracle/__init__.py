@@ -75,6 +75,8 @@ def lib():
         L.ref_focus_fwd.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         L.ref_focus_bwd.restype = i32
         L.ref_focus_bwd.argtypes = [p, p, p, i64, i64, i32, p]
+        L.ref_fp4_gemm.restype = i32
+        L.ref_fp4_gemm.argtypes = [p, p, C.c_float, p, p, C.c_float, i64, i64, i64, i32, p]
         L.ref_dequantize_unrotate.restype = i32
         L.ref_dequantize_unrotate.argtypes = [p, p, p, i64, i64, i32, i32, i32, p, p]
         for name in ("ref_rne_e2m1_array", "ref_rne_e4m3_array"):
@@ -246,6 +248,22 @@ def dequantize_unrotate(codes, scales, global_scale, rows, cols, fmt="nvfp4", bl
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")
     return of if out == "f32" else ob
+
+
+def fp4_gemm(a_codes, a_scales, a_sg, b_codes, b_scales, b_sg, fmt="nvfp4"):
+    """D = s_a s_b A B^T from packed codes and row-major block scales (float32)."""
+    a_codes = np.ascontiguousarray(a_codes, np.uint8)
+    b_codes = np.ascontiguousarray(b_codes, np.uint8)
+    a_scales = np.ascontiguousarray(a_scales, np.uint8)
+    b_scales = np.ascontiguousarray(b_scales, np.uint8)
+    M, K = a_codes.shape[0], 2 * a_codes.shape[1]
+    N = b_codes.shape[0]
+    d = np.zeros((M, N), np.float32)
+    rc = lib().ref_fp4_gemm(_ptr(a_codes), _ptr(a_scales), float(a_sg or 1.0), _ptr(b_codes),
+                            _ptr(b_scales), float(b_sg or 1.0), M, N, K, _fmt(fmt), _ptr(d))
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return d
 
 
 def block_mse(x_bf16, codes, scales, global_scale, fmt="nvfp4", block=16, rot=0):

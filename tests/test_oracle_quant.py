@@ -416,3 +416,41 @@ def test_rotated_round_trip_error_equals_block_sse(ref, fmt, block, rot):
     err = np.sum((f32_of_bf16(x).astype(np.float64) - back.astype(np.float64)) ** 2)
     sse = np.sum(q["mse"].astype(np.float64) * block)
     assert abs(err - sse) <= 1e-4 * sse
+
+
+# ----------------------------------------------------- FP4 x FP4 matrix product
+
+@pytest.mark.parametrize("fmt,block", [("nvfp4", 16), ("mxfp4", 32)])
+def test_fp4_gemm_equals_product_of_dequantized(ref, fmt, block):
+    # the product of the two dequantized operands (numpy's float64 matmul of the
+    # oracle's own dequantized values) times the two global scales
+    rng = np.random.default_rng(7)
+    M, N, K = 5, 7, 4 * block
+    ac = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    bc = rng.integers(0, 256, (N, K // 2), dtype=np.uint8)
+    hi = 0x50 if fmt == "nvfp4" else 140
+    lo = 0x20 if fmt == "nvfp4" else 110
+    asc = rng.integers(lo, hi, (M, K // block), dtype=np.uint8)
+    bsc = rng.integers(lo, hi, (N, K // block), dtype=np.uint8)
+    sa, sb = (0.75, 1.5) if fmt == "nvfp4" else (None, None)
+    d = ref.fp4_gemm(ac, asc, sa, bc, bsc, sb, fmt)
+    da = ref.dequantize(ac, asc, 1.0, M, K, fmt, block).astype(np.float64)
+    db = ref.dequantize(bc, bsc, 1.0, N, K, fmt, block).astype(np.float64)
+    want = (da @ db.T) * ((sa * sb) if fmt == "nvfp4" else 1.0)
+    assert np.array_equal(d, want.astype(np.float32))
+
+
+def test_fp4_gemm_one_hot_rows(ref):
+    # B rows that select one column of A: code 0x2 (value 1) at k = j, scale 1
+    M, K = 4, 32
+    rng = np.random.default_rng(3)
+    ac = rng.integers(0, 256, (M, K // 2), dtype=np.uint8)
+    asc = np.full((M, K // 16), 0x38, np.uint8)  # E4M3 1.0
+    cols = [0, 5, 17, 31]
+    bc = np.zeros((len(cols), K // 2), np.uint8)
+    for n, j in enumerate(cols):
+        bc[n, j // 2] = 0x2 << (4 * (j % 2))
+    bsc = np.full((len(cols), K // 16), 0x38, np.uint8)
+    d = ref.fp4_gemm(ac, asc, 2.0, bc, bsc, 0.5, "nvfp4")
+    a = ref.dequantize(ac, asc, 1.0, M, K, "nvfp4", 16)
+    assert np.array_equal(d, a[:, cols])
