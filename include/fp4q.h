@@ -138,6 +138,48 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
                                      fp4q_dtype out_dtype, cudaStream_t stream);
 
 /*
+ * W4A4 FP4 GEMM on the tcgen05 block-scaled tensor cores -- the consumer of
+ * the quantizer's output ("Bridging the Gap Between Promise and Performance
+ * for Microscaling FP4 Quantization", 技術概要 §2.3: MXFP4 / NVFP4 matrix
+ * multiplication on Blackwell SM100; §2.2 item 3: activations rotated and
+ * quantized online in front of it).
+ *
+ * fp4q_mma_scale_bytes -- size in bytes of the scale buffer that
+ * fp4q_scales_to_mma fills for a [rows, K] operand (rows padded to 128, blocks
+ * to 4). 0 for invalid arguments (rows <= 0, K not a multiple of the block:
+ * 16 for NVFP4, 32 for MXFP4). Host only; no GPU work.
+ *
+ * fp4q_scales_to_mma -- reorders the row-major block scales written by
+ * fp4q_quantize (uint8 [rows, K/block]) into the block-scaled MMA's layout:
+ * 512-byte atoms of 128 rows x 4 blocks, row r of an atom at byte
+ * 16 (r % 32) + 4 (r / 32), block j at + j; atoms along K first; padding
+ * bytes are zero. mma_scales: device, fp4q_mma_scale_bytes(rows, K, fmt)
+ * bytes, caller-owned. Errors: UNSUPPORTED (fmt), SHAPE, NULL, CUDA.
+ *
+ * fp4q_gemm -- D[m, n] = alpha * sum_k A[m, k] * B[n, k], where A [M, K] and
+ * B [N, K] (a weight in PyTorch's Linear layout) are packed E2M1 codes as
+ * written by fp4q_quantize (uint8 [rows, K/2], K contiguous, element 2j in
+ * the low nibble) with their block scales in MMA layout (fp4q_scales_to_mma
+ * of the same rows and K). NVFP4: alpha = s_g(A) * s_g(B) from the two device
+ * global scales; MXFP4: alpha = 1 (global scales ignored, may be NULL).
+ * alpha_out: a caller-owned device float the library writes alpha into before
+ * the GEMM reads it (so overlapping calls need distinct alpha_out). d: device
+ * row-major [M, N] of d_dtype (fp32, or bf16 = RNE of the fp32 result).
+ * Products are accumulated in fp32 on the tensor cores (order not specified).
+ * K must be a multiple of 32 and N of 4 (fp32 output) or 8 (bf16); code,
+ * scale and output pointers 16-byte aligned. Errors: UNSUPPORTED (fmt,
+ * d_dtype), SHAPE, NULL, ALIGN, CUDA (also when the GEMM rejects the shape).
+ */
+size_t fp4q_mma_scale_bytes(int64_t rows, int64_t K, fp4q_format fmt);
+fp4q_status fp4q_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, fp4q_format fmt,
+                               uint8_t* mma_scales, cudaStream_t stream);
+fp4q_status fp4q_gemm(const uint8_t* a_codes, const uint8_t* a_mma_scales,
+                      const float* a_global_scale, const uint8_t* b_codes,
+                      const uint8_t* b_mma_scales, const float* b_global_scale, int64_t M,
+                      int64_t N, int64_t K, fp4q_format fmt, float* alpha_out, void* d,
+                      fp4q_dtype d_dtype, cudaStream_t stream);
+
+/*
  * fp4q_block_mse -- per-block mean squared error of x (rotated by rot first)
  * against dequantize(codes, scales): tree sum of (y - yhat)^2 divided by
  * block ("Finer is Better (with the Right Scaling)", 手法 1: MSE per block

@@ -160,6 +160,46 @@ def focus_bwd(w: torch.Tensor, g: torch.Tensor, c: torch.Tensor, sub: int = 8,
     return out
 
 
+def mma_scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
+    n = _abi.load().fp4q_mma_scale_bytes(rows, K, _fmt(fmt))
+    if n == 0:
+        raise ValueError(f"no MMA scale layout for rows={rows}, K={K}, {fmt}")
+    return n
+
+
+def scales_to_mma(scales: torch.Tensor, K: int, fmt="nvfp4",
+                  out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Row-major block scales [rows, K/block] -> the block-scaled MMA layout
+    (flat uint8 of mma_scale_bytes(rows, K, fmt) bytes)."""
+    _check(scales, torch.uint8, "scales")
+    rows = scales.shape[0]
+    if out is None:
+        out = torch.empty(mma_scale_bytes(rows, K, fmt), dtype=torch.uint8, device=scales.device)
+    _abi.call("fp4q_scales_to_mma", scales.data_ptr(), rows, K, _fmt(fmt), out.data_ptr(), _stream())
+    return out
+
+
+def gemm(a_codes: torch.Tensor, a_mma_scales: torch.Tensor, a_global_scale: Optional[torch.Tensor],
+         b_codes: torch.Tensor, b_mma_scales: torch.Tensor, b_global_scale: Optional[torch.Tensor],
+         fmt="nvfp4", out_dtype: torch.dtype = torch.bfloat16, out: Optional[torch.Tensor] = None,
+         alpha_out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """W4A4 GEMM on the block-scaled tensor cores: [M, K] x [N, K]^T -> [M, N].
+    Codes as written by quantize; scales converted by scales_to_mma."""
+    for t, nm in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_mma_scales, "a_mma_scales"),
+                  (b_mma_scales, "b_mma_scales")):
+        _check(t, torch.uint8, nm)
+    M, K = a_codes.shape[0], 2 * a_codes.shape[1]
+    N = b_codes.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a_codes.device)
+    if alpha_out is None:
+        alpha_out = torch.empty(1, dtype=torch.float32, device=a_codes.device)
+    _abi.call("fp4q_gemm", a_codes.data_ptr(), a_mma_scales.data_ptr(), _ptr(a_global_scale),
+              b_codes.data_ptr(), b_mma_scales.data_ptr(), _ptr(b_global_scale), M, N, K, _fmt(fmt),
+              alpha_out.data_ptr(), out.data_ptr(), DTYPES[out.dtype], _stream())
+    return out
+
+
 def global_amax(x: torch.Tensor, rot: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     _check(x, torch.bfloat16, "x")
     rows, cols = x.shape

@@ -29,6 +29,25 @@ CFLAGS = ARCH + ["-O3", "-std=c++17", "-lineinfo", "-fmad=false", "-prec-div=tru
                  "-I" + INCLUDE, "-I" + CSRC]
 
 
+def _cutlass_include() -> list[str]:
+    """CUTLASS/CuTe header trees (vendored with flashinfer in this image),
+    used by the GEMM sources only."""
+    import importlib.util
+    spec = importlib.util.find_spec("flashinfer")
+    if spec is None or not spec.submodule_search_locations:
+        raise RuntimeError("CUTLASS headers not found (flashinfer's vendored copy)")
+    base = os.path.join(list(spec.submodule_search_locations)[0], "data", "cutlass")
+    inc = [os.path.join(base, "include"), os.path.join(base, "tools", "util", "include")]
+    if not os.path.exists(os.path.join(inc[0], "cutlass", "cutlass.h")):
+        raise RuntimeError(f"CUTLASS headers not found under {base}")
+    return ["-I" + d for d in inc] + ["--expt-relaxed-constexpr"]
+
+
+def _flags_for(src: str) -> list[str]:
+    name = os.path.basename(src)
+    return CFLAGS + (_cutlass_include() if name.startswith("gemm_") else [])
+
+
 def _nvcc() -> str:
     p = shutil.which("nvcc") or "/usr/local/cuda/bin/nvcc"
     if not os.path.exists(p):
@@ -62,7 +81,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
 
     def compile_one(pair):
         src, obj = pair
-        cmd = [nvcc] + CFLAGS + ["-c", src, "-o", obj]
+        cmd = [nvcc] + _flags_for(src) + ["-c", src, "-o", obj]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"nvcc failed on {src}:\n{r.stdout}\n{r.stderr}")

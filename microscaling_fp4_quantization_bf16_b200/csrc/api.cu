@@ -277,6 +277,68 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
     return cuda_status(launch_dequant_rot(nv ? 0 : 1, block, rot, a, stream));
 }
 
+size_t fp4q_mma_scale_bytes(int64_t rows, int64_t K, fp4q_format fmt)
+{
+    const int sfv = fmt == FP4Q_FMT_NVFP4 ? 16 : (fmt == FP4Q_FMT_MXFP4 ? 32 : 0);
+    if (sfv == 0 || rows <= 0 || K <= 0 || K % sfv != 0 || rows > 0x7FFFFFFF || K > 0x7FFFFFFF)
+        return 0;
+    return mma_scale_bytes(rows, K, sfv);
+}
+
+fp4q_status fp4q_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, fp4q_format fmt,
+                               uint8_t* mma_scales, cudaStream_t stream)
+{
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+        return FP4Q_ERR_UNSUPPORTED;
+    const int sfv = fmt == FP4Q_FMT_NVFP4 ? 16 : 32;
+    if (rows <= 0 || K <= 0 || K % sfv != 0 || rows > 0x7FFFFFFF || K > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    if (scales == nullptr || mma_scales == nullptr)
+        return FP4Q_ERR_NULL;
+    return cuda_status(launch_scales_to_mma(scales, rows, K, sfv, mma_scales, stream));
+}
+
+fp4q_status fp4q_gemm(const uint8_t* a_codes, const uint8_t* a_mma_scales,
+                      const float* a_global_scale, const uint8_t* b_codes,
+                      const uint8_t* b_mma_scales, const float* b_global_scale, int64_t M,
+                      int64_t N, int64_t K, fp4q_format fmt, float* alpha_out, void* d,
+                      fp4q_dtype d_dtype, cudaStream_t stream)
+{
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (d_dtype != FP4Q_OUT_F32 && d_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t nalign = d_dtype == FP4Q_OUT_F32 ? 4 : 8;  // 16-byte output rows
+    if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || N % nalign != 0 || M > 0x7FFFFFFF ||
+        N > 0x7FFFFFFF || K > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    if (a_codes == nullptr || a_mma_scales == nullptr || b_codes == nullptr ||
+        b_mma_scales == nullptr || alpha_out == nullptr || d == nullptr)
+        return FP4Q_ERR_NULL;
+    if (nv && (a_global_scale == nullptr || b_global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(a_codes) || !aligned16(a_mma_scales) || !aligned16(b_codes) ||
+        !aligned16(b_mma_scales) || !aligned16(d) || !aligned4(alpha_out) ||
+        (nv && (!aligned4(a_global_scale) || !aligned4(b_global_scale))))
+        return FP4Q_ERR_ALIGN;
+    fp4q_status st = cuda_status(
+        launch_alpha(nv ? a_global_scale : nullptr, nv ? b_global_scale : nullptr, alpha_out, stream));
+    if (st != FP4Q_OK)
+        return st;
+    const int m = (int)M, n = (int)N, k = (int)K;
+    cudaError_t e;
+    if (nv)
+        e = d_dtype == FP4Q_OUT_F32
+                ? launch_gemm_nv_f32(a_codes, a_mma_scales, b_codes, b_mma_scales, m, n, k, alpha_out, d, stream)
+                : launch_gemm_nv_bf16(a_codes, a_mma_scales, b_codes, b_mma_scales, m, n, k, alpha_out, d, stream);
+    else
+        e = d_dtype == FP4Q_OUT_F32
+                ? launch_gemm_mx_f32(a_codes, a_mma_scales, b_codes, b_mma_scales, m, n, k, alpha_out, d, stream)
+                : launch_gemm_mx_bf16(a_codes, a_mma_scales, b_codes, b_mma_scales, m, n, k, alpha_out, d, stream);
+    return cuda_status(e);
+}
+
 fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* scales,
                            const float* global_scale, int64_t rows, int64_t cols,
                            fp4q_format fmt, int block, int rot, float* block_mse,

@@ -347,6 +347,20 @@ cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a,
     }
 }
 
+// ------------------------------------------------------------ GEMM alpha
+
+// alpha = s_g(A) * s_g(B) for the NVFP4 GEMM (1 for MXFP4: both NULL).
+__global__ void alpha_kernel(const float* sga, const float* sgb, float* alpha)
+{
+    pdl_begin();
+    *alpha = (sga != nullptr && sgb != nullptr) ? __fmul_rn(*sga, *sgb) : 1.0f;
+}
+
+cudaError_t launch_alpha(const float* sga, const float* sgb, float* alpha, cudaStream_t st)
+{
+    return launch_pdl(alpha_kernel, dim3(1), dim3(1), 0, st, sga, sgb, alpha);
+}
+
 // ------------------------------------------------------------ block MSE
 
 template <int B, int ROT, bool MX>

@@ -115,6 +115,20 @@ cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a,
 cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st);
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);
+// W4A4 FP4 GEMM (gemm_*.cu): scale layout for the block-scaled MMA and the
+// four GEMM configurations (NVFP4 / MXFP4 x fp32 / bf16 output).
+size_t mma_scale_bytes(int64_t rows, int64_t K, int sfv);
+cudaError_t launch_scales_to_mma(const uint8_t* src, int64_t rows, int64_t K, int sfv, uint8_t* dst,
+                                 cudaStream_t st);
+cudaError_t launch_alpha(const float* sga, const float* sgb, float* alpha, cudaStream_t st);
+#define FP4Q_DECLARE_GEMM(NAME)                                                                  \
+    cudaError_t NAME(const uint8_t* a, const uint8_t* sfa, const uint8_t* b, const uint8_t* sfb, \
+                     int M, int N, int K, const float* alpha, void* d, cudaStream_t st);
+FP4Q_DECLARE_GEMM(launch_gemm_nv_f32)
+FP4Q_DECLARE_GEMM(launch_gemm_nv_bf16)
+FP4Q_DECLARE_GEMM(launch_gemm_mx_f32)
+FP4Q_DECLARE_GEMM(launch_gemm_mx_bf16)
+#undef FP4Q_DECLARE_GEMM
 cudaError_t launch_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream_t st);
 cudaError_t launch_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 

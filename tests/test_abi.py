@@ -150,3 +150,20 @@ def test_python_wrapper_rejects_cpu_tensors():
     with pytest.raises(ValueError):
         fp4q.focus_bwd(torch.zeros(4, 64, dtype=torch.bfloat16),
                        torch.zeros(4, 64, dtype=torch.bfloat16), torch.zeros(4, 8))
+
+
+def test_gemm_validation(lib):
+    L = lib
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 128, 48, NV, A, A, 0, None) == SHAPE  # K % 32
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 130, 64, NV, A, A, 0, None) == SHAPE  # N % 4 (fp32)
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 132, 64, NV, A, A, 1, None) == SHAPE  # N % 8 (bf16)
+    assert L.fp4q_gemm(A, A, None, A, A, A, 128, 128, 64, NV, A, A, 0, None) == NULL  # NVFP4 s_g
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 128, 64, NV, None, A, 0, None) == NULL  # alpha_out
+    assert L.fp4q_gemm(MIS, A, A, A, A, A, 128, 128, 64, NV, A, A, 0, None) == ALIGN
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 128, 64, 2, A, A, 0, None) == UNSUP
+    assert L.fp4q_gemm(A, A, A, A, A, A, 128, 128, 64, NV, A, A, 5, None) == UNSUP
+    assert L.fp4q_mma_scale_bytes(128, 48, NV) == 512   # 128 rows x 3 blocks, padded to 4
+    assert L.fp4q_mma_scale_bytes(300, 64, MX) == 384 * 4  # rows padded to 384, 2 blocks -> 4
+    assert L.fp4q_mma_scale_bytes(128, 40, NV) == 0
+    assert L.fp4q_scales_to_mma(A, 128, 40, NV, A, None) == SHAPE
+    assert L.fp4q_scales_to_mma(None, 128, 64, NV, A, None) == NULL
