@@ -452,6 +452,34 @@ def breakdown(dev, peaks, reps: int = 10):
                                                   "brute_force")], want_mse=True)
     quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
                                           ("mxfp4", 32, "absmax", 128)])
+    # W4A4 GEMM on the block-scaled tensor cores, LLM layer shapes (tokens x hidden
+    # -> out): operands quantized (abs-max) once, scales in MMA layout; timed: the
+    # GEMM alone (alpha + tcgen05 GEMM), bf16 output. Roofline: the dense FP4 peak
+    # taken as the measured bf16 peak x 4 (the nominal fp4 / bf16 ratio).
+    fp4_peak = peaks["bf16_tflops"] * 4.0
+    for fmt, block in (("nvfp4", 16), ("mxfp4", 32)):
+        for M, N, K in ((8192, 4096, 4096), (8192, 4096, 14336)):
+            a = torch.randn(M, K, device=dev).to(torch.bfloat16)
+            w = (torch.randn(N, K, device=dev) * 0.02).to(torch.bfloat16)
+            qa = fp4q.quantize(a, fmt, block, "absmax", 0)
+            qw = fp4q.quantize(w, fmt, block, "absmax", 0)
+            sa, sw = fp4q.scales_to_mma(qa.scales, K, fmt), fp4q.scales_to_mma(qw.scales, K, fmt)
+            dout = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            alpha = torch.empty(1, device=dev)
+            secs = timeit([lambda: fp4q.gemm(qa.codes, sa, qa.global_scale, qw.codes, sw,
+                                             qw.global_scale, fmt, out=dout, alpha_out=alpha)])
+            tf = 2.0 * M * N * K / secs / 1e12
+            # the same layer in bf16 through torch.matmul (cuBLAS), for the
+            # layer-wise speedup the pages quote (context, not a target)
+            ref_secs = timeit([lambda: torch.matmul(a, w.t(), out=dout)])
+            rows_out.append({"run": f"w4a4 gemm {fmt} M={M} N={N} K={K} -> bf16", "us": round(secs * 1e6, 2),
+                             "tflops": round(tf, 1), "bound": "tensor",
+                             "tensor_frac": round(tf / fp4_peak, 4),
+                             "peak_tflops": fp4_peak, "peak_source": "measured bf16 x 4 (nominal fp4/bf16)",
+                             "bf16_matmul_us": round(ref_secs * 1e6, 2),
+                             "speedup_vs_bf16": round(ref_secs / secs, 2), "launches": 2})
+            del a, w, qa, qw, sa, sw, dout
+    torch.cuda.empty_cache()
     # FOCUS
     d = synth.workload("c4_focus")
     w0, c0, g0 = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)
