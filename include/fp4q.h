@@ -170,6 +170,20 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
  * scale and output pointers 16-byte aligned. Errors: UNSUPPORTED (fmt,
  * d_dtype), SHAPE, NULL, ALIGN, CUDA (also when the GEMM rejects the shape).
  */
+/*
+ * fp4q_quantize_mma -- fp4q_quantize (block 16 for NVFP4, 32 for MXFP4; no MSE or
+ * dq outputs) writing the scale bytes straight into the block-scaled MMA
+ * layout of fp4q_scales_to_mma: the quantizer feeding fp4q_gemm in one launch
+ * (rotation fused in front, "Bridging the Gap ...", 技術概要 §2.2 item 3).
+ * mma_scales: fp4q_mma_scale_bytes(rows, cols, fmt) bytes whose padding bytes
+ * (rows past rows, blocks past cols / block) must already be zero -- only the
+ * real blocks are written. cols % 32 == 0 and rows * cols / 32 < 2^32.
+ * Other arguments and errors as fp4q_quantize.
+ */
+fp4q_status fp4q_quantize_mma(const void* x, int64_t rows, int64_t cols, fp4q_format fmt,
+                              fp4q_strategy strat, int rot, const float* global_amax_in,
+                              float* global_scale_out, uint8_t* codes, uint8_t* mma_scales,
+                              cudaStream_t stream);
 size_t fp4q_mma_scale_bytes(int64_t rows, int64_t K, fp4q_format fmt);
 fp4q_status fp4q_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, fp4q_format fmt,
                                uint8_t* mma_scales, cudaStream_t stream);

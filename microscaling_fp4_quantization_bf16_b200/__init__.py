@@ -167,6 +167,30 @@ def mma_scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
     return n
 
 
+def quantize_mma(x: torch.Tensor, fmt="nvfp4", strategy="absmax", rot: int = 0,
+                 global_amax: Optional[torch.Tensor] = None,
+                 out: Optional[Quantized] = None) -> Quantized:
+    """quantize() with the scales written in the block-scaled MMA layout (block 16
+    for NVFP4, 32 for MXFP4): the activation side of gemm() in one launch. The
+    returned Quantized holds the flat MMA-layout scale bytes in .scales."""
+    _check(x, torch.bfloat16, "x")
+    rows, cols = x.shape
+    f = _fmt(fmt)
+    if out is None:
+        dev = x.device
+        out = Quantized(
+            codes=torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev),
+            scales=torch.zeros(mma_scale_bytes(rows, cols, fmt), dtype=torch.uint8, device=dev),
+            global_scale=torch.empty(1, dtype=torch.float32, device=dev) if f == 0 else None,
+            mse=None, dq=None)
+    if global_amax is not None:
+        _check(global_amax, torch.float32, "global_amax")
+    _abi.call("fp4q_quantize_mma", x.data_ptr(), rows, cols, f, _strat(strategy), rot,
+              _ptr(global_amax), _ptr(out.global_scale), out.codes.data_ptr(), out.scales.data_ptr(),
+              _stream())
+    return out
+
+
 def scales_to_mma(scales: torch.Tensor, K: int, fmt="nvfp4",
                   out: Optional[torch.Tensor] = None) -> torch.Tensor:
     """Row-major block scales [rows, K/block] -> the block-scaled MMA layout

@@ -156,12 +156,15 @@ fp4q_status accumulate_amax(const void* x, int64_t n, int rot, float* global_sca
 
 }  // namespace
 
-extern "C" {
+namespace {
 
-fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+// fp4q_quantize and fp4q_quantize_mma: mma != 0 writes the scale bytes in the
+// block-scaled MMA layout instead of row-major.
+fp4q_status quantize_impl(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
                           fp4q_strategy strat, int rot, const float* global_amax_in,
                           float* global_scale_out, uint8_t* codes, uint8_t* scales,
-                          float* block_mse, void* dq, fp4q_dtype dq_dtype, cudaStream_t stream)
+                          float* block_mse, void* dq, fp4q_dtype dq_dtype, bool mma,
+                          cudaStream_t stream)
 {
     fp4q_status st = check_format(rows, cols, fmt, block, rot);
     if (st != FP4Q_OK)
@@ -199,6 +202,12 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
     a.amax = nullptr;
     a.sg_out = nullptr;
     a.keep = 0xFFFFFFFFu;
+    a.mma_spr = 0;
+    a.mma_atoms_k = 0;
+    if (mma) {  // cols % 32 == 0 and rows * cols / 32 < 2^32 (checked by the caller)
+        a.mma_spr = (uint32_t)(cols / 32);
+        a.mma_atoms_k = (uint32_t)((cols / block + 3) / 4);
+    }
     int kstrat = nv ? (int)strat : (strat == FP4Q_BRUTE_FORCE ? K_MX_BRUTE : K_MX);
     if (nv) {
         if (global_amax_in != nullptr) {
@@ -217,6 +226,34 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
     if (nv && global_amax_in == nullptr)
         st = cuda_status(launch_finalize_sg(global_scale_out, stream));
     return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                          fp4q_strategy strat, int rot, const float* global_amax_in,
+                          float* global_scale_out, uint8_t* codes, uint8_t* scales,
+                          float* block_mse, void* dq, fp4q_dtype dq_dtype, cudaStream_t stream)
+{
+    return quantize_impl(x, rows, cols, fmt, block, strat, rot, global_amax_in, global_scale_out,
+                         codes, scales, block_mse, dq, dq_dtype, false, stream);
+}
+
+fp4q_status fp4q_quantize_mma(const void* x, int64_t rows, int64_t cols, fp4q_format fmt,
+                              fp4q_strategy strat, int rot, const float* global_amax_in,
+                              float* global_scale_out, uint8_t* codes, uint8_t* mma_scales,
+                              cudaStream_t stream)
+{
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0 || cols % 32 != 0 || (rows > 0 && rows * (cols / 32) > 0xFFFFFFFFll) ||
+        rows > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    return quantize_impl(x, rows, cols, fmt, fmt == FP4Q_FMT_NVFP4 ? 16 : 32, strat, rot,
+                         global_amax_in, global_scale_out, codes, mma_scales, nullptr, nullptr,
+                         FP4Q_OUT_F32, true, stream);
 }
 
 fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,

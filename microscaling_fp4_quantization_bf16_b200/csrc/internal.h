@@ -45,6 +45,9 @@ struct QuantArgs {
     void* dq;               // [n] or NULL
     int dq_kind;            // 0 none, 1 fp32, 2 bf16
     uint32_t keep;          // 0xFFFFFFFF, passed at run time (see encode_seg)
+    uint32_t mma_spr;       // 0: row-major scales; else segments per row, and scales are
+                            // written in the block-scaled MMA layout (see gemm_sf.cu)
+    uint32_t mma_atoms_k;   // MMA layout: 4-block atoms per 128-row tile along K
 };
 
 struct DequantArgs {

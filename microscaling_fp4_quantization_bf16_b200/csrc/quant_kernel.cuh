@@ -311,7 +311,19 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
 
     if (nvalid == SEG) {
         *reinterpret_cast<uint4*>(a.codes + s * (SEG / 2)) = make_uint4(q[0], q[1], q[2], q[3]);
-        store_bytes<NB>(a.scales + s * NB, sc);
+        if (NB <= 2 && a.mma_spr != 0) {
+            // block-scaled MMA layout: 512-byte atoms of 128 rows x 4 blocks (row r
+            // at 16 (r % 32) + 4 (r / 32 % 4), block j at + j % 4), atoms along K
+            // first. Blocks of 16 or 32 only: the segment's first block is even,
+            // so its one or two bytes are adjacent inside one atom row.
+            const uint32_t r = (uint32_t)s / a.mma_spr;
+            const uint32_t kb = ((uint32_t)s - r * a.mma_spr) * NB;
+            const int64_t off = ((int64_t)(r >> 7) * a.mma_atoms_k + (kb >> 2)) * 512 +
+                                16 * (r & 31) + 4 * ((r >> 5) & 3) + (kb & 3);
+            store_bytes<NB>(a.scales + off, sc);
+        } else {
+            store_bytes<NB>(a.scales + s * NB, sc);
+        }
         if (a.mse != nullptr)
             store_floats<NB>(a.mse + s * NB, m);
     } else {

@@ -167,3 +167,9 @@ def test_gemm_validation(lib):
     assert L.fp4q_mma_scale_bytes(128, 40, NV) == 0
     assert L.fp4q_scales_to_mma(A, 128, 40, NV, A, None) == SHAPE
     assert L.fp4q_scales_to_mma(None, 128, 64, NV, A, None) == NULL
+    qm = lambda **k: L.fp4q_quantize_mma(A, 4, k.get("cols", 64), k.get("fmt", NV), 0, 0, None,
+                                         A3, A2, k.get("sc", A), None)
+    assert qm(cols=48) == SHAPE      # not a multiple of 32
+    assert qm(fmt=3) == UNSUP
+    assert qm(sc=None) == NULL
+    assert qm(sc=MIS) == ALIGN

@@ -80,3 +80,22 @@ def test_gemm_matches_oracle(gpu, fmt, block, M, N, K, out_dtype):
     got, want, tol = gemm_case(gpu, fmt, block, M, N, K, out_dtype, seed=M + N + K)
     bad = np.abs(got - want) > tol
     assert not bad.any(), f"{bad.sum()} of {bad.size} outside the fp32 summation bound"
+
+
+@pytest.mark.parametrize("fmt,block,strat,rot", [("nvfp4", 16, "absmax", 0), ("nvfp4", 16, "four_over_six", 16),
+                                                 ("mxfp4", 32, "absmax", 32), ("mxfp4", 32, "brute_force", 0)])
+@pytest.mark.parametrize("rows,cols", [(300, 256), (128, 2048), (7, 64)])
+def test_quantize_mma_equals_quantize_then_convert(gpu, fmt, block, strat, rot, rows, cols):
+    """The fused quantizer writes the same codes as quantize() and the same scale
+    bytes as scales_to_mma() of its row-major scales (padding zero)."""
+    if cols % max(rot, 1):
+        pytest.skip("cols must be a multiple of the rotation")
+    x = synth.laplace_outliers(rows, cols, seed=rows + cols).cuda()
+    q = gpu.quantize(x, fmt, block, strat, rot)
+    conv = gpu.scales_to_mma(q.scales, cols, fmt)
+    f = gpu.quantize_mma(x, fmt, strat, rot)
+    torch.cuda.synchronize()
+    assert np.array_equal(f.codes.cpu().numpy(), q.codes.cpu().numpy())
+    assert np.array_equal(f.scales.cpu().numpy(), conv.cpu().numpy())
+    if fmt == "nvfp4":
+        assert f.global_scale.item() == q.global_scale.item()
