@@ -478,7 +478,23 @@ def breakdown(dev, peaks, reps: int = 10):
                              "peak_tflops": fp4_peak, "peak_source": "measured bf16 x 4 (nominal fp4/bf16)",
                              "bf16_matmul_us": round(ref_secs * 1e6, 2),
                              "speedup_vs_bf16": round(ref_secs / secs, 2), "launches": 2})
-            del a, w, qa, qw, sa, sw, dout
+            # the whole W4A4 layer: the activations rotated (MXFP4: 32-wide Hadamard;
+            # NVFP4: none, its abs-max computed on the device) and quantized straight
+            # into the MMA scale layout, then the GEMM against the pre-quantized weight
+            rot = 32 if fmt == "mxfp4" else 0
+            qw2 = fp4q.quantize_mma(w, fmt, "absmax", rot)
+            qa2 = fp4q.quantize_mma(a, fmt, "absmax", rot)
+            layer = [lambda: (fp4q.quantize_mma(a, fmt, "absmax", rot, out=qa2),
+                              fp4q.gemm(qa2.codes, qa2.scales, qa2.global_scale, qw2.codes, qw2.scales,
+                                        qw2.global_scale, fmt, out=dout, alpha_out=alpha))]
+            lsecs = timeit(layer)
+            rows_out.append({"run": f"w4a4 layer {fmt} (rot {rot}) quantize activations + gemm "
+                                    f"M={M} N={N} K={K} -> bf16", "us": round(lsecs * 1e6, 2),
+                             "tflops": round(2.0 * M * N * K / lsecs / 1e12, 1), "bound": "tensor",
+                             "bf16_matmul_us": round(ref_secs * 1e6, 2),
+                             "speedup_vs_bf16": round(ref_secs / lsecs, 2),
+                             "launches": 2 + (3 if fmt == "nvfp4" else 1)})
+            del a, w, qa, qw, sa, sw, dout, qa2, qw2
     torch.cuda.empty_cache()
     # FOCUS
     d = synth.workload("c4_focus")
