@@ -171,6 +171,24 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
  * d_dtype), SHAPE, NULL, ALIGN, CUDA (also when the GEMM rejects the shape).
  */
 /*
+ * fp4q_gemm_noalloc -- fp4q_gemm without the alpha_out argument: alpha is
+ * written into a 256-byte scratch array inside the library image (one float
+ * of it is used) instead of a caller-owned device float. For callers that
+ * cannot hand over memory on the call path. Limits: all calls on a device
+ * share that one scratch float, so calls that overlap (in flight at the same
+ * time on different streams or threads) race on it -- serialise them or use
+ * fp4q_gemm; the first call on each device looks the scratch address up
+ * (cudaGetSymbolAddress), so make that first call before any stream capture
+ * begins. The pages have no counterpart: this is an interface detail. Other
+ * arguments, results and errors as fp4q_gemm.
+ */
+fp4q_status fp4q_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_mma_scales,
+                              const float* a_global_scale, const uint8_t* b_codes,
+                              const uint8_t* b_mma_scales, const float* b_global_scale, int64_t M,
+                              int64_t N, int64_t K, fp4q_format fmt, void* d, fp4q_dtype d_dtype,
+                              cudaStream_t stream);
+
+/*
  * fp4q_quantize_mma -- fp4q_quantize (block 16 for NVFP4, 32 for MXFP4; no MSE or
  * dq outputs) writing the scale bytes straight into the block-scaled MMA
  * layout of fp4q_scales_to_mma: the quantizer feeding fp4q_gemm in one launch

@@ -224,6 +224,26 @@ def gemm(a_codes: torch.Tensor, a_mma_scales: torch.Tensor, a_global_scale: Opti
     return out
 
 
+def gemm_noalloc(a_codes: torch.Tensor, a_mma_scales: torch.Tensor,
+                 a_global_scale: Optional[torch.Tensor], b_codes: torch.Tensor,
+                 b_mma_scales: torch.Tensor, b_global_scale: Optional[torch.Tensor], fmt="nvfp4",
+                 out: Optional[torch.Tensor] = None,
+                 out_dtype: torch.dtype = torch.bfloat16) -> torch.Tensor:
+    """gemm() using the library's own scratch float for alpha (no alpha_out);
+    overlapping calls on one device race on it (see fp4q_gemm_noalloc)."""
+    for t, nm in ((a_codes, "a_codes"), (b_codes, "b_codes"), (a_mma_scales, "a_mma_scales"),
+                  (b_mma_scales, "b_mma_scales")):
+        _check(t, torch.uint8, nm)
+    M, K = a_codes.shape[0], 2 * a_codes.shape[1]
+    N = b_codes.shape[0]
+    if out is None:
+        out = torch.empty(M, N, dtype=out_dtype, device=a_codes.device)
+    _abi.call("fp4q_gemm_noalloc", a_codes.data_ptr(), a_mma_scales.data_ptr(), _ptr(a_global_scale),
+              b_codes.data_ptr(), b_mma_scales.data_ptr(), _ptr(b_global_scale), M, N, K, _fmt(fmt),
+              out.data_ptr(), DTYPES[out.dtype], _stream())
+    return out
+
+
 def global_amax(x: torch.Tensor, rot: int = 0, out: Optional[torch.Tensor] = None) -> torch.Tensor:
     _check(x, torch.bfloat16, "x")
     rows, cols = x.shape

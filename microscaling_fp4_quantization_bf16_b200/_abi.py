@@ -29,6 +29,7 @@ SIGNATURES = {
     "fp4q_global_amax": (_i32, [_p, _i64, _i64, _i32, _p, _p]),
     "fp4q_e2m1_encode": (_i32, [_p, _i64, _p, _p]),
     "fp4q_e4m3_encode": (_i32, [_p, _i64, _p, _p]),
+    "fp4q_gemm_noalloc": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _i32, _p]),
     "fp4q_quantize_mma": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p]),
     "fp4q_mma_scale_bytes": (C.c_size_t, [_i64, _i64, _i32]),
     "fp4q_scales_to_mma": (_i32, [_p, _i64, _i64, _i32, _p, _p]),
