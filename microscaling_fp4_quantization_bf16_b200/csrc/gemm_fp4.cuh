@@ -10,7 +10,7 @@
 // The kernel is CUTLASS's SM100 block-scaled collective (tcgen05.mma
 // kind::mxf4nvf4 with block scales, TMA-fed shared-memory stages, TMEM
 // accumulators), instantiated here with a 128x128x256 tile and a 1x1x1
-// cluster: no TMA multicast anywhere. No source matrix C is read.
+// cluster: every TMA load is a plain single-CTA copy. No source matrix C is read.
 #pragma once
 
 #include <cuda_runtime.h>

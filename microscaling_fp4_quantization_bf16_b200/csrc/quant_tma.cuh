@@ -3,7 +3,7 @@
 // The flattened bf16 tensor is viewed as rows of 64 elements (128 B). Each
 // CTA is a small pipeline: one producer thread streams tiles of TILE_ROWS
 // rows into a ring of STAGES shared-memory buffers with
-// cp.async.bulk.tensor (TMA, no multicast), completion tracked by mbarriers;
+// cp.async.bulk.tensor (TMA, single-CTA copies), completion tracked by mbarriers;
 // four consumer warps take one 32-element segment per thread per tile, read
 // it with four conflict-free 128-bit shared loads (the tensor map's 128-byte
 // swizzle puts the 16-byte chunk c of row r at c ^ (r mod 8)), release the
