@@ -17,16 +17,18 @@
  * row-major (E4M3 code, or E8M0 byte = exponent + 127). Per-block MSE:
  * float [rows, cols/block]. Dequantized values: [rows, cols] fp32 or bf16.
  *
- * Arithmetic. Every result is bit-identical to the plain CPU definition of
- * the operation: one IEEE binary32 operation per step, no fused
- * multiply-add, E2M1 / E4M3 round-to-nearest-even with saturation, the
+ * Arithmetic. Every result except the GEMM's is bit-identical to the plain
+ * CPU definition of the operation: one IEEE binary32 operation per step, no
+ * fused multiply-add, E2M1 / E4M3 round-to-nearest-even with saturation, the
  * optional Hadamard rotation applied as a Walsh-Hadamard butterfly with
- * ascending stages, and block sums taken with the adjacent-pair tree.
+ * ascending stages, and block sums taken with the adjacent-pair tree. The
+ * GEMM accumulates on the tensor cores in fp32 in the hardware's order.
  *
  * Conventions for every entry point:
  *  - All array pointers are DEVICE pointers owned by the caller, 16-byte
  *    aligned, dense row-major (leading dimension = cols). The library never
- *    allocates, frees, or keeps memory or state between calls, and never
+ *    allocates, frees, or keeps memory or state between calls (the one
+ *    exception is the fixed scratch float of fp4q_gemm_noalloc), and never
  *    synchronises: work is enqueued on `stream` (0 = legacy default stream)
  *    and the call returns before it completes.
  *  - Arguments are validated on the host before anything is enqueued; on an
