@@ -75,6 +75,15 @@ def lib():
         L.ref_focus_fwd.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         L.ref_focus_bwd.restype = i32
         L.ref_focus_bwd.argtypes = [p, p, p, i64, i64, i32, p]
+        L.ref_float_to_fp16.restype = C.c_uint16
+        L.ref_float_to_fp16.argtypes = [C.c_float]
+        f32 = C.c_float
+        L.ref_focus_update.restype = i32
+        L.ref_focus_update.argtypes = [p, p, p, p, p, p, i64, i64, i32, i32, f32, f32, f32, f32,
+                                       i64]
+        L.ref_focus_step.restype = i32
+        L.ref_focus_step.argtypes = [p, i64, i64, i32, i32, i32, p, p, p, p, p, p, p, i32, f32,
+                                     f32, f32, f32, i64]
         L.ref_fp4_gemm.restype = i32
         L.ref_fp4_gemm.argtypes = [p, p, C.c_float, p, p, C.c_float, i64, i64, i64, i32, p]
         L.ref_dequantize_unrotate.restype = i32
@@ -310,6 +319,59 @@ def focus_bwd(w_bf16, g_bf16, c_fp16, sub=8):
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")
     return dc
+
+
+OPT_SGD, OPT_ADAM = 0, 1
+_OPT = {"sgd": OPT_SGD, "adam": OPT_ADAM}
+
+
+def float_to_fp16(v) -> int:
+    return int(lib().ref_float_to_fp16(float(v)))
+
+
+def _opt_state(c, m, v, opt):
+    c = np.array(c, np.float32, copy=True)
+    if opt == "adam":
+        m = np.zeros_like(c) if m is None else np.array(m, np.float32, copy=True)
+        v = np.zeros_like(c) if v is None else np.array(v, np.float32, copy=True)
+    else:
+        m = v = None
+    return c, m, v
+
+
+def focus_update(w_bf16, g_bf16, c, m=None, v=None, sub=8, opt="adam", lr=1e-3, beta1=0.9,
+                 beta2=0.999, eps=1e-8, t=1):
+    """One coefficient update from an external gradient g; returns new copies
+    {"c", "c_half", "m", "v"} (inputs are not modified)."""
+    w = _u16(w_bf16)
+    g = _u16(g_bf16)
+    rows, cols = w.shape
+    c, m, v = _opt_state(c, m, v, opt)
+    ch = np.zeros(c.shape, np.uint16)
+    rc = lib().ref_focus_update(_ptr(w), _ptr(g), _ptr(c), _ptr(ch), _ptr(m), _ptr(v), rows,
+                                cols, sub, _OPT[opt], lr, beta1, beta2, eps, t)
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return {"c": c, "c_half": ch, "m": m, "v": v}
+
+
+def focus_step(w_bf16, c, m=None, v=None, fmt="nvfp4", block=16, sub=8, global_amax=None,
+               opt="adam", lr=1e-3, beta1=0.9, beta2=0.999, eps=1e-8, t=1):
+    """One fused calibration step on the weight-reconstruction loss; returns new
+    copies {"c", "c_half", "m", "v", "sse", "global_scale"}."""
+    w = _u16(w_bf16)
+    rows, cols = w.shape
+    c, m, v = _opt_state(c, m, v, opt)
+    ch = np.zeros(c.shape, np.uint16)
+    sse = np.zeros(c.shape, np.float32)
+    gs = np.zeros(1, np.float32)
+    ga = None if global_amax is None else np.array([global_amax], np.float32)
+    rc = lib().ref_focus_step(_ptr(w), rows, cols, _fmt(fmt), block, sub, _ptr(ga), _ptr(gs),
+                              _ptr(c), _ptr(ch), _ptr(m), _ptr(v), _ptr(sse), _OPT[opt], lr,
+                              beta1, beta2, eps, t)
+    if rc != 0:
+        raise ValueError(f"oracle rejected arguments (rc={rc})")
+    return {"c": c, "c_half": ch, "m": m, "v": v, "sse": sse, "global_scale": gs[0]}
 
 
 def unpack_codes(codes: np.ndarray) -> np.ndarray:

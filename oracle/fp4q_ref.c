@@ -67,6 +67,18 @@
  *      §2.2 item 1 (per group, the scale minimising the MSE) over the
  *      format's own scales: every E8M0 byte 0..254, scanned upward, a strictly
  *      smaller SSE wins, a tie keeps the lower byte.
+ *  R15 FOCUS calibration: the pages learn c by gradient descent through the
+ *      STE but name neither the optimizer nor the precision of the update.
+ *      The learnable state is an fp32 master copy of c; the forward uses its
+ *      fp16 rounding (the pages' FP16 parameter) and the gradient of R9 is
+ *      taken at that fp16 value. Optimizers: plain SGD, and Adam in the
+ *      order of Kingma & Ba's algorithm, with the bias corrections 1 - b^t
+ *      computed in double and rounded once to fp32.
+ *  R16 The fused calibration step minimises the weight-reconstruction loss
+ *      sum (W_hat - W)^2 with g = 2 (W_hat - W) in fp32. (At c == 1 every
+ *      element already lands on its nearest point of the S_dq grid, so this
+ *      loss cannot go lower; losses that couple elements, such as a layer's
+ *      output, are served by the update from an external gradient.)
  */
 #include <float.h>
 #include <math.h>
@@ -800,6 +812,219 @@ int ref_focus_bwd(const uint16_t* w, const uint16_t* g, const uint16_t* c, int64
         float cc = ck * ck;
         dc[k] = -(acc / cc);
     }
+    return REF_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* FOCUS calibration: one optimizer step on the coefficients (R15, R16).     */
+/* ------------------------------------------------------------------------ */
+
+/* float -> IEEE binary16 bits, round to nearest, ties to the even bit
+ * pattern; magnitudes past the largest finite half (65504) round as if 65536
+ * were the next number and then become infinity. The two candidates come from
+ * a binary search over the ordered positive bit patterns 0x0000..0x7BFF,
+ * valued by ref_fp16_to_float. */
+uint16_t ref_float_to_fp16(float v)
+{
+    uint16_t sign = signbit(v) ? 0x8000 : 0;
+    double a = fabs((double)v);
+    if (isnan(v))
+        return (uint16_t)(sign | 0x7E00);
+    if (isinf(v))
+        return (uint16_t)(sign | 0x7C00);
+    int lo = 0, hi = 0x7BFF; /* largest pattern whose value is <= a */
+    if (a >= (double)ref_fp16_to_float(0x7BFF)) {
+        lo = 0x7BFF;
+    } else {
+        while (lo < hi) {
+            int mid = (lo + hi + 1) / 2;
+            if ((double)ref_fp16_to_float((uint16_t)mid) <= a)
+                lo = mid;
+            else
+                hi = mid - 1;
+        }
+    }
+    double vlo = (double)ref_fp16_to_float((uint16_t)lo);
+    if (vlo == a)
+        return (uint16_t)(sign | lo);
+    int up = lo + 1;
+    double vup = (up == 0x7C00) ? 65536.0 : (double)ref_fp16_to_float((uint16_t)up);
+    double dlo = a - vlo, dup = vup - a;
+    int pick;
+    if (dlo < dup)
+        pick = lo;
+    else if (dup < dlo)
+        pick = up;
+    else
+        pick = (lo & 1) ? up : lo;
+    return (uint16_t)(sign | pick); /* pick == 0x7C00 is infinity */
+}
+
+#define REF_OPT_SGD 0
+#define REF_OPT_ADAM 1
+
+static int valid_opt(int opt, const float* m, const float* v, int64_t t)
+{
+    if (opt == REF_OPT_SGD)
+        return 1;
+    return opt == REF_OPT_ADAM && m != NULL && v != NULL && t >= 1;
+}
+
+/* Adam's bias corrections 1 - beta^t, computed in double and rounded once. */
+static float bias_correction(float beta, int64_t t)
+{
+    return (float)(1.0 - pow((double)beta, (double)t));
+}
+
+/* One step on the fp32 master coefficient c of a sub-block with gradient dc
+ * (R15). SGD: c <- c - lr * dc. Adam, in the order of Kingma & Ba's
+ * algorithm: m <- b1 m + (1 - b1) dc; v <- b2 v + (1 - b2) dc^2;
+ * m_hat = m / (1 - b1^t); v_hat = v / (1 - b2^t);
+ * c <- c - lr * m_hat / (sqrt(v_hat) + eps). */
+static void opt_update(int opt, float dc, float lr, float b1, float b2, float eps, float bc1,
+                       float bc2, float* c, float* m, float* v)
+{
+    if (opt == REF_OPT_SGD) {
+        float step = lr * dc;
+        *c = *c - step;
+        return;
+    }
+    float om1 = 1.0f - b1;
+    float om2 = 1.0f - b2;
+    float m1 = b1 * (*m);
+    float m2 = om1 * dc;
+    float mn = m1 + m2;
+    float v1 = b2 * (*v);
+    float g2 = dc * dc;
+    float v2 = om2 * g2;
+    float vn = v1 + v2;
+    float mh = mn / bc1;
+    float vh = vn / bc2;
+    float rt = sqrtf(vh);
+    float den = rt + eps;
+    float num = lr * mh;
+    float step = num / den;
+    *m = mn;
+    *v = vn;
+    *c = *c - step;
+}
+
+/* The forward pass consumes the FP16 coefficient (the pages' parameter type):
+ * the value of the master coefficient rounded to half precision. */
+static float coefficient_used(float c32)
+{
+    return ref_fp16_to_float(ref_float_to_fp16(c32));
+}
+
+/* FOCUS coefficient update from an external gradient g = dL/dW_hat (for a
+ * loss the caller differentiates: the pages' distillation loss, or a layer
+ * output loss): the straight-through gradient of R9 at the coefficient the
+ * forward used, then one optimizer step on the master coefficients.
+ * c (fp32 master), m, v: [rows, cols/sub], updated in place; c_half: fp16
+ * bits of the updated coefficients, nullable. [FOCUS] Metodologia §1 (STE
+ * and gradient descent on the scales), §2 (c as FP16 learnable parameter). */
+int ref_focus_update(const uint16_t* w, const uint16_t* g, float* c, uint16_t* c_half,
+                     float* m, float* v, int64_t rows, int64_t cols, int sub, int opt, float lr,
+                     float b1, float b2, float eps, int64_t t)
+{
+    if (rows <= 0 || cols <= 0 || sub < 1 || sub > 128 || (sub & (sub - 1)) != 0 ||
+        cols % sub != 0 || !valid_opt(opt, m, v, t))
+        return REF_ERR_ARG;
+    float bc1 = opt == REF_OPT_ADAM ? bias_correction(b1, t) : 1.0f;
+    float bc2 = opt == REF_OPT_ADAM ? bias_correction(b2, t) : 1.0f;
+    float p[128];
+    for (int64_t k = 0; k < rows * cols / sub; k++) {
+        for (int j = 0; j < sub; j++) {
+            int64_t e = k * sub + j;
+            p[j] = ref_bf16_to_float(g[e]) * ref_bf16_to_float(w[e]);
+        }
+        float acc = ref_tsum(p, sub);
+        float ck = coefficient_used(c[k]);
+        float cc = ck * ck;
+        float dc = -(acc / cc);
+        opt_update(opt, dc, lr, b1, b2, eps, bc1, bc2, &c[k], m ? &m[k] : NULL,
+                   v ? &v[k] : NULL);
+        if (c_half)
+            c_half[k] = ref_float_to_fp16(c[k]);
+    }
+    return REF_OK;
+}
+
+/* One calibration step on the weight-reconstruction loss L = sum (W_hat - W)^2
+ * (R16): the FOCUS forward at the coefficients used, the loss gradient
+ * g = 2 (W_hat - W) in fp32 (W_hat not rounded to bf16), the straight-through
+ * coefficient gradient dc = -(tsum(g * W) / c^2), one optimizer step.
+ * sse (nullable, fp32 [rows, cols/sub]) receives tsum((W_hat - W)^2) per
+ * sub-block, before the step. [FOCUS] Metodologia §1-§3. */
+int ref_focus_step(const uint16_t* w, int64_t rows, int64_t cols, int fmt, int block, int sub,
+                   const float* global_amax_in, float* global_scale_out, float* c,
+                   uint16_t* c_half, float* m, float* v, float* sse, int opt, float lr, float b1,
+                   float b2, float eps, int64_t t)
+{
+    if (!valid_common(rows, cols, fmt, block, 0))
+        return REF_ERR_ARG;
+    if (sub < 1 || block % sub != 0 || (sub & (sub - 1)) != 0 || !valid_opt(opt, m, v, t))
+        return REF_ERR_ARG;
+    float sg = 1.0f;
+    if (fmt == REF_FMT_NVFP4) {
+        float ga = global_amax_in ? *global_amax_in : ref_global_amax(w, rows, cols, 0);
+        sg = ref_global_scale(ga);
+        if (global_scale_out)
+            *global_scale_out = sg;
+    }
+    float bc1 = opt == REF_OPT_ADAM ? bias_correction(b1, t) : 1.0f;
+    float bc2 = opt == REF_OPT_ADAM ? bias_correction(b2, t) : 1.0f;
+    float* y = (float*)malloc(sizeof(float) * (size_t)cols);
+    float d[128], p[128];
+    int64_t nb = cols / block;
+    for (int64_t i = 0; i < rows; i++) {
+        load_row(w + i * cols, cols, 0, y);
+        for (int64_t b = 0; b < nb; b++) {
+            const float* yb = y + b * block;
+            float amax = 0.0f;
+            for (int j = 0; j < block; j++) {
+                float a = fabsf(yb[j]);
+                if (a > amax)
+                    amax = a;
+            }
+            float Sdq;
+            if (fmt == REF_FMT_MXFP4)
+                Sdq = (float)ldexp(1.0, ref_e8m0_exponent(amax));
+            else
+                (void)nv_candidate(amax, 6.0f, sg, &Sdq);
+            for (int s0 = 0; s0 < block; s0 += sub) {
+                int64_t k = (i * cols + b * block + s0) / sub;
+                float ck = coefficient_used(c[k]);
+                for (int j = 0; j < sub; j++) {
+                    float wj = yb[s0 + j];
+                    float what = 0.0f;
+                    if (Sdq != 0.0f) {
+                        float den = Sdq * ck;
+                        float r = guarded_reciprocal(den);
+                        float u = wj * r;
+                        what = (float)ref_e2m1_value(ref_rne_e2m1(u)) * Sdq;
+                    }
+                    d[j] = what - wj;
+                    float gj = d[j] + d[j];
+                    p[j] = gj * wj;
+                }
+                if (sse) {
+                    float e[128];
+                    for (int j = 0; j < sub; j++)
+                        e[j] = d[j] * d[j];
+                    sse[k] = ref_tsum(e, sub);
+                }
+                float acc = ref_tsum(p, sub);
+                float cc = ck * ck;
+                float dc = -(acc / cc);
+                opt_update(opt, dc, lr, b1, b2, eps, bc1, bc2, &c[k], m ? &m[k] : NULL,
+                           v ? &v[k] : NULL);
+                if (c_half)
+                    c_half[k] = ref_float_to_fp16(c[k]);
+            }
+        }
+    }
+    free(y);
     return REF_OK;
 }
 
