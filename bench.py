@@ -516,6 +516,18 @@ def breakdown(dev, peaks, reps: int = 10):
     secs = timeit([lambda i=i: fp4q.focus_bwd(ws[i], gs[i], cs[i], 8, out=dcs[i])
                    for i in range(nc)])
     add("c4_focus bwd sub8 -> fp32 dc", n, secs, 2 + 2 + 0.25 + 0.5, 1)
+    # FOCUS calibration with Adam: fp32 master c, m and v read and written
+    # (24 B per sub-block) plus the fp16 copy written (2 B), per 8 elements
+    states = [fp4q.focus_state(4096, 4096, 8, "adam", device=dev) for _ in range(nc)]
+    gaw = fp4q.global_amax(w0, 0)
+    gsw = torch.empty(1, device=dev)
+    secs = timeit([lambda i=i: fp4q.focus_step(ws[i], states[i], "nvfp4", 16, 8, global_amax=gaw,
+                                               global_scale=gsw, lr=1e-4) for i in range(nc)])
+    add("c4_focus calibration step nvfp4 B16 sub8 adam (fwd + 2(W_hat-W) + STE grad + update)", n,
+        secs, 2 + 26 / 8, 1)
+    secs = timeit([lambda i=i: fp4q.focus_update(ws[i], gs[i], states[i], 8, lr=1e-4)
+                   for i in range(nc)])
+    add("c4_focus update from gradient sub8 adam", n, secs, 2 + 2 + 26 / 8, 1)
     return rows_out
 
 
@@ -640,7 +652,8 @@ SUITE = ["quant MXFP4 B32 rot0", "quant MXFP4 B32 rot32", "quant MXFP4 B32 rot12
          "quant NVFP4 B4 4-over-6 (+MSE)", "quant NVFP4 B16 brute force (1024 rows, +MSE)",
          "global abs-max rot16", "dequantize NVFP4 B16 -> bf16", "block MSE NVFP4 B16",
          "FOCUS fwd NVFP4 B16 sub8 -> bf16", "FOCUS bwd sub8", "quant NVFP4 B16 4-over-6 (+MSE)",
-         "quant MXFP4 B32 MSE-optimised E8M0 scale", "dequantize MXFP4 B32 + undo 128-wide Hadamard -> bf16"]
+         "quant MXFP4 B32 MSE-optimised E8M0 scale", "dequantize MXFP4 B32 + undo 128-wide Hadamard -> bf16",
+         "FOCUS calibration step NVFP4 B16 sub8 Adam", "FOCUS update from gradient sub8 Adam"]
 
 
 def run_suite(rounds: int = 2):
@@ -664,6 +677,9 @@ def run_suite(rounds: int = 2):
     ga16 = fp4q.global_amax(x, 16)
     gw = fp4q.global_amax(w, 0)
     q16 = fp4q.quantize(x, "nvfp4", 16, "absmax", 0, global_amax=ga)
+    st_step = fp4q.focus_state(R, C, 8, "adam", device=dev)
+    st_upd = fp4q.focus_state(R, C, 8, "adam", device=dev)
+    gsw = torch.empty(1, device=dev)
     torch.cuda.synchronize()
     outs = {}
     for _ in range(rounds):
@@ -683,6 +699,9 @@ def run_suite(rounds: int = 2):
         outs[13] = fp4q.quantize(x, "mxfp4", 32, "brute_force", 0)
         outs[14] = fp4q.dequantize(outs[2].codes, outs[2].scales, None, "mxfp4", 32, torch.bfloat16,
                                    rot=128)
+        outs[15] = fp4q.focus_step(w, st_step, "nvfp4", 16, 8, global_amax=gw, global_scale=gsw,
+                                   lr=1e-4)
+        outs[16] = fp4q.focus_update(w, g, st_upd, 8, lr=1e-4)
         torch.cuda.synchronize()
     print(json.dumps({"suite": SUITE, "rounds": rounds, "shape": [R, C],
                       "device_errors": fp4q._abi.load().fp4q_device_errors()}))

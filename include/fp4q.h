@@ -79,6 +79,11 @@ typedef enum {
 
 typedef enum { FP4Q_OUT_F32 = 0, FP4Q_OUT_BF16 = 1 } fp4q_dtype;
 
+/* Optimizer of the FOCUS coefficient calibration ("FOCUS: ...", Metodologia
+ * §1: the scales are learned by gradient descent through the STE; the page
+ * names no optimizer). FP4Q_OPT_ADAM follows Kingma & Ba's algorithm. */
+typedef enum { FP4Q_OPT_SGD = 0, FP4Q_OPT_ADAM = 1 } fp4q_optimizer;
+
 /*
  * fp4q_quantize -- rotate (optional) -> per-block scale -> E2M1 RNE -> pack,
  * with optional dequantized values and per-block MSE.
@@ -253,6 +258,59 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
  */
 fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t rows,
                            int64_t cols, int sub, float* dc, cudaStream_t stream);
+
+/*
+ * fp4q_focus_update -- one calibration step of the FOCUS coefficients from an
+ * external gradient g = dL/dW_hat (the loss the caller differentiates: the
+ * pages' distillation loss, or a layer-output loss such as
+ * |X (W_hat - W)^T|^2 whose gradient 2 (W_hat - W) X^T X is a plain GEMM).
+ * ("FOCUS: ...", Metodologia §1 STE and gradient descent, §2 c is an FP16
+ * learnable parameter initialised to 1.)
+ * Per sub-block k: c16 = fp16(c[k]) (round to nearest even; the value the
+ * forward pass consumes), dc = -(tree_sum(g * W) / (c16 * c16)) as in
+ * fp4q_focus_bwd, then the optimizer step on the fp32 master c[k]:
+ *   SGD   c <- c - lr * dc
+ *   Adam  m <- b1 m + (1 - b1) dc;  v <- b2 v + (1 - b2) (dc * dc);
+ *         c <- c - (lr * (m / bc1)) / (sqrt(v / bc2) + eps),
+ *         bc1 = 1 - b1^t and bc2 = 1 - b2^t computed in double on the host
+ *         and rounded to fp32; every other step one fp32 operation, RNE.
+ * w, g     bf16 [rows, cols].
+ * c        fp32 [rows, cols/sub], read and overwritten (master coefficients).
+ * c_half   nullable fp16 [rows, cols/sub]: fp16(c) after the step, ready for
+ *          fp4q_focus_fwd.
+ * m, v     fp32 [rows, cols/sub], Adam's moments, read and overwritten
+ *          (start at zero); ignored (may be NULL) for SGD.
+ * t        Adam's step number, >= 1. b1, b2, eps are ignored for SGD.
+ * An unknown opt, or Adam with t < 1, returns FP4Q_ERR_UNSUPPORTED; Adam with
+ * m or v NULL returns FP4Q_ERR_NULL. c, c_half, m, v must not overlap w or g.
+ * Nothing keeps c positive: a coefficient driven to zero or below gives
+ * unspecified codes in the next forward pass.
+ */
+fp4q_status fp4q_focus_update(const void* w, const void* g, float* c, void* c_half, float* m,
+                              float* v, int64_t rows, int64_t cols, int sub, fp4q_optimizer opt,
+                              float lr, float b1, float b2, float eps, int64_t t,
+                              cudaStream_t stream);
+
+/*
+ * fp4q_focus_step -- one fused calibration step on the weight-reconstruction
+ * loss L = sum (W_hat - W)^2: the FOCUS forward at c16 = fp16(c) (exactly
+ * fp4q_focus_fwd's W_hat, kept in fp32), g = 2 (W_hat - W) in fp32, the
+ * straight-through gradient dc = -(tree_sum(g * W) / (c16 * c16)) and the
+ * optimizer step of fp4q_focus_update, in one pass over W
+ * ("FOCUS: ...", Metodologia §1-§3). With c == 1 every element already lands
+ * on its nearest point of the S_dq grid, so this loss is at its minimum there;
+ * the step is the loop's fused building block, and losses that couple
+ * elements go through fp4q_focus_update.
+ * w, fmt, block, sub, global_amax_in, global_scale_out: as fp4q_focus_fwd.
+ * c, c_half, m, v, opt, lr, b1, b2, eps, t: as fp4q_focus_update.
+ * sse      nullable fp32 [rows, cols/sub]: tree_sum((W_hat - W)^2) per
+ *          sub-block, at the coefficients before the step.
+ */
+fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                            int sub, const float* global_amax_in, float* global_scale_out,
+                            float* c, void* c_half, float* m, float* v, float* sse,
+                            fp4q_optimizer opt, float lr, float b1, float b2, float eps,
+                            int64_t t, cudaStream_t stream);
 
 /*
  * fp4q_global_amax -- abs-max of the (rotated) tensor into *amax_out (device

@@ -160,6 +160,75 @@ def focus_bwd(w: torch.Tensor, g: torch.Tensor, c: torch.Tensor, sub: int = 8,
     return out
 
 
+OPTIMIZERS = {"sgd": 0, "adam": 1}
+
+
+@dataclass
+class FocusState:
+    """FOCUS calibration state of one weight: fp32 master coefficients, their
+    fp16 copy (what focus_fwd consumes), Adam's moments and step count."""
+    c: torch.Tensor                # float32 [rows, cols/sub]
+    c_half: torch.Tensor           # float16 [rows, cols/sub]
+    m: Optional[torch.Tensor]      # float32 [rows, cols/sub] (Adam) or None
+    v: Optional[torch.Tensor]
+    opt: str = "adam"
+    t: int = 0
+
+
+def focus_state(rows: int, cols: int, sub: int = 8, opt: str = "adam",
+                device=None) -> FocusState:
+    """Coefficients initialised to 1 (FOCUS Metodologia §2), moments to 0."""
+    n = (rows, cols // sub)
+    adam = opt == "adam"
+    return FocusState(
+        c=torch.ones(n, dtype=torch.float32, device=device),
+        c_half=torch.ones(n, dtype=torch.float16, device=device),
+        m=torch.zeros(n, dtype=torch.float32, device=device) if adam else None,
+        v=torch.zeros(n, dtype=torch.float32, device=device) if adam else None,
+        opt=opt)
+
+
+def _opt_args(state: FocusState, lr, beta1, beta2, eps):
+    return (OPTIMIZERS[state.opt], float(lr), float(beta1), float(beta2), float(eps), state.t + 1)
+
+
+def focus_update(w: torch.Tensor, g: torch.Tensor, state: FocusState, sub: int = 8,
+                 lr: float = 1e-3, beta1: float = 0.9, beta2: float = 0.999,
+                 eps: float = 1e-8) -> FocusState:
+    """One optimizer step of the coefficients from g = dL/dW_hat (bf16), in place."""
+    _check(w, torch.bfloat16, "w")
+    _check(g, torch.bfloat16, "g")
+    _check(state.c, torch.float32, "c")
+    _check(state.c_half, torch.float16, "c_half")
+    rows, cols = w.shape
+    _abi.call("fp4q_focus_update", w.data_ptr(), g.data_ptr(), state.c.data_ptr(),
+              state.c_half.data_ptr(), _ptr(state.m), _ptr(state.v), rows, cols, sub,
+              *_opt_args(state, lr, beta1, beta2, eps), _stream())
+    state.t += 1
+    return state
+
+
+def focus_step(w: torch.Tensor, state: FocusState, fmt="nvfp4", block: int = 16, sub: int = 8,
+               global_amax: Optional[torch.Tensor] = None,
+               global_scale: Optional[torch.Tensor] = None, want_sse: bool = False,
+               lr: float = 1e-3, beta1: float = 0.9, beta2: float = 0.999,
+               eps: float = 1e-8) -> Optional[torch.Tensor]:
+    """One fused step on sum (W_hat - W)^2, in place; returns the per-sub-block
+    SSE before the step (float32 [rows, cols/sub]) when want_sse."""
+    _check(w, torch.bfloat16, "w")
+    _check(state.c, torch.float32, "c")
+    rows, cols = w.shape
+    f = _fmt(fmt)
+    if f == 0 and global_scale is None:
+        global_scale = torch.empty(1, dtype=torch.float32, device=w.device)
+    sse = torch.empty(rows, cols // sub, dtype=torch.float32, device=w.device) if want_sse else None
+    _abi.call("fp4q_focus_step", w.data_ptr(), rows, cols, f, block, sub, _ptr(global_amax),
+              _ptr(global_scale), state.c.data_ptr(), _ptr(state.c_half), _ptr(state.m),
+              _ptr(state.v), _ptr(sse), *_opt_args(state, lr, beta1, beta2, eps), _stream())
+    state.t += 1
+    return sse
+
+
 def mma_scale_bytes(rows: int, K: int, fmt="nvfp4") -> int:
     n = _abi.load().fp4q_mma_scale_bytes(rows, K, _fmt(fmt))
     if n == 0:

@@ -17,6 +17,7 @@ LIB_PATH = os.path.join(HERE, "libfp4q.so")
 _p = C.c_void_p
 _i64 = C.c_int64
 _i32 = C.c_int
+_f32 = C.c_float
 SIGNATURES = {
     "fp4q_quantize": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p,
                              _i32, _p]),
@@ -26,6 +27,10 @@ SIGNATURES = {
     "fp4q_focus_fwd": (_i32, [_p, _p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _i32, _p, _p,
                               _p]),
     "fp4q_focus_bwd": (_i32, [_p, _p, _p, _i64, _i64, _i32, _p, _p]),
+    "fp4q_focus_update": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i32, _i32, _f32, _f32,
+                                 _f32, _f32, _i64, _p]),
+    "fp4q_focus_step": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p,
+                               _i32, _f32, _f32, _f32, _f32, _i64, _p]),
     "fp4q_global_amax": (_i32, [_p, _i64, _i64, _i32, _p, _p]),
     "fp4q_e2m1_encode": (_i32, [_p, _i64, _p, _p]),
     "fp4q_e4m3_encode": (_i32, [_p, _i64, _p, _p]),

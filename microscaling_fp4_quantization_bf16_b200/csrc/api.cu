@@ -2,6 +2,7 @@
 //
 // Host side only: validate every argument, then enqueue kernels on the
 // caller's stream. Nothing is allocated and nothing is synchronised.
+#include <cmath>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -9,6 +10,7 @@
 #include <cuda.h>
 
 #include "fp4q.h"
+
 #include "internal.h"
 
 using namespace fp4q;
@@ -484,6 +486,136 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
     a.n = n;
     a.dc = dc;
     return cuda_status(launch_focus_bwd(sub, a, stream));
+}
+
+namespace {
+
+// Optimizer constants on the host: 1 - b in fp32, Adam's bias corrections
+// 1 - b^t in double, rounded once to fp32.
+OptConsts opt_consts(fp4q_optimizer opt, float lr, float b1, float b2, float eps, int64_t t)
+{
+    OptConsts o;
+    o.lr = lr;
+    o.b1 = b1;
+    o.b2 = b2;
+    o.eps = eps;
+    o.om1 = 1.0f - b1;
+    o.om2 = 1.0f - b2;
+    o.bc1 = 1.0f;
+    o.bc2 = 1.0f;
+    if (opt == FP4Q_OPT_ADAM) {
+        o.bc1 = (float)(1.0 - std::pow((double)b1, (double)t));
+        o.bc2 = (float)(1.0 - std::pow((double)b2, (double)t));
+    }
+    return o;
+}
+
+fp4q_status check_opt(fp4q_optimizer opt, int64_t t, const float* m, const float* v)
+{
+    if (opt != FP4Q_OPT_SGD && opt != FP4Q_OPT_ADAM)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (opt == FP4Q_OPT_ADAM && t < 1)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (opt == FP4Q_OPT_ADAM && (m == nullptr || v == nullptr))
+        return FP4Q_ERR_NULL;
+    return FP4Q_OK;
+}
+
+}  // namespace
+
+fp4q_status fp4q_focus_update(const void* w, const void* g, float* c, void* c_half, float* m,
+                              float* v, int64_t rows, int64_t cols, int sub, fp4q_optimizer opt,
+                              float lr, float b1, float b2, float eps, int64_t t,
+                              cudaStream_t stream)
+{
+    if (!valid_sub(sub))
+        return FP4Q_ERR_UNSUPPORTED;
+    if (rows < 0 || cols < 0 || cols % sub != 0 || (cols > 0 && rows > kMaxElems / cols))
+        return FP4Q_ERR_SHAPE;
+    fp4q_status st = check_opt(opt, t, m, v);
+    if (st != FP4Q_OK)
+        return st;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    if (w == nullptr || g == nullptr || c == nullptr)
+        return FP4Q_ERR_NULL;
+    if (!aligned16(w) || !aligned16(g) || !aligned16(c) || !aligned16(c_half) || !aligned16(m) ||
+        !aligned16(v))
+        return FP4Q_ERR_ALIGN;
+    const bool adam = opt == FP4Q_OPT_ADAM;
+    FocusUpdateArgs a;
+    a.w = static_cast<const uint16_t*>(w);
+    a.g = static_cast<const uint16_t*>(g);
+    a.c = c;
+    a.c_half = static_cast<uint16_t*>(c_half);
+    a.m = adam ? m : nullptr;
+    a.v = adam ? v : nullptr;
+    a.n = n;
+    a.o = opt_consts(opt, lr, b1, b2, eps, t);
+    return cuda_status(launch_focus_update(sub, adam, a, stream));
+}
+
+fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                            int sub, const float* global_amax_in, float* global_scale_out,
+                            float* c, void* c_half, float* m, float* v, float* sse,
+                            fp4q_optimizer opt, float lr, float b1, float b2, float eps,
+                            int64_t t, cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, 0);
+    if (st != FP4Q_OK)
+        return st;
+    if (!valid_sub(sub) || sub > block)
+        return FP4Q_ERR_UNSUPPORTED;
+    st = check_opt(opt, t, m, v);
+    if (st != FP4Q_OK)
+        return st;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t n = rows * cols;
+    if (nv && global_scale_out == nullptr)
+        return FP4Q_ERR_NULL;
+    if (n > 0 && (w == nullptr || c == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(w) || !aligned16(c) || !aligned16(c_half) || !aligned16(m) || !aligned16(v) ||
+        !aligned16(sse))
+        return FP4Q_ERR_ALIGN;
+    if (nv && (!aligned4(global_scale_out) || !aligned4(global_amax_in)))
+        return FP4Q_ERR_ALIGN;
+    if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
+        return FP4Q_ERR_ALIAS;
+    if (n == 0)
+        return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
+
+    const bool adam = opt == FP4Q_OPT_ADAM;
+    FocusStepArgs a;
+    a.w = static_cast<const uint16_t*>(w);
+    a.n = n;
+    a.amax = nullptr;
+    a.sg_out = nullptr;
+    a.c = c;
+    a.c_half = static_cast<uint16_t*>(c_half);
+    a.m = adam ? m : nullptr;
+    a.v = adam ? v : nullptr;
+    a.sse = sse;
+    a.keep = 0xFFFFFFFFu;
+    a.o = opt_consts(opt, lr, b1, b2, eps, t);
+    if (nv) {
+        if (global_amax_in != nullptr) {
+            a.amax = global_amax_in;
+            a.sg_out = global_scale_out;
+        } else {
+            st = accumulate_amax(w, n, 0, global_scale_out, stream);
+            if (st != FP4Q_OK)
+                return st;
+            a.amax = global_scale_out;  // holds the abs-max until finalised below
+        }
+    }
+    st = cuda_status(launch_focus_step(nv ? 0 : 1, block, sub, adam, a, stream));
+    if (st != FP4Q_OK)
+        return st;
+    if (nv && global_amax_in == nullptr)
+        st = cuda_status(launch_finalize_sg(global_scale_out, stream));
+    return st;
 }
 
 fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax_out,

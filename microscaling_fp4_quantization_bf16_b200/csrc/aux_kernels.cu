@@ -172,30 +172,6 @@ __device__ __forceinline__ void scales_of(const uint32_t (&sc)[NB], float sg, fl
         S[b] = MX ? e8m0_dec(sc[b]) : __fmul_rn(e4m3_dec(sc[b]), sg);
 }
 
-// Writes NK floats of segment s (NK = 32 / granularity) to p + s * NK.
-template <int NK>
-__device__ __forceinline__ void store_seg_floats(float* p, int64_t s, int nvalid, int gran,
-                                                 const float (&v)[NK])
-{
-    float* o = p + s * NK;
-    if (nvalid == SEG) {
-        if constexpr (NK >= 4) {
-#pragma unroll
-            for (int k = 0; k < NK / 4; ++k)
-                reinterpret_cast<float4*>(o)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
-        } else if constexpr (NK == 2) {
-            *reinterpret_cast<float2*>(o) = make_float2(v[0], v[1]);
-        } else {
-            *o = v[0];
-        }
-    } else {
-#pragma unroll
-        for (int k = 0; k < NK; ++k)
-            if (k * gran < nvalid)
-                o[k] = v[k];
-    }
-}
-
 // ------------------------------------------------------------ dequantize
 
 // One thread per EPT consecutive elements (EPT = 8 for bf16 output, 4 for
@@ -493,30 +469,10 @@ __global__ void __launch_bounds__(STHREADS) focus_fwd_kernel(FocusFwdArgs a)
     load_seg_bf16(a.w, a.n, s, y);
     load_coeffs<NK>(a.c, s, nvalid, SUB, ck);
 
-    float amax[NB], S[NB];
+    float S[NB];
     uint32_t sc[NB];
     bool zb[NB];
-    block_amax<B>(y, amax);
-    if constexpr (MX) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int e = e8m0_exp(amax[b]);
-            sc[b] = (uint32_t)(e + 127);
-            S[b] = pow2f(e);
-        }
-    } else {
-        const NvConsts kc = nv_consts(sg);
-        float qd[NB], qr[NB];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            qd[b] = kc.den6;
-            qr[b] = kc.rden6;
-        }
-        e4m3_quotient_codes<NB>(amax, qd, qr, kc.fast, sc);
-#pragma unroll
-        for (int b = 0; b < NB; ++b)
-            S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
-    }
+    focus_block_scales<B, MX>(y, sg, S, sc);
 #pragma unroll
     for (int b = 0; b < NB; ++b)
         zb[b] = (S[b] == 0.0f);

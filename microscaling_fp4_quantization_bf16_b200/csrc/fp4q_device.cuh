@@ -766,7 +766,63 @@ __device__ __forceinline__ float saturation_lb(float a, float r, float S)
     return __fmul_rn(d, d);
 }
 
+// The FOCUS dequantization scale S_dq of each block of a segment: the
+// format's abs-max scale (E8M0 2^(floor(log2 amax) - 2) for MXFP4; E4M3 code
+// RNE(amax / (6 s_g)) times s_g for NVFP4) and its scale byte.
+template <int B, bool MX>
+__device__ __forceinline__ void focus_block_scales(const float (&y)[SEG], float sg, float (&S)[SEG / B],
+                                                   uint32_t (&sc)[SEG / B])
+{
+    constexpr int NB = SEG / B;
+    float amax[NB];
+    block_amax<B>(y, amax);
+    if constexpr (MX) {
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            const int e = e8m0_exp(amax[b]);
+            sc[b] = (uint32_t)(e + 127);
+            S[b] = pow2f(e);
+        }
+    } else {
+        const NvConsts kc = nv_consts(sg);
+        float qd[NB], qr[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b) {
+            qd[b] = kc.den6;
+            qr[b] = kc.rden6;
+        }
+        e4m3_quotient_codes<NB>(amax, qd, qr, kc.fast, sc);
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            S[b] = __fmul_rn(e4m3_dec(sc[b]), sg);
+    }
+}
+
 // ------------------------------------------------------------------ stores
+
+// Writes NK floats of segment s (NK = 32 / granularity) to p + s * NK.
+template <int NK>
+__device__ __forceinline__ void store_seg_floats(float* p, int64_t s, int nvalid, int gran,
+                                                 const float (&v)[NK])
+{
+    float* o = p + s * NK;
+    if (nvalid == SEG) {
+        if constexpr (NK >= 4) {
+#pragma unroll
+            for (int k = 0; k < NK / 4; ++k)
+                reinterpret_cast<float4*>(o)[k] = make_float4(v[4 * k], v[4 * k + 1], v[4 * k + 2], v[4 * k + 3]);
+        } else if constexpr (NK == 2) {
+            *reinterpret_cast<float2*>(o) = make_float2(v[0], v[1]);
+        } else {
+            *o = v[0];
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < NK; ++k)
+            if (k * gran < nvalid)
+                o[k] = v[k];
+    }
+}
 
 // NB = SEG / B bytes (one per block) at p (NB-byte aligned).
 template <int NB>

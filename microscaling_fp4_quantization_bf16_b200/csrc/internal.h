@@ -90,6 +90,37 @@ struct FocusBwdArgs {
     float* dc;
 };
 
+// Optimizer constants of one FOCUS calibration step; om1 = 1 - b1 and
+// om2 = 1 - b2 in fp32, bc1 / bc2 Adam's bias corrections (1 for SGD).
+struct OptConsts {
+    float lr, b1, b2, om1, om2, bc1, bc2, eps;
+};
+
+struct FocusUpdateArgs {
+    const uint16_t* w;      // bf16 [n]
+    const uint16_t* g;      // bf16 [n]
+    float* c;               // fp32 [n / sub], in place
+    uint16_t* c_half;       // fp16 [n / sub], optional
+    float* m;               // Adam moments [n / sub] (Adam only)
+    float* v;
+    int64_t n;
+    OptConsts o;
+};
+
+struct FocusStepArgs {
+    const uint16_t* w;      // bf16 [n]
+    int64_t n;
+    const float* amax;      // NVFP4 tensor abs-max (device)
+    float* sg_out;
+    float* c;
+    uint16_t* c_half;
+    float* m;
+    float* v;
+    float* sse;             // fp32 [n / sub], optional
+    uint32_t keep;          // 0xFFFFFFFF, passed at run time (see encode_seg)
+    OptConsts o;
+};
+
 // Each launcher returns cudaErrorInvalidValue for a combination it does not
 // provide (the ABI layer validates before calling), else the launch status.
 cudaError_t launch_quant_b4(int strat, int rot, const QuantArgs& a, cudaStream_t st);
@@ -118,6 +149,9 @@ cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a,
 cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st);
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);
+cudaError_t launch_focus_update(int sub, bool adam, const FocusUpdateArgs& a, cudaStream_t st);
+cudaError_t launch_focus_step(int mx, int block, int sub, bool adam, const FocusStepArgs& a,
+                              cudaStream_t st);
 // W4A4 FP4 GEMM (gemm_*.cu): scale layout for the block-scaled MMA and the
 // four GEMM configurations (NVFP4 / MXFP4 x fp32 / bf16 output).
 size_t mma_scale_bytes(int64_t rows, int64_t K, int sfv);

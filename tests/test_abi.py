@@ -132,6 +132,33 @@ def test_other_entry_points_validation(lib):
     assert L.fp4q_focus_bwd(A, A, A, 4, 64, 6, A, None) == UNSUP
     assert L.fp4q_focus_bwd(A, None, A, 4, 64, 8, A, None) == NULL
     assert L.fp4q_focus_bwd(A, A, A, 4, 64, 8, MIS, None) == ALIGN
+    # focus calibration: coefficient update from a gradient, fused step
+    fu = lambda **k: L.fp4q_focus_update(k.get("w", A), k.get("g", A), k.get("c", A),
+                                         k.get("ch"), k.get("m", A2), k.get("v", A3), 4,
+                                         k.get("cols", 64), k.get("sub", 8), k.get("opt", 1),
+                                         1e-3, 0.9, 0.999, 1e-8, k.get("t", 1), None)
+    assert fu(sub=6) == UNSUP
+    assert fu(cols=60) == SHAPE
+    assert fu(opt=2) == UNSUP
+    assert fu(t=0) == UNSUP          # Adam counts steps from 1
+    assert fu(m=None) == NULL        # Adam needs its moments
+    assert fu(g=None) == NULL
+    assert fu(ch=MIS) == ALIGN
+    assert fu(v=MIS) == ALIGN
+    fs = lambda **k: L.fp4q_focus_step(k.get("w", A), 4, k.get("cols", 64), k.get("fmt", NV),
+                                       k.get("block", 16), k.get("sub", 8), k.get("gin"),
+                                       k.get("gout", A3), k.get("c", A), None, k.get("m", A2),
+                                       k.get("v", A2 + 4096), k.get("sse"), k.get("opt", 1),
+                                       1e-3, 0.9, 0.999, 1e-8, k.get("t", 1), None)
+    assert fs(sub=32) == UNSUP       # sub > block
+    assert fs(fmt=MX, block=16) == UNSUP
+    assert fs(cols=40) == SHAPE
+    assert fs(opt=0, t=0, m=None, v=None, c=None) == NULL   # SGD ignores t, m, v; c required
+    assert fs(t=-3) == UNSUP
+    assert fs(v=None) == NULL
+    assert fs(gout=None) == NULL     # NVFP4 writes s_g
+    assert fs(sse=MIS) == ALIGN
+    assert fs(gin=A3, gout=A3) == ALIAS
     # global amax, primitives
     assert L.fp4q_global_amax(A, 4, 64, 24, A, None) == UNSUP
     assert L.fp4q_global_amax(A, 4, 48, 32, A, None) == SHAPE
