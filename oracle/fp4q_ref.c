@@ -72,8 +72,9 @@
  *      The learnable state is an fp32 master copy of c; the forward uses its
  *      fp16 rounding (the pages' FP16 parameter) and the gradient of R9 is
  *      taken at that fp16 value. Optimizers: plain SGD, and Adam in the
- *      order of Kingma & Ba's algorithm, with the bias corrections 1 - b^t
- *      computed in double and rounded once to fp32.
+ *      efficient ordering Kingma & Ba give beside their algorithm: the step
+ *      size alpha_t = lr sqrt(1 - b2^t) / (1 - b1^t) is computed in double
+ *      and rounded once to fp32, and eps is added to sqrt(v).
  *  R16 The fused calibration step minimises the weight-reconstruction loss
  *      sum (W_hat - W)^2 with g = 2 (W_hat - W) in fp32. (At c == 1 every
  *      element already lands on its nearest point of the S_dq grid, so this
@@ -870,19 +871,23 @@ static int valid_opt(int opt, const float* m, const float* v, int64_t t)
     return opt == REF_OPT_ADAM && m != NULL && v != NULL && t >= 1;
 }
 
-/* Adam's bias corrections 1 - beta^t, computed in double and rounded once. */
-static float bias_correction(float beta, int64_t t)
+/* Adam's step size for step t in Kingma & Ba's efficient ordering:
+ * alpha_t = lr * sqrt(1 - b2^t) / (1 - b1^t), computed in double and rounded
+ * once to fp32. */
+static float adam_step_size(float lr, float b1, float b2, int64_t t)
 {
-    return (float)(1.0 - pow((double)beta, (double)t));
+    double bc1 = 1.0 - pow((double)b1, (double)t);
+    double bc2 = 1.0 - pow((double)b2, (double)t);
+    return (float)((double)lr * sqrt(bc2) / bc1);
 }
 
 /* One step on the fp32 master coefficient c of a sub-block with gradient dc
- * (R15). SGD: c <- c - lr * dc. Adam, in the order of Kingma & Ba's
- * algorithm: m <- b1 m + (1 - b1) dc; v <- b2 v + (1 - b2) dc^2;
- * m_hat = m / (1 - b1^t); v_hat = v / (1 - b2^t);
- * c <- c - lr * m_hat / (sqrt(v_hat) + eps). */
-static void opt_update(int opt, float dc, float lr, float b1, float b2, float eps, float bc1,
-                       float bc2, float* c, float* m, float* v)
+ * (R15). SGD: c <- c - lr * dc. Adam, in the efficient ordering that Kingma &
+ * Ba give beside their algorithm (the bias corrections folded into the step
+ * size): m <- b1 m + (1 - b1) dc; v <- b2 v + (1 - b2) dc^2;
+ * c <- c - alpha_t * (m / (sqrt(v) + eps)). */
+static void opt_update(int opt, float dc, float lr, float b1, float b2, float eps, float alpha,
+                       float* c, float* m, float* v)
 {
     if (opt == REF_OPT_SGD) {
         float step = lr * dc;
@@ -898,12 +903,10 @@ static void opt_update(int opt, float dc, float lr, float b1, float b2, float ep
     float g2 = dc * dc;
     float v2 = om2 * g2;
     float vn = v1 + v2;
-    float mh = mn / bc1;
-    float vh = vn / bc2;
-    float rt = sqrtf(vh);
+    float rt = sqrtf(vn);
     float den = rt + eps;
-    float num = lr * mh;
-    float step = num / den;
+    float ratio = mn / den;
+    float step = alpha * ratio;
     *m = mn;
     *v = vn;
     *c = *c - step;
@@ -930,8 +933,7 @@ int ref_focus_update(const uint16_t* w, const uint16_t* g, float* c, uint16_t* c
     if (rows <= 0 || cols <= 0 || sub < 1 || sub > 128 || (sub & (sub - 1)) != 0 ||
         cols % sub != 0 || !valid_opt(opt, m, v, t))
         return REF_ERR_ARG;
-    float bc1 = opt == REF_OPT_ADAM ? bias_correction(b1, t) : 1.0f;
-    float bc2 = opt == REF_OPT_ADAM ? bias_correction(b2, t) : 1.0f;
+    float alpha = opt == REF_OPT_ADAM ? adam_step_size(lr, b1, b2, t) : lr;
     float p[128];
     for (int64_t k = 0; k < rows * cols / sub; k++) {
         for (int j = 0; j < sub; j++) {
@@ -942,7 +944,7 @@ int ref_focus_update(const uint16_t* w, const uint16_t* g, float* c, uint16_t* c
         float ck = coefficient_used(c[k]);
         float cc = ck * ck;
         float dc = -(acc / cc);
-        opt_update(opt, dc, lr, b1, b2, eps, bc1, bc2, &c[k], m ? &m[k] : NULL,
+        opt_update(opt, dc, lr, b1, b2, eps, alpha, &c[k], m ? &m[k] : NULL,
                    v ? &v[k] : NULL);
         if (c_half)
             c_half[k] = ref_float_to_fp16(c[k]);
@@ -972,8 +974,7 @@ int ref_focus_step(const uint16_t* w, int64_t rows, int64_t cols, int fmt, int b
         if (global_scale_out)
             *global_scale_out = sg;
     }
-    float bc1 = opt == REF_OPT_ADAM ? bias_correction(b1, t) : 1.0f;
-    float bc2 = opt == REF_OPT_ADAM ? bias_correction(b2, t) : 1.0f;
+    float alpha = opt == REF_OPT_ADAM ? adam_step_size(lr, b1, b2, t) : lr;
     float* y = (float*)malloc(sizeof(float) * (size_t)cols);
     float d[128], p[128];
     int64_t nb = cols / block;
@@ -1017,7 +1018,7 @@ int ref_focus_step(const uint16_t* w, int64_t rows, int64_t cols, int fmt, int b
                 float acc = ref_tsum(p, sub);
                 float cc = ck * ck;
                 float dc = -(acc / cc);
-                opt_update(opt, dc, lr, b1, b2, eps, bc1, bc2, &c[k], m ? &m[k] : NULL,
+                opt_update(opt, dc, lr, b1, b2, eps, alpha, &c[k], m ? &m[k] : NULL,
                            v ? &v[k] : NULL);
                 if (c_half)
                     c_half[k] = ref_float_to_fp16(c[k]);
