@@ -271,9 +271,11 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
  * fp4q_focus_bwd, then the optimizer step on the fp32 master c[k]:
  *   SGD   c <- c - lr * dc
  *   Adam  m <- b1 m + (1 - b1) dc;  v <- b2 v + (1 - b2) (dc * dc);
- *         c <- c - (lr * (m / bc1)) / (sqrt(v / bc2) + eps),
- *         bc1 = 1 - b1^t and bc2 = 1 - b2^t computed in double on the host
- *         and rounded to fp32; every other step one fp32 operation, RNE.
+ *         c <- c - alpha_t * (m / (sqrt(v) + eps)), the efficient ordering
+ *         Kingma & Ba give beside their algorithm: the bias corrections sit
+ *         in alpha_t = lr sqrt(1 - b2^t) / (1 - b1^t), computed in double on
+ *         the host and rounded to fp32; every other step is one fp32
+ *         operation, RNE.
  * w, g     bf16 [rows, cols].
  * c        fp32 [rows, cols/sub], read and overwritten (master coefficients).
  * c_half   nullable fp16 [rows, cols/sub]: fp16(c) after the step, ready for

@@ -490,8 +490,9 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
 
 namespace {
 
-// Optimizer constants on the host: 1 - b in fp32, Adam's bias corrections
-// 1 - b^t in double, rounded once to fp32.
+// Optimizer constants on the host: 1 - b in fp32; Adam's step size for step t
+// in Kingma & Ba's efficient ordering, lr * sqrt(1 - b2^t) / (1 - b1^t),
+// computed in double and rounded once to fp32.
 OptConsts opt_consts(fp4q_optimizer opt, float lr, float b1, float b2, float eps, int64_t t)
 {
     OptConsts o;
@@ -501,11 +502,11 @@ OptConsts opt_consts(fp4q_optimizer opt, float lr, float b1, float b2, float eps
     o.eps = eps;
     o.om1 = 1.0f - b1;
     o.om2 = 1.0f - b2;
-    o.bc1 = 1.0f;
-    o.bc2 = 1.0f;
+    o.alpha = lr;
     if (opt == FP4Q_OPT_ADAM) {
-        o.bc1 = (float)(1.0 - std::pow((double)b1, (double)t));
-        o.bc2 = (float)(1.0 - std::pow((double)b2, (double)t));
+        const double bc1 = 1.0 - std::pow((double)b1, (double)t);
+        const double bc2 = 1.0 - std::pow((double)b2, (double)t);
+        o.alpha = (float)((double)lr * std::sqrt(bc2) / bc1);
     }
     return o;
 }

@@ -74,6 +74,11 @@ __device__ __forceinline__ void store_seg_halves(uint16_t* p, int64_t s, int nva
     }
 }
 
+__device__ __forceinline__ void prefetch_l2(const float* p)
+{
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
 // fp32 -> fp16 (round to nearest even) -> fp32: the coefficient the forward uses.
 __device__ __forceinline__ float coef_used(float c)
 {
@@ -82,7 +87,8 @@ __device__ __forceinline__ float coef_used(float c)
 
 // One optimizer step on a master coefficient; every operation is one IEEE
 // fp32 operation with round-to-nearest-even (explicit intrinsics: nothing is
-// contracted). Adam in the order of Kingma & Ba's algorithm.
+// contracted). Adam in the efficient ordering Kingma & Ba give beside their
+// algorithm: the bias corrections are folded into the step size o.alpha.
 template <bool ADAM>
 __device__ __forceinline__ void opt_step(float dc, const OptConsts& o, float& c, float& m, float& v)
 {
@@ -91,26 +97,24 @@ __device__ __forceinline__ void opt_step(float dc, const OptConsts& o, float& c,
     } else {
         m = __fadd_rn(__fmul_rn(o.b1, m), __fmul_rn(o.om1, dc));
         v = __fadd_rn(__fmul_rn(o.b2, v), __fmul_rn(o.om2, __fmul_rn(dc, dc)));
-        const float mh = __fdiv_rn(m, o.bc1);
-        const float vh = __fdiv_rn(v, o.bc2);
-        const float den = __fadd_rn(__fsqrt_rn(vh), o.eps);
-        c = __fsub_rn(c, __fdiv_rn(__fmul_rn(o.lr, mh), den));
+        const float den = __fadd_rn(__fsqrt_rn(v), o.eps);
+        c = __fsub_rn(c, __fmul_rn(o.alpha, __fdiv_rn(m, den)));
     }
 }
 
-// dc of every sub-block of the segment from the products p = g * W, then the
-// optimizer step, then the stores of c (and m, v, fp16(c)).
-template <int SUB, bool ADAM>
-__device__ __forceinline__ void update_segment(float (&p)[SEG], const float (&ck)[SEG / SUB], float (&c)[SEG / SUB],
-                                               float (&m)[SEG / SUB], float (&v)[SEG / SUB], const OptConsts& o,
-                                               float* cp, uint16_t* chp, float* mp, float* vp, int64_t s, int nvalid)
+// dc of every sub-block of the segment from its tree sum of g * W (acc[k]),
+// then the optimizer step, then the stores of c (and m, v, fp16(c)).
+template <int SUB, bool ADAM, int NA>
+__device__ __forceinline__ void update_sums(const float (&acc)[NA], const float (&ck)[SEG / SUB], float (&c)[SEG / SUB],
+                                            float (&m)[SEG / SUB], float (&v)[SEG / SUB], const OptConsts& o,
+                                            float* cp, uint16_t* chp, float* mp, float* vp, int64_t s, int nvalid)
 {
     constexpr int NK = SEG / SUB;
+    static_assert(NA >= NK, "one sum per sub-block");
     uint32_t h[NK];
 #pragma unroll
     for (int k = 0; k < NK; ++k) {
-        const float acc = tree_sum<SUB>(p + k * SUB);
-        const float dc = -__fdiv_rn(acc, __fmul_rn(ck[k], ck[k]));
+        const float dc = -__fdiv_rn(acc[k], __fmul_rn(ck[k], ck[k]));
         opt_step<ADAM>(dc, o, c[k], m[k], v[k]);
         h[k] = __half_as_ushort(__float2half_rn(c[k]));
     }
@@ -147,14 +151,25 @@ __global__ void __launch_bounds__(OTHREADS) focus_update_kernel(FocusUpdateArgs 
 #pragma unroll
     for (int i = 0; i < SEG; ++i)
         w[i] = __fmul_rn(g[i], w[i]);
-    update_segment<SUB, ADAM>(w, ck, c, m, v, a.o, a.c, a.c_half, a.m, a.v, s, nvalid);
+    float acc[NK];
+#pragma unroll
+    for (int k = 0; k < NK; ++k)
+        acc[k] = tree_sum<SUB>(w + k * SUB);
+    update_sums<SUB, ADAM>(acc, ck, c, m, v, a.o, a.c, a.c_half, a.m, a.v, s, nvalid);
 }
+
+// Resident CTAs the step kernel is compiled for. With sub-blocks of 8 or more
+// it is held to 64 registers (8 CTAs, 32 warps per SM; a few bytes spill):
+// measured 8% faster than its unconstrained 80 registers on the 4096 x 4096
+// NVFP4 B16 sub-8 step. Smaller sub-blocks keep more per-thread state.
+template <int SUB>
+constexpr int step_min_blocks() { return SUB >= 8 ? 8 : (SUB == 4 ? 6 : 4); }
 
 // Fused step on L = sum (W_hat - W)^2: the forward is fp4q_focus_fwd's
 // (S_dq = the format's abs-max block scale, u = W * (1 / (S_dq * c16)),
 // E2M1 RNE, W_hat = val * S_dq), then d = W_hat - W, g = d + d, p = g * W.
 template <int B, int SUB, bool MX, bool ADAM>
-__global__ void __launch_bounds__(OTHREADS) focus_step_kernel(FocusStepArgs a)
+__global__ void __launch_bounds__(OTHREADS, step_min_blocks<SUB>()) focus_step_kernel(FocusStepArgs a)
 {
     pdl_begin();
     constexpr int NB = SEG / B;
@@ -174,8 +189,10 @@ __global__ void __launch_bounds__(OTHREADS) focus_step_kernel(FocusStepArgs a)
     load_seg_bf16(a.w, a.n, s, y);
     load_seg_coef<NK>(a.c, s, nvalid, SUB, c);
     if constexpr (ADAM) {
-        load_seg_coef<NK>(a.m, s, nvalid, SUB, m);
-        load_seg_coef<NK>(a.v, s, nvalid, SUB, v);
+        // the moments are needed only at the end: start their lines towards
+        // L2 now, load them into registers after the forward pass
+        prefetch_l2(a.m + s * NK);
+        prefetch_l2(a.v + s * NK);
     }
     float S[NB];
     uint32_t sc[NB];
@@ -191,23 +208,53 @@ __global__ void __launch_bounds__(OTHREADS) focus_step_kernel(FocusStepArgs a)
     }
     uint32_t q[4];
     encode_seg<SUB, true>(y, r, zk, a.keep, q);
-    float yh[SEG];
-    decode_seg<B>(q, S, yh);
-    float p[SEG];
+    // Word by word (8 elements): W_hat = val * S_dq, d = W_hat - W, the
+    // products g * W = (d + d) * W in place of W, and d * d; each is
+    // tree-summed over groups of G = min(sub, 8) at once. The adjacent-pair
+    // tree of a sub-block finishes its groups first, so the group sums are then
+    // combined by the same tree: the sums equal tree_sum over the sub-block.
+    constexpr int G = SUB < 8 ? SUB : 8;
+    constexpr int NG = SEG / G;
+    const bool want_sse = a.sse != nullptr;
+    float pg[NG], eg[NG];
 #pragma unroll
-    for (int i = 0; i < SEG; ++i) {
-        const float d = __fsub_rn(yh[i], y[i]);
-        p[i] = __fmul_rn(__fadd_rn(d, d), y[i]);
-        yh[i] = __fmul_rn(d, d);
+    for (int w = 0; w < 4; ++w) {
+        float v[8], e[8];
+        e2m1_unpack8(q[w], v);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;
+            const float d = __fsub_rn(__fmul_rn(v[j], S[i / B]), y[i]);
+            y[i] = __fmul_rn(__fadd_rn(d, d), y[i]);
+            e[j] = __fmul_rn(d, d);
+        }
+#pragma unroll
+        for (int h = 0; h < 8 / G; ++h) {
+            pg[w * (8 / G) + h] = tree_sum<G>(y + 8 * w + h * G);
+            if (want_sse)
+                eg[w * (8 / G) + h] = tree_sum<G>(e + h * G);
+        }
     }
-    if (a.sse != nullptr) {
-        float e[NK];
+    if constexpr (SUB > 8) {
+#pragma unroll
+        for (int k = 0; k < NK; ++k) {
+            pg[k] = tree_sum<SUB / 8>(pg + k * (SUB / 8));
+            if (want_sse)
+                eg[k] = tree_sum<SUB / 8>(eg + k * (SUB / 8));
+        }
+    }
+    if (want_sse) {
+        float es[NK];
 #pragma unroll
         for (int k = 0; k < NK; ++k)
-            e[k] = tree_sum<SUB>(yh + k * SUB);
-        store_seg_floats<NK>(a.sse, s, nvalid, SUB, e);
+            es[k] = eg[k];
+        store_seg_floats<NK>(a.sse, s, nvalid, SUB, es);
     }
-    update_segment<SUB, ADAM>(p, ck, c, m, v, a.o, a.c, a.c_half, a.m, a.v, s, nvalid);
+    if constexpr (ADAM) {
+        load_seg_coef<NK>(a.m, s, nvalid, SUB, m);
+        load_seg_coef<NK>(a.v, s, nvalid, SUB, v);
+    }
+    update_sums<SUB, ADAM>(pg, ck, c, m, v, a.o, a.c, a.c_half, a.m, a.v, s, nvalid);
 }
 
 unsigned grid_of(int64_t n)

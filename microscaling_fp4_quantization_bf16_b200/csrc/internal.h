@@ -91,9 +91,9 @@ struct FocusBwdArgs {
 };
 
 // Optimizer constants of one FOCUS calibration step; om1 = 1 - b1 and
-// om2 = 1 - b2 in fp32, bc1 / bc2 Adam's bias corrections (1 for SGD).
+// om2 = 1 - b2 in fp32; alpha = Adam's step size for this step (lr for SGD).
 struct OptConsts {
-    float lr, b1, b2, om1, om2, bc1, bc2, eps;
+    float lr, b1, b2, om1, om2, alpha, eps;
 };
 
 struct FocusUpdateArgs {
