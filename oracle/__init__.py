@@ -17,9 +17,9 @@ import numpy as np
 
 from . import build as _build
 
-FMT_NVFP4, FMT_MXFP4 = 0, 1
+FMT_NVFP4, FMT_MXFP4, FMT_UE5M3 = 0, 1, 2
 ABSMAX, PREVENT_ZERO, FOUR_OVER_SIX, BRUTE_FORCE = 0, 1, 2, 3
-_FMT = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4}
+_FMT = {"nvfp4": FMT_NVFP4, "mxfp4": FMT_MXFP4, "ue5m3": FMT_UE5M3}
 _STRAT = {"absmax": ABSMAX, "prevent_zero": PREVENT_ZERO, "four_over_six": FOUR_OVER_SIX,
           "brute_force": BRUTE_FORCE}
 
@@ -75,6 +75,14 @@ def lib():
         L.ref_focus_fwd.argtypes = [p, p, i64, i64, i32, i32, i32, p, p, p, p, p, p]
         L.ref_focus_bwd.restype = i32
         L.ref_focus_bwd.argtypes = [p, p, p, i64, i64, i32, p]
+        L.ref_ue5m3_value.restype = C.c_double
+        L.ref_ue5m3_value.argtypes = [i32]
+        L.ref_rne_ue5m3_sat.restype = i32
+        L.ref_rne_ue5m3_sat.argtypes = [C.c_float]
+        L.ref_rne_ue5m3_array.restype = None
+        L.ref_rne_ue5m3_array.argtypes = [p, i64, p]
+        L.ref_rne_ue5m3_bits_range.restype = None
+        L.ref_rne_ue5m3_bits_range.argtypes = [C.c_uint32, i64, p]
         L.ref_float_to_fp16.restype = C.c_uint16
         L.ref_float_to_fp16.argtypes = [C.c_float]
         f32 = C.c_float
@@ -129,6 +137,27 @@ def e4m3_value(code: int) -> float:
 
 def e8m0_value(b: int) -> float:
     return lib().ref_e8m0_value(int(b))
+
+
+def ue5m3_value(code: int) -> float:
+    return lib().ref_ue5m3_value(code)
+
+
+def rne_ue5m3_sat(v: float) -> int:
+    return lib().ref_rne_ue5m3_sat(v)
+
+
+def rne_ue5m3_array(v: np.ndarray) -> np.ndarray:
+    v = np.ascontiguousarray(v, np.float32)
+    out = np.zeros(v.shape, np.uint8)
+    lib().ref_rne_ue5m3_array(_ptr(v), v.size, _ptr(out))
+    return out
+
+
+def rne_ue5m3_bits_range(first: int, n: int) -> np.ndarray:
+    out = np.zeros(n, np.uint8)
+    lib().ref_rne_ue5m3_bits_range(first, n, _ptr(out))
+    return out
 
 
 def rne_e2m1(u: float) -> int:

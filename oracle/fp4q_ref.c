@@ -67,6 +67,13 @@
  *      §2.2 item 1 (per group, the scale minimising the MSE) over the
  *      format's own scales: every E8M0 byte 0..254, scanned upward, a strictly
  *      smaller SSE wins, a tie keeps the lower byte.
+ *  R17 UE5M3 block scales ([FINER] 意義と主張 names the unsigned wide-exponent
+ *      format without its encoding): 8 bits, 5 exponent bits with the IEEE
+ *      bias 15, 3 mantissa bits, exponent field 0 subnormal (m * 2^-17),
+ *      only 0xFF NaN as in OCP E4M3; largest 1.75 * 2^16 (0xFE). Its range
+ *      needs no hierarchical scaling, so s_g = 1: candidate code =
+ *      RNE_UE5M3_sat(amax / T); the four strategies as for E4M3, brute force
+ *      over codes 0x01..0xFE.
  *  R15 FOCUS calibration: the pages learn c by gradient descent through the
  *      STE but name neither the optimizer nor the precision of the update.
  *      The learnable state is an fp32 master copy of c; the forward uses its
@@ -89,6 +96,7 @@
 
 #define REF_FMT_NVFP4 0
 #define REF_FMT_MXFP4 1
+#define REF_FMT_UE5M3 2
 
 #define REF_ABSMAX 0
 #define REF_PREVENT_ZERO 1
@@ -268,6 +276,50 @@ int ref_rne_e4m3_sat(float v)
     return (k & 1) ? k - 1 : k;
 }
 
+/* UE5M3 value of a byte 0..0xFE (reading R17): unsigned, 5 exponent bits with
+ * bias 15, 3 mantissa bits, exponent field 0 subnormal; 0xFF is NaN.
+ * [FINER] 意義と主張 (UE5M3 as the wide-range scale format compared with
+ * E4M3 + hierarchical scaling). */
+double ref_ue5m3_value(int code)
+{
+    int e = (code >> 3) & 31;
+    int m = code & 7;
+    if ((code & 0xFF) == 0xFF)
+        return NAN;
+    return (e == 0) ? ldexp(m / 8.0, 1 - 15) : ldexp(1.0 + m / 8.0, e - 15);
+}
+
+/* Round v >= 0 to the nearest finite UE5M3 value, ties to the even code,
+ * saturating above the largest value 1.75 * 2^16 (code 0xFE); bisection over
+ * the enumerated codes 0..0xFE, which increase with their value. */
+int ref_rne_ue5m3_sat(float v)
+{
+    double top = ref_ue5m3_value(0xFE);
+    if (!((double)v <= top))
+        return 0xFE;
+    double x = (double)v;
+    if (x <= 0.0)
+        return 0;
+    int lo = 0, hi = 0xFE;
+    while (lo < hi) {
+        int mid = (lo + hi) / 2;
+        if (ref_ue5m3_value(mid) >= x)
+            hi = mid;
+        else
+            lo = mid + 1;
+    }
+    int k = lo;
+    if (ref_ue5m3_value(k) == x)
+        return k;
+    double dk = ref_ue5m3_value(k) - x;
+    double dp = x - ref_ue5m3_value(k - 1);
+    if (dp < dk)
+        return k - 1;
+    if (dk < dp)
+        return k;
+    return (k & 1) ? k - 1 : k;
+}
+
 /* E8M0 exponent for a block abs-max a >= 0: floor(log2 a) - 2, clamped to
  * [-127, 127]; a == 0 gives -127. frexp writes a = f * 2^k, f in [0.5, 1),
  * so floor(log2 a) = k - 1 exactly. */
@@ -405,9 +457,21 @@ static float quant_block(const float* y, int B, float S, uint8_t* q, float* yhat
     return ref_tsum(e, B);
 }
 
-/* NVFP4 scale candidate for target T (6 = abs-max, 4 = the 4-over-6
- * alternative): raw = amax / (T * s_g), code = RNE_E4M3_sat(raw),
- * S = e4m3(code) * s_g. [FINER] 手法 2 (abs-max rounded to the nearest E4M3
+/* The block-scale formats of the NVFP4 family: E4M3 (under the FP32 global
+ * scale s_g) and UE5M3 (reading R17: its range needs no global scale, so s_g
+ * is 1). max_code is the largest finite code. */
+typedef struct {
+    int (*rne)(float);
+    double (*value)(int);
+    int max_code;
+} scale_format;
+
+static const scale_format FMT_E4M3 = {ref_rne_e4m3_sat, ref_e4m3_value, 0x7E};
+static const scale_format FMT_UE5M3 = {ref_rne_ue5m3_sat, ref_ue5m3_value, 0xFE};
+
+/* Scale candidate for target T (6 = abs-max, 4 = the 4-over-6 alternative):
+ * raw = amax / (T * s_g), code = RNE_sat(raw) in the scale format,
+ * S = value(code) * s_g. [FINER] 手法 2 (abs-max rounded to the nearest E4M3
  * value; 4-over-6 targets; hierarchical scaling). */
 static int nv_candidate(float amax, float T, float sg, float* S)
 {
@@ -418,10 +482,20 @@ static int nv_candidate(float amax, float T, float sg, float* S)
     return c;
 }
 
-/* Selects the NVFP4 scale of one block by the given strategy and quantizes it
- * with that scale. Returns the block SSE; writes scale byte, codes, yhat. */
-static float nv_block(const float* y, int B, int strat, float sg, uint8_t* scale, uint8_t* q,
-                      float* yhat)
+static int scale_candidate(const scale_format* f, float amax, float T, float sg, float* S)
+{
+    float den = T * sg;
+    float raw = amax / den;
+    int c = f->rne(raw);
+    *S = (float)f->value(c) * sg;
+    return c;
+}
+
+/* Selects the block scale (E4M3 or UE5M3 format f) of one block by the given
+ * strategy and quantizes it with that scale. Returns the block SSE; writes
+ * scale byte, codes, yhat. */
+static float nv_block(const float* y, int B, int strat, float sg, const scale_format* f,
+                      uint8_t* scale, uint8_t* q, float* yhat)
 {
     float amax = 0.0f;
     for (int i = 0; i < B; i++) {
@@ -430,16 +504,16 @@ static float nv_block(const float* y, int B, int strat, float sg, uint8_t* scale
             amax = a;
     }
     float S6;
-    int c6 = nv_candidate(amax, 6.0f, sg, &S6);
+    int c6 = scale_candidate(f, amax, 6.0f, sg, &S6);
     if (strat == REF_ABSMAX) {
         *scale = (uint8_t)c6;
         return quant_block(y, B, S6, q, yhat);
     }
     if (strat == REF_PREVENT_ZERO) {
-        /* clip the scale to the smallest positive E4M3 value 2^-9 (code 0x01),
-         * [FINER] 手法 2 prevent-zero */
+        /* clip the scale to the smallest positive value of the format (code
+         * 0x01: 2^-9 in E4M3), [FINER] 手法 2 prevent-zero */
         int c = c6 < 1 ? 1 : c6;
-        float S = (float)ref_e4m3_value(c) * sg;
+        float S = (float)f->value(c) * sg;
         *scale = (uint8_t)c;
         return quant_block(y, B, S, q, yhat);
     }
@@ -447,7 +521,7 @@ static float nv_block(const float* y, int B, int strat, float sg, uint8_t* scale
         uint8_t q4[128];
         float yh4[128];
         float S4;
-        int c4 = nv_candidate(amax, 4.0f, sg, &S4);
+        int c4 = scale_candidate(f, amax, 4.0f, sg, &S4);
         float sse6 = quant_block(y, B, S6, q, yhat);
         float sse4 = quant_block(y, B, S4, q4, yh4);
         if (sse4 < sse6) {
@@ -459,20 +533,20 @@ static float nv_block(const float* y, int B, int strat, float sg, uint8_t* scale
         *scale = (uint8_t)c6;
         return sse6;
     }
-    /* brute force over every positive finite E4M3 code, [FINER] 手法 2 */
+    /* brute force over every positive finite code, [FINER] 手法 2 */
     uint8_t qt[128];
     float yht[128];
     int best_c = -1;
     float best = 0.0f;
-    for (int c = 0x01; c <= 0x7E; c++) {
-        float S = (float)ref_e4m3_value(c) * sg;
+    for (int c = 0x01; c <= f->max_code; c++) {
+        float S = (float)f->value(c) * sg;
         float sse = quant_block(y, B, S, qt, yht);
         if (best_c < 0 || sse < best) {
             best = sse;
             best_c = c;
         }
     }
-    float S = (float)ref_e4m3_value(best_c) * sg;
+    float S = (float)f->value(best_c) * sg;
     *scale = (uint8_t)best_c;
     return quant_block(y, B, S, q, yhat);
 }
@@ -517,9 +591,9 @@ static int valid_common(int64_t rows, int64_t cols, int fmt, int block, int rot)
         return 0;
     if (fmt == REF_FMT_MXFP4 && block != 32)
         return 0;
-    if (fmt == REF_FMT_NVFP4 && block != 4 && block != 8 && block != 16 && block != 32)
+    if (fmt != REF_FMT_MXFP4 && block != 4 && block != 8 && block != 16 && block != 32)
         return 0;
-    if (fmt != REF_FMT_NVFP4 && fmt != REF_FMT_MXFP4)
+    if (fmt != REF_FMT_NVFP4 && fmt != REF_FMT_MXFP4 && fmt != REF_FMT_UE5M3)
         return 0;
     if (rot != 0 && rot != 16 && rot != 32 && rot != 64 && rot != 128)
         return 0;
@@ -563,8 +637,10 @@ int ref_quantize(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int blo
         for (int64_t b = 0; b < nb; b++) {
             const float* yb = y + b * block;
             uint8_t sc;
-            float sse = (fmt == REF_FMT_MXFP4) ? mx_block(yb, block, strat, &sc, q, yhat)
-                                               : nv_block(yb, block, strat, sg, &sc, q, yhat);
+            float sse = (fmt == REF_FMT_MXFP4)
+                            ? mx_block(yb, block, strat, &sc, q, yhat)
+                            : nv_block(yb, block, strat, sg,
+                                       fmt == REF_FMT_UE5M3 ? &FMT_UE5M3 : &FMT_E4M3, &sc, q, yhat);
             int64_t base = i * cols + b * block;
             scales[i * nb + b] = sc;
             if (block_mse)
@@ -588,6 +664,8 @@ static float block_scale(int fmt, uint8_t sc, float sg)
 {
     if (fmt == REF_FMT_MXFP4)
         return (float)ref_e8m0_value(sc);
+    if (fmt == REF_FMT_UE5M3)
+        return (float)ref_ue5m3_value(sc);
     return (float)ref_e4m3_value(sc) * sg;
 }
 
@@ -728,6 +806,8 @@ int ref_focus_fwd(const uint16_t* w, const uint16_t* c, int64_t rows, int64_t co
 {
     if (!valid_common(rows, cols, fmt, block, 0))
         return REF_ERR_ARG;
+    if (fmt == REF_FMT_UE5M3)
+        return REF_ERR_ARG; /* FOCUS is defined for MXFP4 and NVFP4 */
     if (sub < 1 || block % sub != 0 || (sub & (sub - 1)) != 0)
         return REF_ERR_ARG;
     float sg = 1.0f;
@@ -965,6 +1045,8 @@ int ref_focus_step(const uint16_t* w, int64_t rows, int64_t cols, int fmt, int b
 {
     if (!valid_common(rows, cols, fmt, block, 0))
         return REF_ERR_ARG;
+    if (fmt == REF_FMT_UE5M3)
+        return REF_ERR_ARG; /* FOCUS is defined for MXFP4 and NVFP4 */
     if (sub < 1 || block % sub != 0 || (sub & (sub - 1)) != 0 || !valid_opt(opt, m, v, t))
         return REF_ERR_ARG;
     float sg = 1.0f;
@@ -1057,6 +1139,18 @@ void ref_rne_e4m3_bits_range(uint32_t first, int64_t n, uint8_t* out)
 {
     for (int64_t i = 0; i < n; i++)
         out[i] = (uint8_t)ref_rne_e4m3_sat(bits2f(first + (uint32_t)i));
+}
+
+void ref_rne_ue5m3_array(const float* v, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = (uint8_t)ref_rne_ue5m3_sat(v[i]);
+}
+
+void ref_rne_ue5m3_bits_range(uint32_t first, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; i++)
+        out[i] = (uint8_t)ref_rne_ue5m3_sat(bits2f(first + (uint32_t)i));
 }
 
 void ref_fwht_array(float* t, int64_t n_chunks, int n)

@@ -224,3 +224,62 @@ def test_e4m3_dense_and_sweep(ref):
     sweep = np.arange(0, 0x7F800001, 9973, dtype=np.uint64).astype(np.uint32)
     v = np.concatenate([bits, sweep]).view(np.float32)
     _check_e4m3(ref, v, ref.rne_e4m3_array(v))
+
+
+# ---------------------------------------------------------- UE5M3 (reading)
+
+def _ue5m3_table(ref):
+    return np.array([ref.ue5m3_value(c) for c in range(0xFF)], np.float64)
+
+
+def test_ue5m3_table_closed_form(ref):
+    # the reading of the unsigned 5-exponent / 3-mantissa scale format: bias 15,
+    # subnormals m * 2^-17, 0xFF NaN; the value set is exactly the subnormals
+    # and {k * 2^(e-3): 8 <= k < 16, -14 <= e <= 16} less its top (1.875 * 2^16,
+    # the NaN pattern)
+    vals = list(_ue5m3_table(ref))
+    assert vals[0] == 0.0 and math.isnan(ref.ue5m3_value(0xFF))
+    assert all(b > a for a, b in zip(vals, vals[1:])), "codes 0..0xFE must increase"
+    subn = [k * 2.0 ** -17 for k in range(1, 8)]
+    normals = sorted(k * 2.0 ** (e - 3) for e in range(-14, 17) for k in range(8, 16))[:-1]
+    assert vals[1:] == subn + normals
+    assert vals[0xFE] == 1.75 * 2 ** 16 and vals[1] == 2.0 ** -17 and vals[8] == 2.0 ** -14
+    assert ref.ue5m3_value(15 << 3) == 1.0
+
+
+def _check_ue5m3(ref, v: np.ndarray, codes: np.ndarray):
+    tab = _ue5m3_table(ref)
+    x = v.astype(np.float64)
+    assert np.all(codes <= 0xFE)
+    sat = x > tab[-1]
+    assert np.all(codes[sat] == 0xFE)
+    xi = x[~sat]
+    ci = codes[~sat].astype(np.int64)
+    d = np.abs(xi[:, None] - tab[None, :])
+    dmin = d.min(axis=1)
+    assert np.all(d[np.arange(len(xi)), ci] == dmin)
+    ties = (d == dmin[:, None]).sum(axis=1) > 1
+    assert np.all(ci[ties] % 2 == 0)
+
+
+def test_ue5m3_closed_form_points(ref):
+    assert ref.rne_ue5m3_sat(1.0) == 0x78
+    assert ref.rne_ue5m3_sat(1.0625) == 0x78        # tie 1 / 1.125 -> even code
+    assert ref.rne_ue5m3_sat(1.1875) == 0x7A        # tie 1.125 / 1.25 -> even code
+    assert ref.rne_ue5m3_sat(2.0 ** -18) == 0       # tie 0 / 2^-17 -> code 0
+    assert ref.rne_ue5m3_sat(3 * 2.0 ** -18) == 2   # tie 2^-17 / 2^-16 -> even code 2
+    assert ref.rne_ue5m3_sat(114688.0) == 0xFE and ref.rne_ue5m3_sat(1e30) == 0xFE
+    assert ref.rne_ue5m3_sat(float("inf")) == 0xFE
+    assert ref.rne_ue5m3_sat(0.0) == 0 and ref.rne_ue5m3_sat(-0.0) == 0
+
+
+def test_ue5m3_dense_and_sweep(ref):
+    tab = _ue5m3_table(ref).astype(np.float32)
+    mids = ((tab[1:].astype(np.float64) + tab[:-1]) / 2).astype(np.float32)
+    base = np.concatenate([tab, mids]).view(np.uint32)
+    offs = np.arange(-100, 101, dtype=np.int64)
+    bits = (base[:, None].astype(np.int64) + offs[None, :]).reshape(-1)
+    bits = bits[(bits >= 0) & (bits < 0x7F800000)].astype(np.uint32)
+    sweep = np.arange(0, 0x7F800001, 19997, dtype=np.uint64).astype(np.uint32)
+    v = np.concatenate([bits, sweep]).view(np.float32)
+    _check_ue5m3(ref, v, ref.rne_ue5m3_array(v))

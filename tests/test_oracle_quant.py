@@ -454,3 +454,59 @@ def test_fp4_gemm_one_hot_rows(ref):
     d = ref.fp4_gemm(ac, asc, 2.0, bc, bsc, 0.5, "nvfp4")
     a = ref.dequantize(ac, asc, 1.0, M, K, "nvfp4", 16)
     assert np.array_equal(d, a[:, cols])
+
+
+# ------------------------------------------------- UE5M3 block scales (R17)
+
+def ue5m3_table(ref):
+    return np.array([ref.ue5m3_value(c) for c in range(0xFF)], np.float64)
+
+
+@pytest.mark.parametrize("block", [4, 8, 16, 32])
+@pytest.mark.parametrize("strategy", ["absmax", "prevent_zero", "four_over_six", "brute_force"])
+def test_ue5m3_exact_round_trip(ref, block, strategy):
+    # y = value(q) * ue5m3(c) with one element per block at +-6: every strategy
+    # must return c and q exactly (no global scale: the code is set by the block)
+    rng = np.random.default_rng(100 + block)
+    rows, cols = 8, 64
+    nb = cols // block
+    c = rng.integers(1, 0xFF, size=(rows, nb))
+    c[0, 0], c[0, -1] = 1, 0xFE          # smallest subnormal and largest code
+    q = rng.integers(0, 16, size=(rows, cols))
+    q.reshape(rows, nb, block)[:, :, 0] = rng.choice([7, 15], size=(rows, nb))
+    y = E2M1[q] * np.repeat(ue5m3_table(ref)[c], block, axis=1)
+    x = bf16_bits(y)
+    assert np.array_equal(f32_of_bf16(x).astype(np.float64), y)
+    out = ref.quantize(x, "ue5m3", block, strategy, 0, dq="f32")
+    assert np.array_equal(out["scales"], c.astype(np.uint8))
+    assert np.array_equal(ref.unpack_codes(out["codes"]), q.astype(np.uint8))
+    assert np.array_equal(out["dq"].astype(np.float64), y)
+    assert np.all(out["mse"] == 0)
+
+
+@pytest.mark.parametrize("block", [4, 16])
+def test_ue5m3_strategy_relations_and_scale_shift(ref, block):
+    x = _with_tiny_rows(synth.workload("c3_strategy_sweep_t3", rows=32, cols=256)["x"])
+    xb = synth.bits16(x)
+    res = {s: ref.quantize(xb, "ue5m3", block, s, 0, dq="f32")
+           for s in ("absmax", "prevent_zero", "four_over_six", "brute_force")}
+    am, pz, fs, bf = (res[s] for s in ("absmax", "prevent_zero", "four_over_six", "brute_force"))
+    assert np.all(pz["scales"] >= 1) and np.all(bf["scales"] >= 1)
+    assert np.all(fs["mse"] <= am["mse"])
+    assert np.all(bf["mse"] <= pz["mse"])
+    pos = fs["scales"] >= 1
+    assert np.all(bf["mse"][pos] <= fs["mse"][pos])
+    for r in res.values():
+        dq = ref.dequantize(r["codes"], r["scales"], None, *xb.shape, "ue5m3", block, "f32")
+        assert np.array_equal(dq.view(np.uint32), r["dq"].view(np.uint32))
+        m = ref.block_mse(xb, r["codes"], r["scales"], None, "ue5m3", block, 0)
+        assert np.array_equal(m.view(np.uint32), r["mse"].view(np.uint32))
+    # no global scale: scaling the tensor by 2^k moves every normal-range code
+    # by 8k (one exponent step is 8 codes) and keeps the element codes
+    big = am["scales"] >= 8 + 8 * 3
+    x8 = bf16_bits(f32_of_bf16(xb).astype(np.float64) / 8.0)
+    a8 = ref.quantize(x8, "ue5m3", block, "absmax", 0)
+    assert np.array_equal(a8["scales"][big].astype(np.int64), am["scales"][big].astype(np.int64) - 24)
+    cb = ref.unpack_codes(am["codes"]).reshape(32, -1, block)
+    c8 = ref.unpack_codes(a8["codes"]).reshape(32, -1, block)
+    assert np.array_equal(cb[big], c8[big])
