@@ -408,8 +408,9 @@ def breakdown(dev, peaks, reps: int = 10):
                 for _ in range(nc)]
             dqb = 0 if dq is None else torch.tensor([], dtype=dq).element_size()
             bpe = bytes_per_elem(block, mse=want_mse, dq=dqb)
-            ops = n * (126 if nv else 255) * 5 if strat == "brute_force" else None
-            label = "mse_grid (E8M0 brute force)" if (strat == "brute_force" and not nv) else strat
+            ncodes = {"nvfp4": 126, "mxfp4": 255, "ue5m3": 254}[fmt]
+            ops = n * ncodes * 5 if strat == "brute_force" else None
+            label = "mse_grid (E8M0 brute force)" if (strat == "brute_force" and fmt == "mxfp4") else strat
             tag = f"{wl} {fmt} B{block} {label} H{rot}"
             if nv:
                 ga = fp4q.global_amax(x0, rot)
@@ -450,6 +451,25 @@ def breakdown(dev, peaks, reps: int = 10):
     quant_runs("c3_strategy_sweep_t3", [("nvfp4", b, s, 0) for b in (4, 8, 16, 32)
                                         for s in ("absmax", "prevent_zero", "four_over_six",
                                                   "brute_force")], want_mse=True)
+    quant_runs("c3_strategy_sweep_t3", [("ue5m3", 16, s, 0) for s in ("absmax", "four_over_six",
+                                                                       "brute_force")]
+               + [("ue5m3", 4, "four_over_six", 0)], want_mse=True)
+    # quality beside speed: the tensor's mean block MSE on C3 with E4M3 scales
+    # under the FP32 global scale (hierarchical) and with UE5M3 scales (none),
+    # the comparison "Finer is Better ..." draws (意義と主張)
+    x3 = synth.workload("c3_strategy_sweep_t3")["x"].to(dev)
+    ga3 = fp4q.global_amax(x3, 0)
+    qual = {}
+    for block in (4, 16):
+        for fmt in ("nvfp4", "ue5m3"):
+            for strat in ("absmax", "four_over_six", "brute_force"):
+                q3 = fp4q.quantize(x3, fmt, block, strat, 0,
+                                   global_amax=ga3 if fmt == "nvfp4" else None, want_mse=True)
+                qual[f"{fmt} B{block} {strat}"] = float(q3.mse.double().mean())
+    rows_out.append({"run": "c3_strategy_sweep_t3 quality: mean block MSE (E4M3 + s_g vs UE5M3)",
+                     "mse": {k: float(f"{v:.6e}") for k, v in qual.items()}})
+    del x3, q3
+    torch.cuda.empty_cache()
     quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
                                           ("mxfp4", 32, "absmax", 128)])
     # W4A4 GEMM on the block-scaled tensor cores, LLM layer shapes (tokens x hidden

@@ -63,7 +63,18 @@ typedef enum {
     FP4Q_ERR_CUDA = 6         /* the CUDA runtime rejected a launch */
 } fp4q_status;
 
-typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1 } fp4q_format;
+/* Block formats: FP4 (E2M1) elements with
+ *   NVFP4  E4M3 block scales under an FP32 per-tensor scale s_g; blocks 4..32
+ *   MXFP4  E8M0 (power-of-two) block scales; block 32
+ *   UE5M3  unsigned 5-exponent / 3-mantissa block scales with no per-tensor
+ *          scale; blocks 4..32. "Finer is Better (with the Right Scaling)"
+ *          (意義と主張) compares this wide-range format with E4M3 +
+ *          hierarchical scaling but gives no encoding; this library reads it
+ *          as bias 15, subnormals at exponent field 0 (m * 2^-17), 0xFF the
+ *          only NaN, largest 1.75 * 2^16 (0xFE), values above it saturating,
+ *          round to nearest even. Quantize, dequantize and block MSE take it;
+ *          FOCUS and the GEMM do not (FP4Q_ERR_UNSUPPORTED). */
+typedef enum { FP4Q_FMT_NVFP4 = 0, FP4Q_FMT_MXFP4 = 1, FP4Q_FMT_UE5M3 = 2 } fp4q_format;
 
 /* Block-scale selection ("Finer is Better (with the Right Scaling)", 手法 2).
  * MXFP4 offers FP4Q_ABSMAX (E8M0 byte floor(log2 amax) - 2 + 127) and
@@ -89,7 +100,9 @@ typedef enum { FP4Q_OPT_SGD = 0, FP4Q_OPT_ADAM = 1 } fp4q_optimizer;
  * with optional dequantized values and per-block MSE.
  *
  * x                bf16 [rows, cols].
- * fmt, block       NVFP4 with block in {4, 8, 16, 32}; MXFP4 with block 32.
+ * fmt, block       NVFP4 or UE5M3 with block in {4, 8, 16, 32}; MXFP4 with
+ *                  block 32. UE5M3 candidate codes: RNE_UE5M3(amax / T), T = 6
+ *                  (and 4 for 4-over-6); brute force over codes 0x01..0xFE.
  * strat            see fp4q_strategy.
  * rot              0 (none) or the blockwise Hadamard size 16, 32, 64, 128:
  *                  every rot-wide chunk of a row becomes H_rot x / sqrt(rot)
@@ -98,9 +111,9 @@ typedef enum { FP4Q_OPT_SGD = 0, FP4Q_OPT_ADAM = 1 } fp4q_optimizer;
  * global_amax_in   NVFP4: NULL to compute the abs-max of the (rotated)
  *                  tensor on the device (an extra read of x), or a device
  *                  float holding a calibrated abs-max (single pass). Ignored
- *                  for MXFP4.
+ *                  for MXFP4 and UE5M3.
  * global_scale_out NVFP4: required device float, receives s_g. Ignored for
- *                  MXFP4. When global_amax_in is NULL it is also used to
+ *                  MXFP4 and UE5M3. When global_amax_in is NULL it is also used to
  *                  accumulate the abs-max before s_g replaces it.
  * codes            uint8 [rows, cols/2], required.
  * scales           uint8 [rows, cols/block], required.
@@ -115,11 +128,11 @@ fp4q_status fp4q_quantize(const void* x, int64_t rows, int64_t cols, fp4q_format
                           float* block_mse, void* dq, fp4q_dtype dq_dtype, cudaStream_t stream);
 
 /*
- * fp4q_dequantize -- value(code) * S with S = E4M3(scale) * s_g (NVFP4) or
- * 2^(scale - 127) (MXFP4); only the dequantization scale is needed at
+ * fp4q_dequantize -- value(code) * S with S = E4M3(scale) * s_g (NVFP4),
+ * 2^(scale - 127) (MXFP4) or UE5M3(scale); only the dequantization scale is needed at
  * inference ("FOCUS: FP4 Optimization via Coupled-Relaxation and
  * Dual-Granularity Scaling", Metodologia §4).
- * global_scale: NVFP4 device float s_g (required); ignored for MXFP4.
+ * global_scale: NVFP4 device float s_g (required); ignored for MXFP4 and UE5M3.
  * out: [rows, cols] of out_dtype (bf16 output is the RNE rounding of the fp32 value).
  */
 fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,

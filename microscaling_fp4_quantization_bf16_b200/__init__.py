@@ -21,7 +21,7 @@ import torch
 from ._abi import Fp4qError, load  # noqa: F401
 from . import _abi
 
-FORMATS = {"nvfp4": 0, "mxfp4": 1}
+FORMATS = {"nvfp4": 0, "mxfp4": 1, "ue5m3": 2}
 STRATEGIES = {"absmax": 0, "prevent_zero": 1, "four_over_six": 2, "brute_force": 3}
 DTYPES = {torch.float32: 0, torch.bfloat16: 1}
 

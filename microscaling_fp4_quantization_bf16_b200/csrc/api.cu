@@ -45,11 +45,11 @@ constexpr int64_t kMaxElems = (int64_t)1 << 40;
 // Shared checks of format, block and rotation against the shape.
 fp4q_status check_format(int64_t rows, int64_t cols, int fmt, int block, int rot)
 {
-    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4 && fmt != FP4Q_FMT_UE5M3)
         return FP4Q_ERR_UNSUPPORTED;
     if (fmt == FP4Q_FMT_MXFP4 && block != 32)
         return FP4Q_ERR_UNSUPPORTED;
-    if (fmt == FP4Q_FMT_NVFP4 && block != 4 && block != 8 && block != 16 && block != 32)
+    if (fmt != FP4Q_FMT_MXFP4 && block != 4 && block != 8 && block != 16 && block != 32)
         return FP4Q_ERR_UNSUPPORTED;
     if (!valid_rot(rot))
         return FP4Q_ERR_UNSUPPORTED;
@@ -112,7 +112,8 @@ bool make_row_map(CUtensorMap* map, const void* x, int64_t n)
 cudaError_t launch_quant(int block, int strat, int rot, const QuantArgs& a, cudaStream_t st)
 {
     const bool tma_shape = a.n % 64 == 0 && a.n / 64 < ((int64_t)1 << 31);
-    if (strat != K_BRUTE_FORCE && strat != K_MX_BRUTE && tma_shape && tma_requested()) {
+    const bool tma_strat = strat != K_BRUTE_FORCE && strat != K_MX_BRUTE && !is_ue_strat(strat);
+    if (tma_strat && tma_shape && tma_requested()) {
         CUtensorMap map;
         if (make_row_map(&map, a.x, a.n)) {
             int dev = 0, sms = 0;
@@ -211,6 +212,8 @@ fp4q_status quantize_impl(const void* x, int64_t rows, int64_t cols, fp4q_format
         a.mma_atoms_k = (uint32_t)((cols / block + 3) / 4);
     }
     int kstrat = nv ? (int)strat : (strat == FP4Q_BRUTE_FORCE ? K_MX_BRUTE : K_MX);
+    if (fmt == FP4Q_FMT_UE5M3)
+        kstrat = K_UE_ABSMAX + (int)strat;
     if (nv) {
         if (global_amax_in != nullptr) {
             a.amax = global_amax_in;
@@ -284,7 +287,7 @@ fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
     a.out = out;
     a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
     a.keep = 0xFFFFFFFFu;
-    return cuda_status(launch_dequant(nv ? 0 : 1, block, a, stream));
+    return cuda_status(launch_dequant((int)fmt, block, a, stream));
 }
 
 fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales,
@@ -313,7 +316,7 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
     a.out = out;
     a.out_kind = out_dtype == FP4Q_OUT_F32 ? 1 : 2;
     a.keep = 0xFFFFFFFFu;
-    return cuda_status(launch_dequant_rot(nv ? 0 : 1, block, rot, a, stream));
+    return cuda_status(launch_dequant_rot((int)fmt, block, rot, a, stream));
 }
 
 size_t fp4q_mma_scale_bytes(int64_t rows, int64_t K, fp4q_format fmt)
@@ -403,7 +406,7 @@ fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* s
     a.sg = nv ? global_scale : nullptr;
     a.n = n;
     a.mse = block_mse;
-    return cuda_status(launch_block_mse(nv ? 0 : 1, block, rot, a, stream));
+    return cuda_status(launch_block_mse((int)fmt, block, rot, a, stream));
 }
 
 fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t cols,
@@ -414,6 +417,8 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
     fp4q_status st = check_format(rows, cols, fmt, block, 0);
     if (st != FP4Q_OK)
         return st;
+    if (fmt == FP4Q_FMT_UE5M3)
+        return FP4Q_ERR_UNSUPPORTED;  // FOCUS is defined for MXFP4 and NVFP4
     if (!valid_sub(sub) || sub > block)
         return FP4Q_ERR_UNSUPPORTED;
     if (out_dtype != FP4Q_OUT_F32 && out_dtype != FP4Q_OUT_BF16)
@@ -566,6 +571,8 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
     fp4q_status st = check_format(rows, cols, fmt, block, 0);
     if (st != FP4Q_OK)
         return st;
+    if (fmt == FP4Q_FMT_UE5M3)
+        return FP4Q_ERR_UNSUPPORTED;  // FOCUS is defined for MXFP4 and NVFP4
     if (!valid_sub(sub) || sub > block)
         return FP4Q_ERR_UNSUPPORTED;
     st = check_opt(opt, t, m, v);

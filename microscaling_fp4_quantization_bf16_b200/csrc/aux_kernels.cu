@@ -164,12 +164,14 @@ __device__ __forceinline__ void load_scale_bytes(const uint8_t* scales, int64_t 
         sc[b] = (b * B < nvalid) ? (uint32_t)scales[s * NB + b] : 0u;
 }
 
-template <int NB, bool MX>
+// Block scales from their bytes. FMT: 0 NVFP4 (E4M3 times s_g), 1 MXFP4
+// (E8M0), 2 UE5M3 (no global scale).
+template <int NB, int FMT>
 __device__ __forceinline__ void scales_of(const uint32_t (&sc)[NB], float sg, float (&S)[NB])
 {
 #pragma unroll
     for (int b = 0; b < NB; ++b)
-        S[b] = MX ? e8m0_dec(sc[b]) : __fmul_rn(e4m3_dec(sc[b]), sg);
+        S[b] = FMT == 1 ? e8m0_dec(sc[b]) : (FMT == 2 ? ue5m3_dec(sc[b]) : __fmul_rn(e4m3_dec(sc[b]), sg));
 }
 
 // ------------------------------------------------------------ dequantize
@@ -177,7 +179,7 @@ __device__ __forceinline__ void scales_of(const uint32_t (&sc)[NB], float sg, fl
 // One thread per EPT consecutive elements (EPT = 8 for bf16 output, 4 for
 // fp32): its 16 output bytes are one store, and a warp's stores cover 512
 // contiguous bytes. A thread's elements lie in one block unless B = 4 < EPT.
-template <int B, bool MX, int EPT>
+template <int B, int FMT, int EPT>
 __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 {
     pdl_begin();
@@ -196,9 +198,9 @@ __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 #pragma unroll
     for (int k = 0; k < NS; ++k)
         sc[k] = (k * B < nvalid) ? (uint32_t)a.scales[e0 / B + k] : 0u;
-    const float sg = MX ? 1.0f : *a.sg;
+    const float sg = FMT == 0 ? *a.sg : 1.0f;
     float S[NS];
-    scales_of<NS, MX>(sc, sg, S);
+    scales_of<NS, FMT>(sc, sg, S);
     float v[EPT];
     if constexpr (EPT == 8)
         e2m1_unpack8(q, v);
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
     }
 }
 
-template <int B, bool MX>
+template <int B, int FMT>
 static cudaError_t launch_dequant_b(const DequantArgs& a, cudaStream_t st)
 {
     const int ept = a.out_kind == 2 ? 8 : 4;
@@ -236,19 +238,30 @@ static cudaError_t launch_dequant_b(const DequantArgs& a, cudaStream_t st)
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nthr);
     if (ept == 8)
-        return launch_pdl(dequant_kernel<B, MX, 8>, dim3(g), dim3(ATHREADS), 0, st, a);
-    return launch_pdl(dequant_kernel<B, MX, 4>, dim3(g), dim3(ATHREADS), 0, st, a);
+        return launch_pdl(dequant_kernel<B, FMT, 8>, dim3(g), dim3(ATHREADS), 0, st, a);
+    return launch_pdl(dequant_kernel<B, FMT, 4>, dim3(g), dim3(ATHREADS), 0, st, a);
 }
 
-cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st)
+template <int FMT>
+static cudaError_t launch_dequant_blocks(int block, const DequantArgs& a, cudaStream_t st)
 {
-    if (mx)
-        return block == 32 ? launch_dequant_b<32, true>(a, st) : cudaErrorInvalidValue;
+    if (FMT == 1 && block != 32)
+        return cudaErrorInvalidValue;
     switch (block) {
-    case 4: return launch_dequant_b<4, false>(a, st);
-    case 8: return launch_dequant_b<8, false>(a, st);
-    case 16: return launch_dequant_b<16, false>(a, st);
-    case 32: return launch_dequant_b<32, false>(a, st);
+    case 4: return launch_dequant_b<4, FMT>(a, st);
+    case 8: return launch_dequant_b<8, FMT>(a, st);
+    case 16: return launch_dequant_b<16, FMT>(a, st);
+    case 32: return launch_dequant_b<32, FMT>(a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_dequant(int fmt, int block, const DequantArgs& a, cudaStream_t st)
+{
+    switch (fmt) {
+    case 0: return launch_dequant_blocks<0>(block, a, st);
+    case 1: return launch_dequant_blocks<1>(block, a, st);
+    case 2: return launch_dequant_blocks<2>(block, a, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -260,7 +273,7 @@ cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t
 // `keep` before the butterflies: ptxas would otherwise fuse the packed
 // multiply of the decode into the first packed add of the rotation, which
 // changes the rounding.
-template <int B, bool MX, int ROT>
+template <int B, int FMT, int ROT>
 __global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
 {
     pdl_begin();
@@ -280,9 +293,9 @@ __global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
         load_codes(a.codes, s, nvalid, q);
         load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
     }
-    const float sg = MX ? 1.0f : *a.sg;
+    const float sg = FMT == 0 ? *a.sg : 1.0f;
     float S[NB], yh[SEG];
-    scales_of<NB, MX>(sc, sg, S);
+    scales_of<NB, FMT>(sc, sg, S);
     decode_seg<B>(q, S, yh);
 #pragma unroll
     for (int i = 0; i < SEG; ++i)
@@ -292,7 +305,7 @@ __global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
         store_seg_values(a.out, a.out_kind, s, nvalid, yh);
 }
 
-template <int B, bool MX>
+template <int B, int FMT>
 static cudaError_t launch_dequant_rot_b(int rot, const DequantArgs& a, cudaStream_t st)
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
@@ -300,25 +313,36 @@ static cudaError_t launch_dequant_rot_b(int rot, const DequantArgs& a, cudaStrea
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nseg);
     switch (rot) {
-    case 16: return launch_pdl(dequant_rot_kernel<B, MX, 16>, dim3(g), dim3(ATHREADS), 0, st, a);
-    case 32: return launch_pdl(dequant_rot_kernel<B, MX, 32>, dim3(g), dim3(ATHREADS), 0, st, a);
-    case 64: return launch_pdl(dequant_rot_kernel<B, MX, 64>, dim3(g), dim3(ATHREADS), 0, st, a);
-    case 128: return launch_pdl(dequant_rot_kernel<B, MX, 128>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 16: return launch_pdl(dequant_rot_kernel<B, FMT, 16>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 32: return launch_pdl(dequant_rot_kernel<B, FMT, 32>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 64: return launch_pdl(dequant_rot_kernel<B, FMT, 64>, dim3(g), dim3(ATHREADS), 0, st, a);
+    case 128: return launch_pdl(dequant_rot_kernel<B, FMT, 128>, dim3(g), dim3(ATHREADS), 0, st, a);
     default: return cudaErrorInvalidValue;
     }
 }
 
-cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a, cudaStream_t st)
+template <int FMT>
+static cudaError_t launch_dequant_rot_blocks(int block, int rot, const DequantArgs& a, cudaStream_t st)
+{
+    if (FMT == 1 && block != 32)
+        return cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_dequant_rot_b<4, FMT>(rot, a, st);
+    case 8: return launch_dequant_rot_b<8, FMT>(rot, a, st);
+    case 16: return launch_dequant_rot_b<16, FMT>(rot, a, st);
+    case 32: return launch_dequant_rot_b<32, FMT>(rot, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_dequant_rot(int fmt, int block, int rot, const DequantArgs& a, cudaStream_t st)
 {
     if (rot == 0)
-        return launch_dequant(mx, block, a, st);
-    if (mx)
-        return block == 32 ? launch_dequant_rot_b<32, true>(rot, a, st) : cudaErrorInvalidValue;
-    switch (block) {
-    case 4: return launch_dequant_rot_b<4, false>(rot, a, st);
-    case 8: return launch_dequant_rot_b<8, false>(rot, a, st);
-    case 16: return launch_dequant_rot_b<16, false>(rot, a, st);
-    case 32: return launch_dequant_rot_b<32, false>(rot, a, st);
+        return launch_dequant(fmt, block, a, st);
+    switch (fmt) {
+    case 0: return launch_dequant_rot_blocks<0>(block, rot, a, st);
+    case 1: return launch_dequant_rot_blocks<1>(block, rot, a, st);
+    case 2: return launch_dequant_rot_blocks<2>(block, rot, a, st);
     default: return cudaErrorInvalidValue;
     }
 }
@@ -339,7 +363,7 @@ cudaError_t launch_alpha(const float* sga, const float* sgb, float* alpha, cudaS
 
 // ------------------------------------------------------------ block MSE
 
-template <int B, int ROT, bool MX>
+template <int B, int ROT, int FMT>
 __global__ void __launch_bounds__(STHREADS) block_mse_kernel(MseArgs a)
 {
     pdl_begin();
@@ -352,7 +376,7 @@ __global__ void __launch_bounds__(STHREADS) block_mse_kernel(MseArgs a)
         return;
     float y[SPT][SEG];
     load_rotate<ROT>(a.x, a.n, t, lane, y);
-    const float sg = MX ? 1.0f : *a.sg;
+    const float sg = FMT == 0 ? *a.sg : 1.0f;
 #pragma unroll
     for (int k = 0; k < SPT; ++k) {
         const int64_t s = t * SPT + k;
@@ -363,7 +387,7 @@ __global__ void __launch_bounds__(STHREADS) block_mse_kernel(MseArgs a)
         load_codes(a.codes, s, nvalid, q);
         load_scale_bytes<NB>(a.scales, s, nvalid, B, sc);
         float S[NB], sse[NB], m[NB];
-        scales_of<NB, MX>(sc, sg, S);
+        scales_of<NB, FMT>(sc, sg, S);
         sse_seg<B>(y[k], q, S, sse);
 #pragma unroll
         for (int b = 0; b < NB; ++b)
@@ -372,35 +396,46 @@ __global__ void __launch_bounds__(STHREADS) block_mse_kernel(MseArgs a)
     }
 }
 
-template <int B, bool MX>
+template <int B, int FMT>
 static cudaError_t launch_mse_rot(int rot, unsigned g, const MseArgs& a, cudaStream_t st)
 {
     cudaError_t e_ = cudaSuccess;
     switch (rot) {
-    case 0: e_ = launch_pdl(block_mse_kernel<B, 0, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
-    case 16: e_ = launch_pdl(block_mse_kernel<B, 16, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
-    case 32: e_ = launch_pdl(block_mse_kernel<B, 32, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
-    case 64: e_ = launch_pdl(block_mse_kernel<B, 64, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
-    case 128: e_ = launch_pdl(block_mse_kernel<B, 128, MX>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 0: e_ = launch_pdl(block_mse_kernel<B, 0, FMT>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 16: e_ = launch_pdl(block_mse_kernel<B, 16, FMT>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 32: e_ = launch_pdl(block_mse_kernel<B, 32, FMT>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 64: e_ = launch_pdl(block_mse_kernel<B, 64, FMT>, dim3(g), dim3(STHREADS), 0, st, a); break;
+    case 128: e_ = launch_pdl(block_mse_kernel<B, 128, FMT>, dim3(g), dim3(STHREADS), 0, st, a); break;
     default: return cudaErrorInvalidValue;
     }
     return e_;
 }
 
-cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st)
+template <int FMT>
+static cudaError_t launch_mse_blocks(int block, int rot, unsigned g, const MseArgs& a, cudaStream_t st)
+{
+    if (FMT == 1 && block != 32)
+        return cudaErrorInvalidValue;
+    switch (block) {
+    case 4: return launch_mse_rot<4, FMT>(rot, g, a, st);
+    case 8: return launch_mse_rot<8, FMT>(rot, g, a, st);
+    case 16: return launch_mse_rot<16, FMT>(rot, g, a, st);
+    case 32: return launch_mse_rot<32, FMT>(rot, g, a, st);
+    default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_block_mse(int fmt, int block, int rot, const MseArgs& a, cudaStream_t st)
 {
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t nthr = nseg;
     if (!grid_ok(nthr, STHREADS))
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nthr, STHREADS);
-    if (mx)
-        return block == 32 ? launch_mse_rot<32, true>(rot, g, a, st) : cudaErrorInvalidValue;
-    switch (block) {
-    case 4: return launch_mse_rot<4, false>(rot, g, a, st);
-    case 8: return launch_mse_rot<8, false>(rot, g, a, st);
-    case 16: return launch_mse_rot<16, false>(rot, g, a, st);
-    case 32: return launch_mse_rot<32, false>(rot, g, a, st);
+    switch (fmt) {
+    case 0: return launch_mse_blocks<0>(block, rot, g, a, st);
+    case 1: return launch_mse_blocks<1>(block, rot, g, a, st);
+    case 2: return launch_mse_blocks<2>(block, rot, g, a, st);
     default: return cudaErrorInvalidValue;
     }
 }

@@ -212,6 +212,33 @@ __device__ __forceinline__ float e4m3_dec(uint32_t code)
     return h2_to_f2(h).x;
 }
 
+// ------------------------------------------------------------------ UE5M3
+
+// UE5M3 scale byte -> exact value: unsigned, 5 exponent bits with bias 15,
+// 3 mantissa bits, exponent field 0 subnormal (m * 2^-17); 0xFF is NaN.
+__device__ __forceinline__ float ue5m3_dec(uint32_t c)
+{
+    if (c >= 0xFFu)
+        return __uint_as_float(0x7FFFFFFFu);
+    if (c < 8u)
+        return __fmul_rn((float)c, 0x1p-17f);  // exact
+    return __uint_as_float((((c >> 3) + 112u) << 23) | ((c & 7u) << 20));
+}
+
+// v >= 0 -> the nearest UE5M3 byte, ties to the even code, saturating at
+// 0xFE. Below 2^-14 the step is 2^-17: v * 2^17 is exact and rounded to the
+// nearest even integer (8 is the first normal code). Above, the fp32
+// significand is rounded to 3 bits at bit 20 (ties to even, the carry moving
+// into the exponent), then re-biased from 127 to 15.
+__device__ __forceinline__ uint32_t ue5m3_enc(float v)
+{
+    const uint32_t b = __float_as_uint(v);
+    if (b < 0x38800000u)  // v < 2^-14
+        return (uint32_t)__float2int_rn(__fmul_rn(v, 0x1p17f));
+    const uint32_t r = (b + 0x7FFFFu + ((b >> 20) & 1u)) >> 20;
+    return min(r - (112u << 3), 0xFEu);
+}
+
 // ------------------------------------------------------------------ scales
 
 // FP32 global scale of hierarchical scaling: amax / (448 * 6); 1 when that is

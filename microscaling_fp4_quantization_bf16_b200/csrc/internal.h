@@ -32,7 +32,11 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // Strategy ids used by the kernels (NVFP4 strategies follow the ABI enum;
 // MXFP4 abs-max is its own kernel family).
 enum KStrat { K_ABSMAX = 0, K_PREVENT_ZERO = 1, K_FOUR_OVER_SIX = 2, K_BRUTE_FORCE = 3, K_MX = 4,
-              K_MX_BRUTE = 5 };
+              K_MX_BRUTE = 5,
+              // UE5M3 block scales (no global scale), the four strategies in order
+              K_UE_ABSMAX = 6, K_UE_PREVENT_ZERO = 7, K_UE_FOUR_OVER_SIX = 8, K_UE_BRUTE_FORCE = 9 };
+
+__host__ __device__ constexpr bool is_ue_strat(int s) { return s >= K_UE_ABSMAX && s <= K_UE_BRUTE_FORCE; }
 
 struct QuantArgs {
     const uint16_t* x;      // bf16 [n]
@@ -144,9 +148,10 @@ cudaError_t launch_quant_tma_b32(int strat, int rot, const QuantArgs& a, const C
 cudaError_t launch_amax(const uint16_t* x, int64_t n, int rot, unsigned* out, cudaStream_t st);
 cudaError_t launch_finalize_sg(float* g, cudaStream_t st);
 cudaError_t launch_set_one(float* p, cudaStream_t st);
-cudaError_t launch_dequant(int mx, int block, const DequantArgs& a, cudaStream_t st);
-cudaError_t launch_dequant_rot(int mx, int block, int rot, const DequantArgs& a, cudaStream_t st);
-cudaError_t launch_block_mse(int mx, int block, int rot, const MseArgs& a, cudaStream_t st);
+// fmt: 0 NVFP4, 1 MXFP4, 2 UE5M3 (the fp4q_format values).
+cudaError_t launch_dequant(int fmt, int block, const DequantArgs& a, cudaStream_t st);
+cudaError_t launch_dequant_rot(int fmt, int block, int rot, const DequantArgs& a, cudaStream_t st);
+cudaError_t launch_block_mse(int fmt, int block, int rot, const MseArgs& a, cudaStream_t st);
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_update(int sub, bool adam, const FocusUpdateArgs& a, cudaStream_t st);

@@ -13,6 +13,9 @@
 //   brute force  every code 0x01..0x7E, strictly lower SSE wins (ties keep
 //                the lower code)
 // MXFP4 ("Bridging the Gap ...", 技術概要 §1): S = 2^(floor(log2 amax) - 2).
+// UE5M3 scales (the wide-exponent format "Finer is Better ..." compares with
+// E4M3 + hierarchical scaling, 意義と主張): the same four strategies over the
+// codes of the unsigned 5-exponent / 3-mantissa format, with no global scale.
 #pragma once
 
 #include "fp4q_device.cuh"
@@ -28,19 +31,109 @@ namespace fp4q {
 constexpr int QTHREADS = 128;
 template <int STRAT>
 struct QMinBlocks {
-    static constexpr int value = STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE ? 1 : 7);
+    static constexpr int value =
+        STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE || STRAT == K_UE_BRUTE_FORCE ? 1 : 7);
 };
 
 // Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
 // dequantization scale S[c] = E4M3(c) * s_g and its reciprocal R[c] (the
 // zero-scale convention gives R[0] = 0) for every code c (index 0x7F unused),
-// and the scale-selection constants of s_g.
+// and the scale-selection constants of s_g. UE5M3 kernels: S[c] = UE5M3(c)
+// for c = 0..0xFE (index 0xFF unused).
+template <int STRAT>
+constexpr int scale_table_size()
+{
+    return STRAT == K_MX || STRAT == K_MX_BRUTE ? 1 : (is_ue_strat(STRAT) ? 256 : 128);
+}
+
 template <int STRAT>
 struct ScaleTables {
-    float S[STRAT == K_MX || STRAT == K_MX_BRUTE ? 1 : 128];
-    float R[STRAT == K_MX || STRAT == K_MX_BRUTE ? 1 : 128];
+    float S[scale_table_size<STRAT>()];
+    float R[scale_table_size<STRAT>()];
     NvConsts k;
 };
+
+// Exact search of one block's scale over the codes 1..MAXC of an increasing
+// code -> scale table (E4M3 under s_g, or UE5M3). The candidates from the
+// abs-max code c6 - 4 upward are evaluated in ascending order (strictly lower
+// SSE wins, so ties keep the lower code); from c6 + 5 on, every third code
+// checks block_zero_lb, and once it exceeds the best SSE no larger code can
+// win. Codes below c6 - 4 are skipped when saturation_lb at c6 - 5 exceeds the
+// best SSE, else searched as well (ties then go to the lower code). A
+// non-finite block maximum searches every code in order, as the definition
+// does.
+template <int B, int MAXC, class Tab>
+__device__ __forceinline__ void brute_search(const float* yb, float amax, int c6, const Tab& tab,
+                                             uint32_t keep, int& bc_out, float& best_out)
+{
+    const bool finite = amax <= FLT_MAX;
+    const int lo = finite ? max(1, c6 - 4) : 1;
+    float best = 0.0f;
+    int bc = lo;
+#pragma unroll 1
+    for (int c = lo; c <= MAXC; ++c) {
+        if (finite && c >= c6 + 5 && (c - c6 - 5) % 3 == 0 && block_zero_lb<B>(yb, tab.R[c]) > best)
+            break;
+        const float v = block_sse<B>(yb, tab.R[c], tab.S[c], keep);
+        if (c == lo || v < best) {
+            best = v;
+            bc = c;
+        }
+    }
+    if (lo > 1 && !(saturation_lb(amax, tab.R[lo - 1], tab.S[lo - 1]) > best)) {
+        float bl = 0.0f;
+        int cl = 1;
+#pragma unroll 1
+        for (int c = 1; c < lo; ++c) {
+            const float v = block_sse<B>(yb, tab.R[c], tab.S[c], keep);
+            if (c == 1 || v < bl) {
+                bl = v;
+                cl = c;
+            }
+        }
+        if (bl <= best) {
+            best = bl;
+            bc = cl;
+        }
+    }
+    bc_out = bc;
+    best_out = best;
+}
+
+// 4-over-6 choice for a whole segment: q, sc, S hold the target-6 result;
+// the target-4 candidate (c4, S4, r4, z4) is encoded, both block SSEs are
+// computed, and target 4 is kept only where its SSE is strictly lower.
+template <int B>
+__device__ __forceinline__ void choose_four_over_six(const float (&y)[SEG], uint32_t (&q)[4],
+                                                     uint32_t (&sc)[SEG / B], float (&S)[SEG / B],
+                                                     float (&sse)[SEG / B], const uint32_t (&c4)[SEG / B],
+                                                     const float (&S4)[SEG / B], const float (&r4)[SEG / B],
+                                                     const bool (&z4)[SEG / B], uint32_t keep)
+{
+    constexpr int NB = SEG / B;
+    float sse4[NB];
+    uint32_t q4w[4];
+    encode_seg<B, B == 32>(y, r4, z4, keep, q4w);
+    sse_seg<B>(y, q, S, sse);
+    sse_seg<B>(y, q4w, S4, sse4);
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        uint32_t m = 0;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (sse4[(8 * w + j) / B] < sse[(8 * w + j) / B])
+                m |= 0xFu << (4 * j);
+        q[w] = (q[w] & ~m) | (q4w[w] & m);
+    }
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+        if (sse4[b] < sse[b]) {
+            sc[b] = c4[b];
+            S[b] = S4[b];
+            sse[b] = sse4[b];
+        }
+    }
+}
 
 // Scale selection, encoding and stores for one 32-element segment s whose
 // (rotated) values are y. nvalid < 32 only for the last segment.
@@ -116,13 +209,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         encode_seg<B, true>(y, r, zero, a.keep, q);
         have_sse = true;
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
-        // Exact search with pruning. The candidates from the abs-max code c6 - 4
-        // upward are evaluated in ascending order (strictly lower SSE wins, so
-        // ties keep the lower code); from c6 + 5 on, every third code checks
-        // block_zero_lb, and once it exceeds the best SSE no larger code can win.
-        // Codes below c6 - 4 are skipped when saturation_lb at c6 - 5 exceeds the
-        // best SSE, else searched as well (ties then go to the lower code).
-        // Non-finite blocks search every code in order, as the definition does.
+        // Exact search with pruning (brute_search), from the abs-max code c6.
         const NvConsts k = tab.k;
         float qd[NB], qr[NB];
 #pragma unroll
@@ -134,38 +221,9 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         e4m3_quotient_codes<NB>(amax, qd, qr, k.fast, c6);
         static_for<NB>([&](auto bi) {
             constexpr int b = decltype(bi)::value;
-            const float* yb = y + b * B;
-            const bool finite = amax[b] <= FLT_MAX;
-            const int lo = finite ? max(1, (int)c6[b] - 4) : 1;
-            float best = 0.0f;
-            int bc = lo;
-#pragma unroll 1
-            for (int c = lo; c <= 0x7E; ++c) {
-                if (finite && c >= (int)c6[b] + 5 && (c - (int)c6[b] - 5) % 3 == 0 &&
-                    block_zero_lb<B>(yb, tab.R[c]) > best)
-                    break;
-                const float v = block_sse<B>(yb, tab.R[c], tab.S[c], a.keep);
-                if (c == lo || v < best) {
-                    best = v;
-                    bc = c;
-                }
-            }
-            if (lo > 1 && !(saturation_lb(amax[b], tab.R[lo - 1], tab.S[lo - 1]) > best)) {
-                float bl = 0.0f;
-                int cl = 1;
-#pragma unroll 1
-                for (int c = 1; c < lo; ++c) {
-                    const float v = block_sse<B>(yb, tab.R[c], tab.S[c], a.keep);
-                    if (c == 1 || v < bl) {
-                        bl = v;
-                        cl = c;
-                    }
-                }
-                if (bl <= best) {
-                    best = bl;
-                    bc = cl;
-                }
-            }
+            int bc;
+            float best;
+            brute_search<B, 0x7E>(y + b * B, amax[b], (int)c6[b], tab, a.keep, bc, best);
             sc[b] = (uint32_t)bc;
             S[b] = tab.S[bc];
             r[b] = tab.R[bc];
@@ -174,6 +232,55 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         });
         encode_seg<B>(y, r, zero, a.keep, q);
         have_sse = true;
+    } else if constexpr (is_ue_strat(STRAT)) {
+        // UE5M3 scales, no global scale: the candidate code of target T is
+        // RNE_UE5M3(amax / T) -- one IEEE division for T = 6; for T = 4 the
+        // product by 0.25 is the same correctly rounded quotient.
+        uint32_t c6[NB];
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            c6[b] = ue5m3_enc(__fdiv_rn(amax[b], 6.0f));
+        if constexpr (STRAT == K_UE_BRUTE_FORCE) {
+            static_for<NB>([&](auto bi) {
+                constexpr int b = decltype(bi)::value;
+                int bc;
+                float best;
+                brute_search<B, 0xFE>(y + b * B, amax[b], (int)c6[b], tab, a.keep, bc, best);
+                sc[b] = (uint32_t)bc;
+                S[b] = tab.S[bc];
+                r[b] = tab.R[bc];
+                zero[b] = (S[b] == 0.0f);
+                sse[b] = best;
+            });
+            encode_seg<B>(y, r, zero, a.keep, q);
+            have_sse = true;
+        } else {
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                uint32_t c = c6[b];
+                if constexpr (STRAT == K_UE_PREVENT_ZERO)
+                    c = max(c, 1u);
+                sc[b] = c;
+                S[b] = tab.S[c];
+                r[b] = tab.R[c];
+                zero[b] = (S[b] == 0.0f);
+            }
+            encode_seg<B, B == 32>(y, r, zero, a.keep, q);
+            if constexpr (STRAT == K_UE_FOUR_OVER_SIX) {
+                uint32_t c4[NB];
+                float S4[NB], r4[NB];
+                bool z4[NB];
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    c4[b] = ue5m3_enc(__fmul_rn(amax[b], 0.25f));
+                    S4[b] = tab.S[c4[b]];
+                    r4[b] = tab.R[c4[b]];
+                    z4[b] = (S4[b] == 0.0f);
+                }
+                choose_four_over_six<B>(y, q, sc, S, sse, c4, S4, r4, z4, a.keep);
+                have_sse = true;
+            }
+        }
     } else if constexpr (STRAT == K_FOUR_OVER_SIX && B <= 8) {
         // 4-over-6 for blocks of 4 or 8, one half segment (words w and w + 2)
         // at a time, so the candidates' temporaries of only half the blocks
@@ -267,9 +374,9 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         }
         encode_seg<B, B == 32>(y, r, zero, a.keep, q);  // packed measured faster for B = 32 only
         if constexpr (FOUR) {
-            float S4[NB], r4[NB], sse4[NB];
+            float S4[NB], r4[NB];
             bool z4[NB];
-            uint32_t c4[NB], q4w[4];
+            uint32_t c4[NB];
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
                 c4[b] = qc[NB + b];
@@ -277,26 +384,7 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
                 r4[b] = tab.R[c4[b]];
                 z4[b] = (S4[b] == 0.0f);
             }
-            encode_seg<B, B == 32>(y, r4, z4, a.keep, q4w);
-            sse_seg<B>(y, q, S, sse);
-            sse_seg<B>(y, q4w, S4, sse4);
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-                uint32_t m = 0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j)
-                    if (sse4[(8 * w + j) / B] < sse[(8 * w + j) / B])
-                        m |= 0xFu << (4 * j);
-                q[w] = (q[w] & ~m) | (q4w[w] & m);
-            }
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                if (sse4[b] < sse[b]) {
-                    sc[b] = c4[b];
-                    S[b] = S4[b];
-                    sse[b] = sse4[b];
-                }
-            }
+            choose_four_over_six<B>(y, q, sc, S, sse, c4, S4, r4, z4, a.keep);
             have_sse = true;
         }
     }
@@ -354,7 +442,14 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
 template <int STRAT>
 __device__ __forceinline__ void build_scale_tables(ScaleTables<STRAT>& tab, const QuantArgs& a)
 {
-    if constexpr (STRAT != K_MX && STRAT != K_MX_BRUTE) {
+    if constexpr (is_ue_strat(STRAT)) {
+        for (int c = threadIdx.x; c < 256; c += blockDim.x) {
+            const float S = (c <= 0xFE) ? ue5m3_dec((uint32_t)c) : 0.0f;
+            tab.S[c] = S;
+            tab.R[c] = (S == 0.0f) ? 0.0f : guarded_rcp(S);
+        }
+        __syncthreads();
+    } else if constexpr (STRAT != K_MX && STRAT != K_MX_BRUTE) {
         if (threadIdx.x < 128) {
             const float sg = global_scale_of(*a.amax);
             for (int c = threadIdx.x; c < 128; c += blockDim.x) {
@@ -421,6 +516,10 @@ cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream
     FP4Q_QROTS(K_PREVENT_ZERO)
     FP4Q_QROTS(K_FOUR_OVER_SIX)
     FP4Q_QROTS(K_BRUTE_FORCE)
+    FP4Q_QROTS(K_UE_ABSMAX)
+    FP4Q_QROTS(K_UE_PREVENT_ZERO)
+    FP4Q_QROTS(K_UE_FOUR_OVER_SIX)
+    FP4Q_QROTS(K_UE_BRUTE_FORCE)
     if constexpr (B == 32) {
         FP4Q_QROTS(K_MX)
         FP4Q_QROTS(K_MX_BRUTE)

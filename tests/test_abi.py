@@ -21,7 +21,7 @@ A = 0x100000     # a 16-byte-aligned fake device address
 A2 = 0x200000
 A3 = 0x300000
 MIS = 0x100004   # 4-byte but not 16-byte aligned
-NV, MX = 0, 1
+NV, MX, UE = 0, 1, 2
 
 
 @pytest.fixture(scope="module")
@@ -89,7 +89,11 @@ def test_quantize_validation(lib):
     assert q(lib, block=2) == UNSUP
     assert q(lib, rot=8) == UNSUP
     assert q(lib, strat=4) == UNSUP
-    assert q(lib, fmt=2) == UNSUP
+    assert q(lib, fmt=3) == UNSUP
+    assert q(lib, fmt=UE, block=64, gout=None) == UNSUP   # UE5M3: blocks 4..32
+    assert q(lib, fmt=UE, cols=24, gout=None) == SHAPE
+    assert q(lib, fmt=UE, strat=4, gout=None) == UNSUP
+    assert q(lib, fmt=UE, x=None, gout=None) == NULL       # no global scale needed, x is
     assert q(lib, dq=A, dqt=5) == UNSUP
     assert q(lib, gin=A3 + 64, gout=A3 + 64) == ALIAS
 
@@ -127,6 +131,7 @@ def test_other_entry_points_validation(lib):
     assert ff(w=MIS) == ALIGN
     assert ff(cols=40) == SHAPE
     assert ff(gin=A3, gout=A3) == ALIAS
+    assert ff(fmt=UE) == UNSUP      # FOCUS is defined for NVFP4 and MXFP4
     # focus backward
     assert L.fp4q_focus_bwd(A, A, A, 4, 60, 8, A, None) == SHAPE
     assert L.fp4q_focus_bwd(A, A, A, 4, 64, 6, A, None) == UNSUP
@@ -159,6 +164,7 @@ def test_other_entry_points_validation(lib):
     assert fs(gout=None) == NULL     # NVFP4 writes s_g
     assert fs(sse=MIS) == ALIGN
     assert fs(gin=A3, gout=A3) == ALIAS
+    assert fs(fmt=UE) == UNSUP
     # global amax, primitives
     assert L.fp4q_global_amax(A, 4, 64, 24, A, None) == UNSUP
     assert L.fp4q_global_amax(A, 4, 48, 32, A, None) == SHAPE
@@ -200,3 +206,6 @@ def test_gemm_validation(lib):
     assert qm(fmt=3) == UNSUP
     assert qm(sc=None) == NULL
     assert qm(sc=MIS) == ALIGN
+    assert qm(fmt=UE) == UNSUP       # the MMA takes E4M3 / E8M0 scales only
+    assert L.fp4q_mma_scale_bytes(128, 64, UE) == 0
+    assert L.fp4q_scales_to_mma(A, 128, 64, UE, A, None) == UNSUP

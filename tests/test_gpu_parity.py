@@ -120,7 +120,7 @@ def mixed(rows, cols, seed):
 
 # ------------------------------------------------------- all combinations
 
-COMBOS = [("nvfp4", b, s, r) for b in (4, 8, 16, 32)
+COMBOS = [(f, b, s, r) for f in ("nvfp4", "ue5m3") for b in (4, 8, 16, 32)
           for s in ("absmax", "prevent_zero", "four_over_six", "brute_force")
           for r in (0, 16, 32, 64, 128)] + [("mxfp4", 32, s, r) for s in ("absmax", "brute_force")
                                             for r in (0, 16, 32, 64, 128)]
@@ -191,6 +191,20 @@ def test_c3_full_strategy_sweep_sampled(gpu, block):
         compare_quant(g, o, "nvfp4", f"C3 B{block} {strat}")
 
 
+@pytest.mark.parametrize("block", [4, 16])
+def test_c3_full_ue5m3_sampled(gpu, block):
+    # UE5M3 scales have no global scale: every row is independent
+    x = synth.workload("c3_strategy_sweep_t3")["x"]
+    rows = sample_rows(x.shape[0], k=12, seed=100 + block)
+    xs = x[rows]
+    for strat in ("absmax", "prevent_zero", "four_over_six", "brute_force"):
+        g = gpu_quantize(gpu, x, "ue5m3", block, strat, 0)
+        o = oracle_quantize(xs, "ue5m3", block, strat, 0)
+        g = {"codes": g["codes"][rows], "scales": g["scales"][rows], "gs": None,
+             "mse": g["mse"][rows], "dq": None}
+        compare_quant(g, o, "ue5m3", f"C3 UE5M3 B{block} {strat}")
+
+
 @pytest.mark.parametrize("fmt,block", [("nvfp4", 16), ("mxfp4", 32)])
 def test_c4_full_focus(gpu, fmt, block):
     d = synth.workload("c4_focus")
@@ -256,7 +270,9 @@ def test_special_values(gpu, case):
     x = synth.to_bf16(a)
     for fmt, block, strat in [("nvfp4", 16, "absmax"), ("nvfp4", 16, "prevent_zero"),
                               ("nvfp4", 4, "four_over_six"), ("nvfp4", 8, "brute_force"),
-                              ("mxfp4", 32, "absmax")]:
+                              ("mxfp4", 32, "absmax"), ("ue5m3", 16, "absmax"),
+                              ("ue5m3", 4, "four_over_six"), ("ue5m3", 8, "brute_force"),
+                              ("ue5m3", 32, "prevent_zero")]:
         rots = (0,) if case == "huge" else (0, 16, 128)
         for rot in rots:
             for ga in (None, 2688.0, 1e-30, 0.0, -1.0, float("inf")) if fmt == "nvfp4" else (None,):
@@ -268,7 +284,7 @@ def test_special_values(gpu, case):
 # ------------------------------------------------------ dequant, block MSE
 
 @pytest.mark.parametrize("fmt,block", [("nvfp4", 4), ("nvfp4", 8), ("nvfp4", 16), ("nvfp4", 32),
-                                       ("mxfp4", 32)])
+                                       ("mxfp4", 32), ("ue5m3", 4), ("ue5m3", 16), ("ue5m3", 32)])
 def test_dequantize_and_block_mse_any_bytes(gpu, fmt, block):
     rng = np.random.default_rng(block)
     rows, cols = 7, 8 * block if block >= 8 else 36  # 7*36 = 252: ragged last segment
@@ -303,7 +319,7 @@ def test_dequantize_and_block_mse_any_bytes(gpu, fmt, block):
 
 
 @pytest.mark.parametrize("fmt,block", [("nvfp4", 4), ("nvfp4", 8), ("nvfp4", 16), ("nvfp4", 32),
-                                       ("mxfp4", 32)])
+                                       ("mxfp4", 32), ("ue5m3", 8), ("ue5m3", 32)])
 @pytest.mark.parametrize("rot", [16, 32, 64, 128])
 def test_dequantize_unrotate(gpu, fmt, block, rot):
     """Dequantization back to the original domain (the normalised rotation
@@ -317,8 +333,8 @@ def test_dequantize_unrotate(gpu, fmt, block, rot):
     raw_codes = rng.integers(0, 256, size=(rows, cols // 2), dtype=np.uint8)
     # scale bytes whose values stay finite through the butterflies (an infinity
     # would turn into NaN, whose bit pattern is not part of the contract)
-    raw_scales = rng.integers(0, 127 if fmt == "nvfp4" else 201, size=(rows, cols // block),
-                              dtype=np.uint8)
+    raw_scales = rng.integers(0, {"nvfp4": 127, "mxfp4": 201, "ue5m3": 255}[fmt],
+                              size=(rows, cols // block), dtype=np.uint8)
     for codes, scales, sg, what in ((q["codes"], q["scales"], q["gs"], "quantized"),
                                     (raw_codes, raw_scales, np.float32(3.1e-3), "raw bytes")):
         gs = torch.tensor([sg], device="cuda") if fmt == "nvfp4" else None
