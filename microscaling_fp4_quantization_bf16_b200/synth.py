@@ -75,6 +75,29 @@ def focus_coeffs(rows: int, cols: int, sub: int, seed: int, lo: float = 0.9,
     return to_fp16(rng.uniform(lo, hi, size=(rows, cols // sub)))
 
 
+def gptq_problem(rows: int, cols: int, tokens: int, seed: int, damp: float = 0.01,
+                 act_order: bool = True) -> dict:
+    """Inputs of the GPTQ error-feedback step for one synthetic linear layer:
+    W ~ N(0, 0.02^2) bf16 [rows, cols]; calibration inputs X [tokens, cols] with
+    per-channel scales U[0.1, 2.1], 1% of the channels x20 and a random mixing
+    (I + 0.3 N(0,1)/sqrt(cols)) so that channels correlate; the damped Hessian
+    H = X^T X / tokens + damp * mean(diag) * I; the processing order (columns by
+    decreasing diag(H) when act_order, else the identity); and the upper
+    Cholesky factor U of H^-1 in that order, all computed in float64 and
+    handed over as fp32 / int32 (the caller's preparation)."""
+    rng = np.random.default_rng(seed)
+    w = gaussian(rows, cols, seed=seed + 1, std=0.02)
+    x = rng.standard_normal((tokens, cols)) * rng.uniform(0.1, 2.1, cols)
+    x[:, rng.choice(cols, max(1, cols // 100), replace=False)] *= 20
+    x = x @ (np.eye(cols) + 0.3 * rng.standard_normal((cols, cols)) / np.sqrt(cols))
+    h = x.T @ x / tokens
+    h += damp * float(np.mean(np.diag(h))) * np.eye(cols)
+    perm = np.argsort(-np.diag(h), kind="stable") if act_order else np.arange(cols)
+    hp = h[np.ix_(perm, perm)]
+    u = np.linalg.cholesky(np.linalg.inv(hp)).T     # upper: H^-1 = U^T U
+    return {"w": w, "h": h, "perm": perm.astype(np.int32), "u": np.ascontiguousarray(u, np.float32)}
+
+
 def workload(name: str, rows: int | None = None, cols: int | None = None) -> dict:
     """Tensors of one named workload; rows/cols override the full size (same
     distribution and seeds, smaller shape)."""

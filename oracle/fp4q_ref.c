@@ -74,6 +74,16 @@
  *      needs no hierarchical scaling, so s_g = 1: candidate code =
  *      RNE_UE5M3_sat(amax / T); the four strategies as for E4M3, brute force
  *      over codes 0x01..0xFE.
+ *  R18 MR-GPTQ ([BRIDGE] 技術概要 §2.2 lists its parts without formulas):
+ *      GPTQ error feedback over the upper Cholesky factor U of the inverse
+ *      (damped) Hessian, with static groups -- block scales fixed beforehand
+ *      from the original weights by any scale strategy (the MSE-optimised
+ *      grid is the brute force / MSE grid) -- and static activation
+ *      reordering as a processing order of the columns (codes stay in the
+ *      original order). Lazy batch updates over 128 positions; within a
+ *      batch each update is one fma, the trailing update one fma-chain sum
+ *      per element followed by one subtraction. The rotation part is not
+ *      in this step: it takes the bf16 weights as stored.
  *  R15 FOCUS calibration: the pages learn c by gradient descent through the
  *      STE but name neither the optimizer nor the precision of the update.
  *      The learnable state is an fp32 master copy of c; the forward uses its
@@ -763,6 +773,79 @@ int ref_fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_sg, co
     }
     free(av);
     free(bv);
+    return REF_OK;
+}
+
+/* GPTQ error feedback with static groups ([BRIDGE] 技術概要 §2.2: MR-GPTQ =
+ * GPTQ with the MSE-optimised grid, static activation reordering and
+ * rotations), reading R18. The block scales are fixed beforehand (static
+ * groups: scales[rows, K/block] from ref_quantize of the original weights,
+ * any strategy; s_g for NVFP4). The columns are processed in the order perm
+ * (processing position j -> original column perm[j]; NULL = identity) with U
+ * the upper Cholesky factor of the inverse Hessian in that order (fp32
+ * [K, K] row-major). Per row, in blocks of 128 positions (K % 128 == 0):
+ *   for each position j of the block: S = scale of the block holding column
+ *     perm[j]; q = RNE_E2M1(w_j * (1/S)) (code 0 if S == 0); the error
+ *     e_j = (w_j - value(q) * S) / U[j][j]; the later positions k of the
+ *     block take w_k = fma(-e_j, U[j][k], w_k), j ascending;
+ *   then every position k after the block: t = fma sum of e_j * U[j][k] over
+ *     the block's j ascending from t = 0, and w_k = w_k - t.
+ * Codes are written at the original column (packed as in R8). Rows are
+ * independent. */
+int ref_gptq(const uint16_t* w, int64_t rows, int64_t K, int fmt, int block,
+             const uint8_t* scales, float sg, const float* U, const int32_t* perm,
+             uint8_t* codes)
+{
+    if (!valid_common(rows, K, fmt, block, 0) || K % 128 != 0)
+        return REF_ERR_ARG;
+    if (perm) {
+        uint8_t* seen = (uint8_t*)calloc((size_t)K, 1);
+        int ok = 1;
+        for (int64_t j = 0; j < K && ok; j++) {
+            if (perm[j] < 0 || perm[j] >= K || seen[perm[j]])
+                ok = 0;
+            else
+                seen[perm[j]] = 1;
+        }
+        free(seen);
+        if (!ok)
+            return REF_ERR_ARG;
+    }
+    float* W = (float*)malloc(sizeof(float) * (size_t)K);
+    float E[128];
+    int64_t nb = K / block;
+    memset(codes, 0, (size_t)(rows * K / 2));
+    for (int64_t i = 0; i < rows; i++) {
+        for (int64_t j = 0; j < K; j++)
+            W[j] = ref_bf16_to_float(w[i * K + (perm ? perm[j] : j)]);
+        for (int64_t b0 = 0; b0 < K; b0 += 128) {
+            for (int jj = 0; jj < 128; jj++) {
+                int64_t j = b0 + jj;
+                int64_t col = perm ? perm[j] : j;
+                float S = block_scale(fmt, scales[i * nb + col / block], sg);
+                int q = 0;
+                float deq = 0.0f;
+                if (S != 0.0f) {
+                    float u = W[j] * guarded_reciprocal(S);
+                    q = ref_rne_e2m1(u);
+                    deq = (float)ref_e2m1_value(q) * S;
+                }
+                float d = W[j] - deq;
+                E[jj] = d / U[j * K + j];
+                int64_t t = i * K + col;
+                codes[t / 2] = (uint8_t)(codes[t / 2] | (q << (4 * (t & 1))));
+                for (int kk = jj + 1; kk < 128; kk++)
+                    W[b0 + kk] = fmaf(-E[jj], U[j * K + b0 + kk], W[b0 + kk]);
+            }
+            for (int64_t k = b0 + 128; k < K; k++) {
+                float t = 0.0f;
+                for (int jj = 0; jj < 128; jj++)
+                    t = fmaf(E[jj], U[(b0 + jj) * K + k], t);
+                W[k] = W[k] - t;
+            }
+        }
+    }
+    free(W);
     return REF_OK;
 }
 
