@@ -516,6 +516,28 @@ def breakdown(dev, peaks, reps: int = 10):
                              "launches": 2 + (3 if fmt == "nvfp4" else 1)})
             del a, w, qa, qw, sa, sw, dout, qa2, qw2
     torch.cuda.empty_cache()
+    # GPTQ error feedback with static groups (MR-GPTQ) on a 4096 x 4096 layer:
+    # NVFP4 B16 MSE-optimal static scales, activation order; 32 batches of
+    # 128 positions (sequential batch kernel + fp32 fma trailing update).
+    # Roofline: the trailing updates' fma work against the FP32 FMA peak
+    # (148 SMs x 128 lanes x 2 flops x 1.965 GHz).
+    gd = synth.gptq_problem(4096, 4096, 4096, seed=11)
+    gw = gd["w"].to(dev)
+    gqs = fp4q.quantize(gw, "nvfp4", 16, "brute_force", 0)
+    gU = torch.from_numpy(gd["u"]).to(dev)
+    gperm = torch.from_numpy(gd["perm"]).to(dev)
+    gwork = torch.empty(4096, 4096, device=dev)
+    gout = torch.empty(4096, 2048, dtype=torch.uint8, device=dev)
+    gsecs = timeit([lambda: fp4q.gptq(gw, gqs.scales, gqs.global_scale, gU, gperm, "nvfp4", 16,
+                                      work=gwork, out=gout)])
+    gflops = 2.0 * 4096 * 128 * sum(4096 - b0 - 128 for b0 in range(0, 4096, 128))
+    fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
+    rows_out.append({"run": "gptq error feedback nvfp4 B16 4096x4096 (static MSE-optimal scales, act order)",
+                     "us": round(gsecs * 1e6, 1), "tflops": round(gflops / gsecs / 1e12, 2),
+                     "bound": "fp32 fma", "fma_frac": round(gflops / gsecs / 1e12 / fma_peak, 4),
+                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 2 * 32 - 1})
+    del gd, gw, gqs, gU, gperm, gwork, gout
+    torch.cuda.empty_cache()
     # FOCUS
     d = synth.workload("c4_focus")
     w0, c0, g0 = d["w"].to(dev), d["c"].to(dev), d["g"].to(dev)

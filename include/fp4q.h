@@ -328,6 +328,37 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
                             int64_t t, cudaStream_t stream);
 
 /*
+ * fp4q_gptq -- GPTQ error feedback with static groups: the error-feedback part
+ * of MR-GPTQ ("Bridging the Gap Between Promise and Performance for
+ * Microscaling FP4 Quantization", 技術概要 §2.2: GPTQ with the MSE-optimised
+ * grid, static activation reordering and rotations).
+ * The block scales are fixed beforehand (static groups: `scales` and
+ * `global_scale` as fp4q_quantize wrote them for the original weights, any
+ * strategy -- FP4Q_BRUTE_FORCE is the MSE-optimised grid). The columns are
+ * processed in the order perm (static activation reordering) against U, the
+ * upper Cholesky factor of the inverse (damped) Hessian taken in that order
+ * (H^-1 = U^T U); the codes are written in the original column order.
+ * Per row, in batches of 128 positions: for each position j, q = E2M1 code
+ * of w_j / S (code 0 where S == 0), e_j = (w_j - value(q) * S) / U[j][j],
+ * and the later positions k of the batch take w_k = fma(-e_j, U[j][k], w_k);
+ * after the batch every later column takes w_k -= (fma chain over the batch,
+ * j ascending, of e_j * U[j][k]). All fp32, one rounding per operation.
+ * w         bf16 [rows, cols], cols a multiple of 128.
+ * fmt, block, scales [rows, cols/block], global_scale (NVFP4 s_g, device):
+ *           the static block scales; any format.
+ * U         fp32 [cols, cols] row-major (only the upper triangle is read).
+ * perm      int32 [cols]: processing position -> original column, a
+ *           permutation (entries outside 0..cols-1 are counted by
+ *           fp4q_device_errors and read column 0); NULL = natural order.
+ * work      fp32 [rows, cols] caller scratch (overwritten).
+ * codes     uint8 [rows, cols/2] (zeroed, then written).
+ * Launches: 1 memset + 1 + 2 * cols/128 - 1 kernels. Rows are independent.
+ */
+fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                      const uint8_t* scales, const float* global_scale, const float* U,
+                      const int32_t* perm, float* work, uint8_t* codes, cudaStream_t stream);
+
+/*
  * fp4q_global_amax -- abs-max of the (rotated) tensor into *amax_out (device
  * float): the per-tensor statistic of hierarchical scaling ("Finer is Better
  * (with the Right Scaling)", 手法 2). Feed it to global_amax_in of the calls

@@ -626,6 +626,45 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
     return st;
 }
 
+fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
+                      const uint8_t* scales, const float* global_scale, const float* U,
+                      const int32_t* perm, float* work, uint8_t* codes, cudaStream_t stream)
+{
+    fp4q_status st = check_format(rows, cols, fmt, block, 0);
+    if (st != FP4Q_OK)
+        return st;
+    if (cols % 128 != 0 || rows > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t n = rows * cols;
+    if (n == 0)
+        return FP4Q_OK;
+    if (w == nullptr || scales == nullptr || U == nullptr || work == nullptr || codes == nullptr ||
+        (nv && global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(w) || !aligned16(scales) || !aligned16(U) || !aligned16(perm) ||
+        !aligned16(work) || !aligned16(codes) || (nv && !aligned4(global_scale)))
+        return FP4Q_ERR_ALIGN;
+    GptqArgs a;
+    a.w = static_cast<const uint16_t*>(w);
+    a.scales = scales;
+    a.sg = nv ? global_scale : nullptr;
+    a.U = U;
+    a.perm = perm;
+    a.work = work;
+    a.codes = codes;
+    a.rows = rows;
+    a.K = cols;
+    a.fmt = (int)fmt;
+    a.block = block;
+    cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fp4q_device_errors);
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(codes, 0, (size_t)(n / 2), stream);
+    if (e == cudaSuccess)
+        e = launch_gptq(a, stream);
+    return cuda_status(e);
+}
+
 fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot, float* amax_out,
                              cudaStream_t stream)
 {

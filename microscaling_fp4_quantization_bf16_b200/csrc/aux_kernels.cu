@@ -25,14 +25,6 @@ static inline bool grid_ok(int64_t nseg, int threads = ATHREADS)
     return nblk > 0 && nblk <= 0x7FFFFFFF;
 }
 
-// E8M0 byte -> 2^(b - 127); 255 is NaN; byte 0 is the subnormal 2^-127.
-__device__ __forceinline__ float e8m0_dec(uint32_t b)
-{
-    if (b == 255u)
-        return __uint_as_float(0x7FC00000u);
-    return b == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
-}
-
 // ------------------------------------------------------------ global abs-max
 
 // Tensor abs-max of the (rotated) tensor, combined across blocks with an

@@ -219,7 +219,7 @@ __device__ __forceinline__ float e4m3_dec(uint32_t code)
 __device__ __forceinline__ float ue5m3_dec(uint32_t c)
 {
     if (c >= 0xFFu)
-        return __uint_as_float(0x7FFFFFFFu);
+        return __uint_as_float(0x7FC00000u);
     if (c < 8u)
         return __fmul_rn((float)c, 0x1p-17f);  // exact
     return __uint_as_float((((c >> 3) + 112u) << 23) | ((c & 7u) << 20));
@@ -268,6 +268,14 @@ __device__ __forceinline__ int e8m0_exp(float a)
 {
     int E = (int)((__float_as_uint(a) >> 23) & 0xFFu);
     return max(E - 129, -127);
+}
+
+// E8M0 byte -> 2^(b - 127); 255 is NaN; byte 0 is the subnormal 2^-127.
+__device__ __forceinline__ float e8m0_dec(uint32_t b)
+{
+    if (b == 255u)
+        return __uint_as_float(0x7FC00000u);
+    return b == 0u ? __uint_as_float(0x00400000u) : __uint_as_float(b << 23);
 }
 
 // Per-thread constants of E4M3 scale selection for target T in {6, 4}:

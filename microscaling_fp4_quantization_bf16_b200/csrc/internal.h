@@ -125,6 +125,20 @@ struct FocusStepArgs {
     OptConsts o;
 };
 
+// GPTQ error feedback with static groups (gptq.cu).
+struct GptqArgs {
+    const uint16_t* w;      // bf16 [rows, K], original column order
+    const uint8_t* scales;  // [rows, K / block] fixed block scales
+    const float* sg;        // NVFP4 s_g (device), else unused
+    const float* U;         // fp32 [K, K] upper Cholesky factor of H^-1, processing order
+    const int32_t* perm;    // [K] processing position -> column, or NULL
+    float* work;            // fp32 [rows, K] scratch
+    uint8_t* codes;         // [rows, K / 2], zeroed by the caller
+    unsigned* err;          // device error counter
+    int64_t rows, K;
+    int fmt, block;         // fmt: 0 NVFP4, 1 MXFP4, 2 UE5M3
+};
+
 // Each launcher returns cudaErrorInvalidValue for a combination it does not
 // provide (the ABI layer validates before calling), else the launch status.
 cudaError_t launch_quant_b4(int strat, int rot, const QuantArgs& a, cudaStream_t st);
@@ -155,6 +169,7 @@ cudaError_t launch_block_mse(int fmt, int block, int rot, const MseArgs& a, cuda
 cudaError_t launch_focus_fwd(int mx, int block, int sub, const FocusFwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_bwd(int sub, const FocusBwdArgs& a, cudaStream_t st);
 cudaError_t launch_focus_update(int sub, bool adam, const FocusUpdateArgs& a, cudaStream_t st);
+cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st);
 cudaError_t launch_focus_step(int mx, int block, int sub, bool adam, const FocusStepArgs& a,
                               cudaStream_t st);
 // W4A4 FP4 GEMM (gemm_*.cu): scale layout for the block-scaled MMA and the

@@ -165,6 +165,17 @@ def test_other_entry_points_validation(lib):
     assert fs(sse=MIS) == ALIGN
     assert fs(gin=A3, gout=A3) == ALIAS
     assert fs(fmt=UE) == UNSUP
+    # GPTQ error feedback
+    gq = lambda **k: L.fp4q_gptq(k.get("w", A), 4, k.get("cols", 256), k.get("fmt", NV),
+                                 k.get("block", 16), A, k.get("gs", A2), A3, k.get("perm"),
+                                 k.get("work", A), k.get("codes", A2), None)
+    assert gq(cols=192) == SHAPE      # cols % 128
+    assert gq(cols=200) == SHAPE      # cols % block
+    assert gq(block=64) == UNSUP
+    assert gq(gs=None) == NULL        # NVFP4 needs s_g
+    assert gq(work=None) == NULL
+    assert gq(perm=MIS) == ALIGN
+    assert gq(codes=MIS) == ALIGN
     # global amax, primitives
     assert L.fp4q_global_amax(A, 4, 64, 24, A, None) == UNSUP
     assert L.fp4q_global_amax(A, 4, 48, 32, A, None) == SHAPE
