@@ -31,10 +31,10 @@ namespace fp4q {
 namespace {
 
 constexpr int GB = 128;           // positions per batch
-constexpr int ROWS_PER_CTA = 8;   // batch kernel: one warp per row
-constexpr int TT = 64;            // trailing kernel: 64 x 64 output tile
-constexpr int TTHREADS = 256;     // 16 x 16 threads, 4 x 4 outputs each
-constexpr int EL = GB + 1;        // row stride of the error tile (no bank conflicts)
+constexpr int ROWS_PER_CTA = 16;  // batch kernel: one warp per row (4096 rows: one wave)
+constexpr int TR = 128;           // trailing kernel: 128 rows x 64 columns per CTA
+constexpr int TC = 64;
+constexpr int TTHREADS = 256;     // 16 x 16 threads, 8 x 4 outputs each
 
 __device__ __forceinline__ int64_t column_of(const GptqArgs& a, int64_t j)
 {
@@ -133,48 +133,58 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs 
 }
 
 // work[i][k] -= sum over the batch of e[i][j] * U[b0 + j][k] for k >= b0 + GB,
-// each sum an fma chain in j order from 0.
+// each sum an fma chain in j order from 0. A 128 x 64 output tile per CTA
+// (96 KB of shared memory: two CTAs per SM); each thread accumulates 8 x 4
+// outputs (rows 4ty..4ty+3 and 64+4ty.., columns 4tx..4tx+3) from three
+// 128-bit shared loads per j.
 __global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int64_t b0)
 {
     extern __shared__ float sm[];
-    float* ut = sm;             // [GB][TT]: ut[j][c] = U[b0 + j][k0 + c]
-    float* es = sm + GB * TT;   // [TT][EL]: es[r][j] = e of row r0 + r at position j
+    float* es = sm;             // [GB][TR]: es[j][r] = e of row r0 + r at position j
+    float* ut = sm + GB * TR;   // [GB][TC]: ut[j][c] = U[b0 + j][k0 + c]
     pdl_begin();
-    const int64_t r0 = (int64_t)blockIdx.y * TT;
-    const int64_t k0 = b0 + GB + (int64_t)blockIdx.x * TT;
-    for (int e = threadIdx.x; e < GB * TT; e += TTHREADS) {
-        const int r = e / GB, j = e - r * GB;  // coalesced along j in work
+    const int64_t r0 = (int64_t)blockIdx.y * TR;
+    const int64_t k0 = b0 + GB + (int64_t)blockIdx.x * TC;
+    for (int e = threadIdx.x; e < TR * GB / 4; e += TTHREADS) {
+        const int r = e % TR, j4 = e / TR;  // consecutive threads: consecutive rows
         const int64_t row = r0 + r;
-        es[r * EL + j] = row < a.rows ? a.work[row * a.K + b0 + j] : 0.0f;
+        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (row < a.rows)
+            v = *reinterpret_cast<const float4*>(a.work + row * a.K + b0 + 4 * j4);
+        es[(4 * j4) * TR + r] = v.x;
+        es[(4 * j4 + 1) * TR + r] = v.y;
+        es[(4 * j4 + 2) * TR + r] = v.z;
+        es[(4 * j4 + 3) * TR + r] = v.w;
     }
-    for (int e = threadIdx.x; e < GB * TT / 4; e += TTHREADS) {
-        const int j = e / (TT / 4), c4 = e - j * (TT / 4);
+    for (int e = threadIdx.x; e < GB * TC / 4; e += TTHREADS) {
+        const int j = e / (TC / 4), c4 = e - j * (TC / 4);
         reinterpret_cast<float4*>(ut)[e] =
             *reinterpret_cast<const float4*>(a.U + (b0 + j) * a.K + k0 + 4 * c4);
     }
     __syncthreads();
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[4][4];
+    float acc[8][4];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
             acc[r][c] = 0.0f;
 #pragma unroll 4
     for (int j = 0; j < GB; ++j) {
-        const float4 uv = reinterpret_cast<const float4*>(ut + j * TT)[tx];
-        const float er[4] = {es[(4 * ty) * EL + j], es[(4 * ty + 1) * EL + j],
-                             es[(4 * ty + 2) * EL + j], es[(4 * ty + 3) * EL + j]};
-        const float uc[4] = {uv.x, uv.y, uv.z, uv.w};
+        const float4 e0 = reinterpret_cast<const float4*>(es + j * TR)[ty];
+        const float4 e1 = reinterpret_cast<const float4*>(es + j * TR + TR / 2)[ty];
+        const float4 u0 = reinterpret_cast<const float4*>(ut + j * TC)[tx];
+        const float er[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+        const float uc[4] = {u0.x, u0.y, u0.z, u0.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int r = 0; r < 8; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
                 acc[r][c] = __fmaf_rn(er[r], uc[c], acc[r][c]);
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int64_t row = r0 + 4 * ty + r;
+    for (int r = 0; r < 8; ++r) {
+        const int64_t row = r0 + (r < 4 ? 4 * ty + r : TR / 2 + 4 * ty + r - 4);
         if (row >= a.rows)
             continue;
         float4* p = reinterpret_cast<float4*>(a.work + row * a.K + k0 + 4 * tx);
@@ -191,10 +201,10 @@ __global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int
 
 cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
 {
-    if (a.K % GB != 0 || a.rows <= 0 || (a.rows + TT - 1) / TT > 65535 || a.rows * a.K > ((int64_t)1 << 40))
+    if (a.K % GB != 0 || a.rows <= 0 || (a.rows + TR - 1) / TR > 65535 || a.rows * a.K > ((int64_t)1 << 40))
         return cudaErrorInvalidValue;
     const size_t batch_smem = sizeof(float) * GB * GB;
-    const size_t trail_smem = sizeof(float) * (GB * TT + TT * EL);
+    const size_t trail_smem = sizeof(float) * GB * (TR + TC);
     cudaError_t e = cudaFuncSetAttribute(gptq_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)batch_smem);
     if (e == cudaSuccess)
@@ -205,12 +215,12 @@ cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
     const int64_t n = a.rows * a.K;
     e = launch_pdl(gptq_gather_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a);
     const unsigned row_ctas = (unsigned)((a.rows + ROWS_PER_CTA - 1) / ROWS_PER_CTA);
-    const unsigned row_tiles = (unsigned)((a.rows + TT - 1) / TT);
+    const unsigned row_tiles = (unsigned)((a.rows + TR - 1) / TR);
     for (int64_t b0 = 0; b0 < a.K && e == cudaSuccess; b0 += GB) {
         e = launch_pdl(gptq_batch_kernel, dim3(row_ctas), dim3(ROWS_PER_CTA * 32), batch_smem, st, a, b0);
         const int64_t rest = a.K - b0 - GB;
         if (e == cudaSuccess && rest > 0)
-            e = launch_pdl(gptq_trailing_kernel, dim3((unsigned)(rest / TT), row_tiles), dim3(TTHREADS),
+            e = launch_pdl(gptq_trailing_kernel, dim3((unsigned)(rest / TC), row_tiles), dim3(TTHREADS),
                            trail_smem, st, a, b0);
     }
     return e;
