@@ -297,7 +297,8 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
  *          (start at zero); ignored (may be NULL) for SGD.
  * t        Adam's step number, >= 1. b1, b2, eps are ignored for SGD.
  * An unknown opt, or Adam with t < 1, returns FP4Q_ERR_UNSUPPORTED; Adam with
- * m or v NULL returns FP4Q_ERR_NULL. c, c_half, m, v must not overlap w or g.
+ * m or v NULL (with rows * cols > 0) returns FP4Q_ERR_NULL. c, c_half, m, v must not
+ * overlap w or g.
  * Nothing keeps c positive: a coefficient driven to zero or below gives
  * unspecified codes in the next forward pass.
  */

@@ -516,13 +516,14 @@ OptConsts opt_consts(fp4q_optimizer opt, float lr, float b1, float b2, float eps
     return o;
 }
 
-fp4q_status check_opt(fp4q_optimizer opt, int64_t t, const float* m, const float* v)
+// Optimizer arguments; Adam's moments are required only when there is work.
+fp4q_status check_opt(fp4q_optimizer opt, int64_t t, const float* m, const float* v, int64_t n)
 {
     if (opt != FP4Q_OPT_SGD && opt != FP4Q_OPT_ADAM)
         return FP4Q_ERR_UNSUPPORTED;
     if (opt == FP4Q_OPT_ADAM && t < 1)
         return FP4Q_ERR_UNSUPPORTED;
-    if (opt == FP4Q_OPT_ADAM && (m == nullptr || v == nullptr))
+    if (n > 0 && opt == FP4Q_OPT_ADAM && (m == nullptr || v == nullptr))
         return FP4Q_ERR_NULL;
     return FP4Q_OK;
 }
@@ -538,10 +539,10 @@ fp4q_status fp4q_focus_update(const void* w, const void* g, float* c, void* c_ha
         return FP4Q_ERR_UNSUPPORTED;
     if (rows < 0 || cols < 0 || cols % sub != 0 || (cols > 0 && rows > kMaxElems / cols))
         return FP4Q_ERR_SHAPE;
-    fp4q_status st = check_opt(opt, t, m, v);
+    const int64_t n = rows * cols;
+    fp4q_status st = check_opt(opt, t, m, v, n);
     if (st != FP4Q_OK)
         return st;
-    const int64_t n = rows * cols;
     if (n == 0)
         return FP4Q_OK;
     if (w == nullptr || g == nullptr || c == nullptr)
@@ -575,11 +576,11 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
         return FP4Q_ERR_UNSUPPORTED;  // FOCUS is defined for MXFP4 and NVFP4
     if (!valid_sub(sub) || sub > block)
         return FP4Q_ERR_UNSUPPORTED;
-    st = check_opt(opt, t, m, v);
-    if (st != FP4Q_OK)
-        return st;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
     const int64_t n = rows * cols;
+    st = check_opt(opt, t, m, v, n);
+    if (st != FP4Q_OK)
+        return st;
     if (nv && global_scale_out == nullptr)
         return FP4Q_ERR_NULL;
     if (n > 0 && (w == nullptr || c == nullptr))

@@ -228,3 +228,25 @@ def test_layer_objective_loop(gpu):
         assert_exact(u16(state.c_half.cpu()), o["c_half"], f"layer loop c_half t{t}")
         assert_exact(state.m.cpu().numpy(), om, f"layer loop m t{t}")
     assert losses[-1] < losses[0]
+
+
+def test_empty_inputs(gpu):
+    """rows == 0: every new entry point returns without launching; NVFP4 still
+    publishes s_g = 1 for the fused step, as the forward does."""
+    L = gpu._abi.load()
+    w = torch.empty(0, 64, dtype=torch.bfloat16, device="cuda")
+    c = torch.empty(0, 8, dtype=torch.float32, device="cuda")
+    gs = torch.full((1,), -3.0, device="cuda")
+    assert L.fp4q_focus_update(w.data_ptr(), w.data_ptr(), c.data_ptr(), None, c.data_ptr(),
+                               c.data_ptr(), 0, 64, 8, 1, 1e-3, 0.9, 0.999, 1e-8, 1, None) == 0
+    assert L.fp4q_focus_step(w.data_ptr(), 0, 64, 0, 16, 8, None, gs.data_ptr(), c.data_ptr(), None,
+                             c.data_ptr(), c.data_ptr(), None, 1, 1e-3, 0.9, 0.999, 1e-8, 1,
+                             None) == 0
+    torch.cuda.synchronize()
+    assert gs.item() == 1.0
+    u = torch.eye(128, device="cuda")
+    assert L.fp4q_gptq(w.data_ptr(), 0, 128, 1, 32, c.data_ptr(), None, u.data_ptr(), None,
+                       c.data_ptr(), c.data_ptr(), None) == 0
+    q = gpu.quantize(w, "ue5m3", 16, "four_over_six")
+    torch.cuda.synchronize()
+    assert q.codes.numel() == 0 and q.global_scale is None
