@@ -65,10 +65,16 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
+# The sources the headline quantize kernel is compiled from (its template,
+# its block-32 instantiation unit and the headers they include).
+HEADLINE_KERNEL_SOURCES = ("fp4q_device.cuh", "internal.h", "quant_b32.cu", "quant_kernel.cuh",
+                           "quant_tma.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
     d = os.path.join(ROOT, "microscaling_fp4_quantization_bf16_b200", "csrc")
-    for f in sorted(os.listdir(d)):
+    for f in HEADLINE_KERNEL_SOURCES:
         h.update(f.encode())
         h.update(open(os.path.join(d, f), "rb").read())
     return h.hexdigest()[:16]
