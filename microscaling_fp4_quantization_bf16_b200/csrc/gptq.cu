@@ -15,9 +15,9 @@
 //                        (w_k = fma(-e, U[j][k], w_k)); the codes go to their
 //                        original column, e replaces the dead weight in work
 //   gptq_trailing_kernel every later column: t = fma chain of e_j * U[j][k]
-//                        over the batch (j ascending, from 0), w_k -= t; an
-//                        fp32 CUDA-core GEMM tile without split-K, so each
-//                        element's sum has the fixed order
+//                        over the batch (j ascending, from 0), w_k -= t; a
+//                        persistent fp32 CUDA-core GEMM without split-K, so
+//                        each element's sum has the fixed order
 //
 // Rows are independent: a row's result depends only on its weights, its
 // scales and U. Every floating-point step is one IEEE fp32 operation (fma
@@ -132,68 +132,115 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs 
     }
 }
 
+__device__ __forceinline__ void cp_async16(float* smem, const float* gmem)
+{
+    const unsigned d = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
 // work[i][k] -= sum over the batch of e[i][j] * U[b0 + j][k] for k >= b0 + GB,
-// each sum an fma chain in j order from 0. A 128 x 64 output tile per CTA
-// (96 KB of shared memory: two CTAs per SM); each thread accumulates 8 x 4
+// each sum an fma chain in j order from 0. Persistent: every CTA takes a
+// contiguous run of (row tile, column tile) items, row tile major, so the
+// 128 x 128 error tile is loaded once per row tile; the 128 x 64 U tiles
+// stream through two shared buffers by asynchronous copies, the next one in
+// flight while the current one is used. Each thread accumulates 8 x 4
 // outputs (rows 4ty..4ty+3 and 64+4ty.., columns 4tx..4tx+3) from three
-// 128-bit shared loads per j.
-__global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int64_t b0)
+// 128-bit shared loads per j; its old weights are fetched before the sums so
+// their latency hides behind them.
+__global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int64_t b0, int64_t items,
+                                                                   int64_t col_tiles)
 {
     extern __shared__ float sm[];
-    float* es = sm;             // [GB][TR]: es[j][r] = e of row r0 + r at position j
-    float* ut = sm + GB * TR;   // [GB][TC]: ut[j][c] = U[b0 + j][k0 + c]
+    float* es = sm;              // [GB][TR]: es[j][r] = e of row r0 + r at position j
+    float* ub = sm + GB * TR;    // 2 x [GB][TC]: ut[j][c] = U[b0 + j][k0 + c]
     pdl_begin();
-    const int64_t r0 = (int64_t)blockIdx.y * TR;
-    const int64_t k0 = b0 + GB + (int64_t)blockIdx.x * TC;
-    for (int e = threadIdx.x; e < TR * GB / 4; e += TTHREADS) {
-        const int r = e % TR, j4 = e / TR;  // consecutive threads: consecutive rows
-        const int64_t row = r0 + r;
-        float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-        if (row < a.rows)
-            v = *reinterpret_cast<const float4*>(a.work + row * a.K + b0 + 4 * j4);
-        es[(4 * j4) * TR + r] = v.x;
-        es[(4 * j4 + 1) * TR + r] = v.y;
-        es[(4 * j4 + 2) * TR + r] = v.z;
-        es[(4 * j4 + 3) * TR + r] = v.w;
-    }
-    for (int e = threadIdx.x; e < GB * TC / 4; e += TTHREADS) {
-        const int j = e / (TC / 4), c4 = e - j * (TC / 4);
-        reinterpret_cast<float4*>(ut)[e] =
-            *reinterpret_cast<const float4*>(a.U + (b0 + j) * a.K + k0 + 4 * c4);
-    }
-    __syncthreads();
+    const int64_t first = (int64_t)blockIdx.x * items / gridDim.x;
+    const int64_t last = ((int64_t)blockIdx.x + 1) * items / gridDim.x;
+    if (first >= last)
+        return;
     const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-    float acc[8][4];
+    auto load_u = [&](int64_t item, int buf) {
+        const int64_t k0 = b0 + GB + (item % col_tiles) * TC;
+        float* ut = ub + buf * (GB * TC);
+        for (int e = threadIdx.x; e < GB * TC / 4; e += TTHREADS) {
+            const int jj = e / (TC / 4), c4 = e - jj * (TC / 4);
+            cp_async16(ut + 4 * e, a.U + (b0 + jj) * a.K + k0 + 4 * c4);
+        }
+        cp_async_commit();
+    };
+    load_u(first, 0);
+    int64_t cur_rt = -1;
+    int buf = 0;
+    for (int64_t it = first; it < last; ++it) {
+        const int64_t rt = it / col_tiles;
+        const int64_t r0 = rt * TR;
+        const int64_t k0 = b0 + GB + (it % col_tiles) * TC;
+        if (it + 1 < last) {
+            load_u(it + 1, buf ^ 1);
+            cp_async_wait<1>();  // this item's U tile has landed (the next may be in flight)
+        } else {
+            cp_async_wait<0>();
+        }
+        if (rt != cur_rt) {
+            __syncthreads();  // nobody still reads the previous error tile
+            for (int e = threadIdx.x; e < TR * GB / 4; e += TTHREADS) {
+                const int r = e % TR, j4 = e / TR;
+                const int64_t row = r0 + r;
+                float4 v = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                if (row < a.rows)
+                    v = *reinterpret_cast<const float4*>(a.work + row * a.K + b0 + 4 * j4);
+                es[(4 * j4) * TR + r] = v.x;
+                es[(4 * j4 + 1) * TR + r] = v.y;
+                es[(4 * j4 + 2) * TR + r] = v.z;
+                es[(4 * j4 + 3) * TR + r] = v.w;
+            }
+            cur_rt = rt;
+        }
+        __syncthreads();  // error tile and this U tile visible to all
+        float4 old[8];
 #pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-            acc[r][c] = 0.0f;
-#pragma unroll 4
-    for (int j = 0; j < GB; ++j) {
-        const float4 e0 = reinterpret_cast<const float4*>(es + j * TR)[ty];
-        const float4 e1 = reinterpret_cast<const float4*>(es + j * TR + TR / 2)[ty];
-        const float4 u0 = reinterpret_cast<const float4*>(ut + j * TC)[tx];
-        const float er[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-        const float uc[4] = {u0.x, u0.y, u0.z, u0.w};
+        for (int r = 0; r < 8; ++r) {
+            const int64_t row = r0 + (r < 4 ? 4 * ty + r : TR / 2 + 4 * ty + r - 4);
+            old[r] = row < a.rows ? *reinterpret_cast<const float4*>(a.work + row * a.K + k0 + 4 * tx)
+                                  : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+        const float* ut = ub + buf * (GB * TC);
+        float acc[8][4];
 #pragma unroll
         for (int r = 0; r < 8; ++r)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                acc[r][c] = __fmaf_rn(er[r], uc[c], acc[r][c]);
-    }
+                acc[r][c] = 0.0f;
+#pragma unroll 4
+        for (int jj = 0; jj < GB; ++jj) {
+            const float4 e0 = reinterpret_cast<const float4*>(es + jj * TR)[ty];
+            const float4 e1 = reinterpret_cast<const float4*>(es + jj * TR + TR / 2)[ty];
+            const float4 u0 = reinterpret_cast<const float4*>(ut + jj * TC)[tx];
+            const float er[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
+            const float uc[4] = {u0.x, u0.y, u0.z, u0.w};
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int64_t row = r0 + (r < 4 ? 4 * ty + r : TR / 2 + 4 * ty + r - 4);
-        if (row >= a.rows)
-            continue;
-        float4* p = reinterpret_cast<float4*>(a.work + row * a.K + k0 + 4 * tx);
-        float4 v = *p;
-        v.x = __fsub_rn(v.x, acc[r][0]);
-        v.y = __fsub_rn(v.y, acc[r][1]);
-        v.z = __fsub_rn(v.z, acc[r][2]);
-        v.w = __fsub_rn(v.w, acc[r][3]);
-        *p = v;
+            for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c)
+                    acc[r][c] = __fmaf_rn(er[r], uc[c], acc[r][c]);
+        }
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int64_t row = r0 + (r < 4 ? 4 * ty + r : TR / 2 + 4 * ty + r - 4);
+            if (row >= a.rows)
+                continue;
+            float4 v = old[r];
+            v.x = __fsub_rn(v.x, acc[r][0]);
+            v.y = __fsub_rn(v.y, acc[r][1]);
+            v.z = __fsub_rn(v.z, acc[r][2]);
+            v.w = __fsub_rn(v.w, acc[r][3]);
+            *reinterpret_cast<float4*>(a.work + row * a.K + k0 + 4 * tx) = v;
+        }
+        __syncthreads();  // this U buffer is free for the copy two items ahead
+        buf ^= 1;
     }
 }
 
@@ -201,15 +248,21 @@ __global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int
 
 cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
 {
-    if (a.K % GB != 0 || a.rows <= 0 || (a.rows + TR - 1) / TR > 65535 || a.rows * a.K > ((int64_t)1 << 40))
+    if (a.K % GB != 0 || a.rows <= 0 || a.rows * a.K > ((int64_t)1 << 40))
         return cudaErrorInvalidValue;
     const size_t batch_smem = sizeof(float) * GB * GB;
-    const size_t trail_smem = sizeof(float) * GB * (TR + TC);
+    const size_t trail_smem = sizeof(float) * GB * (TR + 2 * TC);
     cudaError_t e = cudaFuncSetAttribute(gptq_batch_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)batch_smem);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(gptq_trailing_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)trail_smem);
+    if (e != cudaSuccess)
+        return e;
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess)
         return e;
     const int64_t n = a.rows * a.K;
@@ -219,9 +272,12 @@ cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
     for (int64_t b0 = 0; b0 < a.K && e == cudaSuccess; b0 += GB) {
         e = launch_pdl(gptq_batch_kernel, dim3(row_ctas), dim3(ROWS_PER_CTA * 32), batch_smem, st, a, b0);
         const int64_t rest = a.K - b0 - GB;
-        if (e == cudaSuccess && rest > 0)
-            e = launch_pdl(gptq_trailing_kernel, dim3((unsigned)(rest / TC), row_tiles), dim3(TTHREADS),
-                           trail_smem, st, a, b0);
+        if (e == cudaSuccess && rest > 0) {
+            const int64_t col_tiles = rest / TC, items = col_tiles * row_tiles;
+            const unsigned ctas = (unsigned)(items < sms ? items : sms);  // one per SM
+            e = launch_pdl(gptq_trailing_kernel, dim3(ctas), dim3(TTHREADS), trail_smem, st, a, b0, items,
+                           col_tiles);
+        }
     }
     return e;
 }
