@@ -8,6 +8,7 @@ import socket
 import sys
 
 import numpy as np
+import pytest
 import torch.multiprocessing as mp
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -65,3 +66,29 @@ def test_sharded_global_amax_two_ranks():
         assert p.exitcode == 0
     assert len(out) == 4
     assert all(all(v) for v in out.values()), dict(out)
+
+
+@pytest.mark.gpu
+def test_sharded_single_rank_nccl_on_gpu():
+    """The NCCL form on one GPU (world size 1): the all-reduce is the identity and
+    the sharded quantization equals the plain one bit for bit."""
+    import datetime
+
+    import torch
+    import torch.distributed as dist
+
+    sys.path.insert(0, ROOT)
+    import microscaling_fp4_quantization_bf16_b200 as fp4q
+    from microscaling_fp4_quantization_bf16_b200 import sharded, synth
+
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{_free_port()}", rank=0,
+                            world_size=1, timeout=datetime.timedelta(seconds=60))
+    try:
+        x = synth.workload("c3_strategy_sweep_t3", rows=64, cols=256)["x"].cuda()
+        a = sharded.quantize_sharded(x, "nvfp4", 16, "four_over_six", rot=16)
+        b = fp4q.quantize(x, "nvfp4", 16, "four_over_six", 16)
+        torch.cuda.synchronize()
+        assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
+        assert torch.equal(a.global_scale, b.global_scale)
+    finally:
+        dist.destroy_process_group()
