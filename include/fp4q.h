@@ -10,16 +10,20 @@
  *   MXFP4: E2M1 elements, one E8M0 (power-of-two) scale byte per block of 32
  *          ("Bridging the Gap Between Promise and Performance for
  *          Microscaling FP4 Quantization", 技術概要 §1).
+ *   UE5M3: E2M1 elements, one unsigned 5-exponent / 3-mantissa scale byte per
+ *          block of 4 / 8 / 16 / 32 and no per-tensor scale (see
+ *          fp4q_format for the encoding read here).
  *
  * Storage. codes: uint8 [rows, cols/2], element 2j in the low nibble of byte
  * j and element 2j+1 in the high nibble; 4-bit code = sign bit (bit 3) and
  * E2M1 magnitude index (bits 0-2). scales: uint8 [rows, cols/block]
- * row-major (E4M3 code, or E8M0 byte = exponent + 127). Per-block MSE:
+ * row-major (E4M3 code, E8M0 byte = exponent + 127, or UE5M3 code). Per-block MSE:
  * float [rows, cols/block]. Dequantized values: [rows, cols] fp32 or bf16.
  *
  * Arithmetic. Every result except the GEMM's is bit-identical to the plain
- * CPU definition of the operation: one IEEE binary32 operation per step, no
- * fused multiply-add, E2M1 / E4M3 round-to-nearest-even with saturation, the
+ * CPU definition of the operation: one IEEE binary32 operation per step (a
+ * fused multiply-add only where the definition has one, as in the GPTQ
+ * updates), E2M1 / E4M3 / UE5M3 round-to-nearest-even with saturation, the
  * optional Hadamard rotation applied as a Walsh-Hadamard butterfly with
  * ascending stages, and block sums taken with the adjacent-pair tree. The
  * GEMM accumulates on the tensor cores in fp32 in the hardware's order.
@@ -36,7 +40,9 @@
  *  - rows == 0 or cols == 0 is an empty tensor: its array pointers may be
  *    NULL, nothing is read or written except that NVFP4 global_scale_out
  *    receives 1.0 (and fp4q_global_amax writes 0).
- *  - Inputs must be finite. Outputs must not overlap inputs or each other.
+ *  - Inputs must be finite. Outputs must not overlap inputs or each other
+ *    (arrays an entry point documents as read and overwritten are the
+ *    exception: they are updated in place).
  *  - FP4Q_ERR_CUDA means a launch was rejected by the CUDA runtime; the
  *    runtime's code is available from fp4q_last_cuda_error(). Faults that
  *    happen while the kernels run surface at the caller's next
