@@ -203,7 +203,7 @@ def test_layer_objective_loop(gpu):
     the GPU forward must equal the oracle's bit for bit; the gradient 2 E H is
     formed on the host from that (identical) W_hat, and the GPU update must
     equal the oracle's. The loss falls over the steps."""
-    import test_oracle_focus_opt as prob
+    import focus_layer as prob
     rows, cols, sub = 128, 256, 8
     wb, h = prob.layer_problem(rows, cols, 1024, seed=0)
     wd = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).cuda()
