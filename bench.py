@@ -475,6 +475,19 @@ def breakdown(dev, peaks, reps: int = 10):
     rows_out.append({"run": "c3_strategy_sweep_t3 quality: mean block MSE (E4M3 + s_g vs UE5M3)",
                      "mse": {k: float(f"{v:.6e}") for k, v in qual.items()}})
     del x3, q3
+    # rotation and round-to-nearest (abs-max), "Bridging the Gap ..." §2.1: the
+    # blockwise Hadamard lowers MXFP4's MSE on Laplace data with outliers and
+    # raises NVFP4's; the MSE is taken in the rotated domain, which the
+    # normalised rotation leaves unchanged up to the rounding of k_n
+    rot_q = {}
+    for wl in ("c2_mxfp4_laplace_outliers", "c5_activation_channels"):
+        xr = synth.workload(wl)["x"].to(dev)
+        for fmt, block, rot in (("mxfp4", 32, 0), ("mxfp4", 32, 32), ("nvfp4", 16, 0), ("nvfp4", 16, 16)):
+            qr = fp4q.quantize(xr, fmt, block, "absmax", rot, want_mse=True)
+            rot_q[f"{wl} {fmt} B{block} H{rot}"] = float(qr.mse.double().mean())
+        del xr, qr
+    rows_out.append({"run": "quality: mean block MSE with and without the blockwise Hadamard (abs-max)",
+                     "mse": {k: float(f"{v:.6e}") for k, v in rot_q.items()}})
     torch.cuda.empty_cache()
     quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
                                           ("mxfp4", 32, "absmax", 128)])
