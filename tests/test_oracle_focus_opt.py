@@ -239,3 +239,27 @@ def test_adam_calibration_lowers_layer_loss(ref):
         c, m, v = out["c"], out["m"], out["v"]
     last, _ = layer_loss_and_grad(ref, wb, c, h)
     assert last < 0.95 * first, (first, last)
+
+
+# -------------------------------------------------------- the pages' facts
+
+def test_calibration_state_follows_the_page():
+    # the Python calibration state starts from the page's c = 1 in fp16, with
+    # one coefficient per sub-block of the page's example size
+    import os
+    import torch
+    import microscaling_fp4_quantization_bf16_b200 as fp4q
+    kv = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", "focus_facts.txt")) as f:
+        for line in f:
+            line = line.split("#")[0].strip()
+            if line:
+                k, v = line.split()
+                kv[k] = float(v)
+    sub = int(kv["focus_sub_block_example"])
+    st = fp4q.focus_state(4, 2 * int(kv["nvfp4_block"]), sub, "adam")   # CPU tensors
+    assert st.c_half.dtype == torch.float16 and st.c_half.element_size() * 8 == kv["focus_coefficient_bits"]
+    assert torch.all(st.c == kv["focus_coefficient_init"]) and torch.all(st.c_half == 1.0)
+    assert st.c.shape == (4, 2 * int(kv["nvfp4_block"]) // sub)
+    assert torch.all(st.m == 0) and torch.all(st.v == 0) and st.t == 0
+    assert int(kv["mxfp4_block"]) % sub == 0 and int(kv["nvfp4_block"]) % sub == 0
