@@ -220,3 +220,22 @@ def test_gemm_validation(lib):
     assert qm(fmt=UE) == UNSUP       # the MMA takes E4M3 / E8M0 scales only
     assert L.fp4q_mma_scale_bytes(128, 64, UE) == 0
     assert L.fp4q_scales_to_mma(A, 128, 64, UE, A, None) == UNSUP
+
+
+def test_header_is_plain_c(tmp_path):
+    """include/fp4q.h compiles as ISO C11 (pedantic) and C++17: no torch or C++
+    types in the interface."""
+    import shutil
+    import subprocess
+    cuda_inc = "/usr/local/cuda/include"
+    if shutil.which("gcc") is None or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime_api.h")):
+        pytest.skip("gcc or the CUDA headers are not available")
+    src = tmp_path / "h.c"
+    src.write_text('#include "fp4q.h"\nint main(void) { return (int)FP4Q_OK; }\n')
+    for cc, std, name in (("gcc", "-std=c11", "h.c"), ("g++", "-std=c++17", "h.cpp")):
+        f = tmp_path / name
+        f.write_text(src.read_text())
+        r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror",
+                            "-I" + os.path.dirname(HEADER), "-I" + cuda_inc, "-c", str(f),
+                            "-o", str(tmp_path / (name + ".o"))], capture_output=True, text=True)
+        assert r.returncode == 0, r.stderr
