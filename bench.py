@@ -491,6 +491,9 @@ def breakdown(dev, peaks, reps: int = 10):
     torch.cuda.empty_cache()
     quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
                                           ("mxfp4", 32, "absmax", 128)])
+    # the headline's kernels on a tensor 8x larger (256 MiB of bf16): the same
+    # code with the launch ramp and tail amortised over 134M elements
+    quant_runs("c5_activation_channels", [("mxfp4", 32, "absmax", 0), ("mxfp4", 32, "absmax", 32)])
     # W4A4 GEMM on the block-scaled tensor cores, LLM layer shapes (tokens x hidden
     # -> out): operands quantized (abs-max) once, scales in MMA layout; timed: the
     # GEMM alone (alpha + tcgen05 GEMM), bf16 output. Roofline: the dense FP4 peak
