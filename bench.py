@@ -1,17 +1,20 @@
 #!/usr/bin/env python
 """Throughput of the block-scaled FP4 quantization hot path on B200.
 
-Headline workload: MXFP4 (E8M0 scales, block 32) quantization of a
-4096 x 4096 bf16 weight drawn from Laplace(0, 0.02) with 0.1% of entries
-times 50, run without rotation and with a 32-wide blockwise Hadamard; one step
-= both runs. Inputs are resident in HBM and larger than L2: every launch
-reads its own copy of the tensor, rotating through enough copies that each
-is evicted before it is read again. ``value`` is quantized
-elements per second over the whole job (all ranks: independent replicas,
-weak scaling). One JSON line is printed by rank 0.
+Headline workload: online activation quantization of a 16384-token x
+8192-hidden bf16 tensor (Laplace(0, 1), 1% of the hidden channels x20). One
+step = both runs the pages pair with that tensor:
+  - NVFP4: 16-wide blockwise Hadamard, tensor abs-max computed on the device
+    (FP32 global scale), E4M3 block-16 scales chosen by 4-over-6, E2M1 codes;
+  - MXFP4: 128-wide blockwise Hadamard, E8M0 block-32 scales, E2M1 codes.
+Outputs are packed codes and scale bytes. Inputs are resident in HBM and
+larger than L2 (each launch reads its own copy of the tensor). ``value`` is
+quantized elements per second over the whole job (all ranks: independent
+replicas, weak scaling). Rank 0 prints ONE compact JSON line, last on stdout.
 
-``--impl reference`` times the oracle (plain C, host cores) on a bounded
-sample of the same workload instead.
+``--breakdown FILE`` also times every configuration of every workload and
+writes that table to FILE. ``--impl reference`` times the oracle (plain C,
+host cores) on a bounded sample of the same workload instead.
 """
 from __future__ import annotations
 
@@ -29,9 +32,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = ("quantized elements/s and achieved HBM GB/s (% of B200 roofline) per "
           "format/strategy")
-WORKLOAD = "c2_mxfp4_laplace_outliers"
-ROWS, COLS = 4096, 4096
-ROTS = (0, 32)
+WORKLOAD = "c5_activation_channels"
+ROWS, COLS = 16384, 8192
+# The two runs of one step: (format, block, strategy, rotation).
+RUNS = (("nvfp4", 16, "four_over_six", 16), ("mxfp4", 32, "absmax", 128))
+RUN_TAGS = ("nvfp4_b16_h16_4over6", "mxfp4_b32_h128")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 SM_COUNT_NOMINAL, FP32_LANES_PER_SM, SM_MAX_MHZ_NOMINAL = 148, 128, 1965.0
 SLEEP_CYCLES_PER_LAUNCH = 100_000  # ~50 us of GPU spin per queued launch (CPU enqueue cover)
@@ -65,10 +70,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-# The sources the headline quantize kernel is compiled from (its template,
-# its block-32 instantiation unit and the headers they include).
-HEADLINE_KERNEL_SOURCES = ("fp4q_device.cuh", "internal.h", "quant_b32.cu", "quant_kernel.cuh",
-                           "quant_tma.cuh")
+# The sources the headline quantize kernels are compiled from (the kernel
+# template, its block-16 / block-32 instantiation units, the headers).
+HEADLINE_KERNEL_SOURCES = ("fp4q_device.cuh", "internal.h", "quant_b16.cu", "quant_b32.cu",
+                           "quant_kernel.cuh", "quant_tma.cuh")
 
 
 def kernel_source_hash():
@@ -81,8 +86,8 @@ def kernel_source_hash():
 
 
 def recorded_traffic(kernel: str):
-    """dram bytes per launch from a committed ncu summary, if the kernels
-    have not changed since it was taken."""
+    """DRAM bytes per launch from a committed ncu summary, if the kernels
+    have not changed since it was taken; else None."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
@@ -102,7 +107,7 @@ class ClockSampler:
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
                0x100: "display_clock_setting"}
 
-    def __init__(self, index: int, period_s: float = 0.005):
+    def __init__(self, index: int, period_s: float = 0.002):
         self.samples = []
         self.ok = False
         self.period = period_s
@@ -173,6 +178,13 @@ def reduce_max(value: float, world: int, dev) -> float:
     return float(t.item())
 
 
+def _outputs(fp4q, torch, dev, fmt, block):
+    nv = fmt == "nvfp4"
+    return fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
+                          torch.empty(ROWS, COLS // block, dtype=torch.uint8, device=dev),
+                          torch.empty(1, device=dev) if nv else None, None, None)
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -188,37 +200,46 @@ def run_ours(args, rank, world, local_rank):
                                 device_id=dev)
     fp4q.load()
     peaks = load_peaks()
-    props = torch.cuda.get_device_properties(dev)
-    l2 = props.L2_cache_size
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     # Inputs larger than L2: every launch reads its own copy of x, and a copy
     # comes round again only after more than 2 x L2 of other traffic.
-    x0 = synth.workload(WORKLOAD)["x"].to(dev)
+    xh = synth.workload(WORKLOAD)["x"]
+    x0 = xh.to(dev)
     n = x0.numel()
-    ncopy = copies_for(x0.numel() * 2, l2)
-    xs = [x0.clone() for _ in range(ncopy)]
-    outs = [fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
-                           torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
-                           None, None, None) for _ in range(ncopy)]
+    ncopy = copies_for(2 * n, l2)
+    xs = [x0] + [x0.clone() for _ in range(ncopy - 1)]
+    outs = [[_outputs(fp4q, torch, dev, f, b) for (f, b, _, _) in RUNS] for _ in range(ncopy)]
+    (fmt_nv, b_nv, s_nv, r_nv), (fmt_mx, b_mx, s_mx, r_mx) = RUNS
     counter = [0]
 
     def run_steps(nsteps):
-        """nsteps steps' work queued behind one sleep (the GPU never waits for
-        the CPU): nsteps rot-0 launches, then nsteps rot-32 launches, each on
-        its own input copy. Events only at the group boundaries, so launches
-        stream back to back (programmatic dependent launch overlaps each
-        launch with the previous kernel). Returns ms per group."""
-        ev = [torch.cuda.Event(enable_timing=True) for _ in range(len(ROTS) + 1)]
-        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nsteps * len(ROTS))
+        """nsteps steps queued behind one GPU sleep (the GPU never waits for
+        the CPU), grouped by kernel: nsteps tensor abs-max passes (16-wide
+        rotation), nsteps NVFP4 quantizations (each reading the abs-max its
+        own step computed), nsteps MXFP4 quantizations; step i works on input
+        copy i mod ncopy. CUDA events only at the group boundaries, so the
+        launches of a group stream back to back (programmatic dependent
+        launch). Returns ms per group."""
+        ga = torch.empty(nsteps, device=dev)
+        base = counter[0]
+        counter[0] += nsteps
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+        torch.cuda._sleep(SLEEP_CYCLES_PER_LAUNCH * nsteps * 3)
         ev[0].record()
-        for k, r in enumerate(ROTS):
-            for _ in range(nsteps):
-                j = counter[0] % ncopy
-                counter[0] += 1
-                fp4q.quantize(xs[j], "mxfp4", 32, "absmax", r, out=outs[j])
-            ev[k + 1].record()
+        for i in range(nsteps):
+            fp4q.global_amax(xs[(base + i) % ncopy], r_nv, out=ga[i:i + 1])
+        ev[1].record()
+        for i in range(nsteps):
+            j = (base + i) % ncopy
+            fp4q.quantize(xs[j], fmt_nv, b_nv, s_nv, r_nv, global_amax=ga[i:i + 1], out=outs[j][0])
+        ev[2].record()
+        for i in range(nsteps):
+            j = (base + i) % ncopy
+            fp4q.quantize(xs[j], fmt_mx, b_mx, s_mx, r_mx, out=outs[j][1])
+        ev[3].record()
         torch.cuda.synchronize()
-        return [ev[k].elapsed_time(ev[k + 1]) for k in range(len(ROTS))]
+        return [ev[k].elapsed_time(ev[k + 1]) for k in range(3)]
 
     sampler = ClockSampler(local_rank)
     with sampler:
@@ -236,44 +257,79 @@ def run_ours(args, rank, world, local_rank):
             dist.barrier()
         t1 = time.perf_counter()
     clocks = sampler.summary(t0, t1)
-    x = xs[0]
-    times = {r: [group_ms[k] / args.steps] for k, r in enumerate(ROTS)}
 
     total_ms = reduce_max(sum(group_ms), world, dev)
-    elems = n * len(ROTS) * args.steps * world
+    elems = n * len(RUNS) * args.steps * world
     value = elems / (total_ms / 1e3)
     ms_per_step = total_ms / args.steps
 
-    # roofline of the dominant kernel (the launch with the larger mean time)
-    mean = {r: statistics.mean(times[r]) for r in ROTS}
-    dom = max(ROTS, key=lambda r: mean[r])
-    alg_bytes = bytes_per_elem(32) * n
-    achieved = alg_bytes / (mean[dom] / 1e3) / 1e9
-    kname = f"quant_kernel<B=32, ROT={dom}, MXFP4 abs-max> (direct loads)"
+    # Per-launch times; the roofline is that of the dominant quantize kernel
+    # (one pass over the tensor: its abs-max is an input).
+    us = [g / args.steps * 1e3 for g in group_ms]
+    kern = {"amax_h16": {"us": round(us[0], 2)}}
+    alg = {}
+    for k, (tag, (fmt, block, strat, rot)) in enumerate(zip(RUN_TAGS, RUNS)):
+        alg[tag] = bytes_per_elem(block) * n
+        gbs = alg[tag] / (us[k + 1] * 1e-6) / 1e9
+        kern[tag] = {"us": round(us[k + 1], 2), "alg_GBps": round(gbs, 1),
+                     "frac": round(gbs / peaks["hbm_gbs"], 4)}
+    dom = max(RUN_TAGS, key=lambda t: kern[t]["us"])
+    kname = {"nvfp4_b16_h16_4over6": "quant_kernel<16, 16, 2> (NVFP4 B16, H16, 4-over-6)",
+             "mxfp4_b32_h128": "quant_kernel<32, 128, 4> (MXFP4 B32, H128)"}[dom]
     traffic = recorded_traffic(kname)
-    roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
-                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "algorithmic_bytes_per_launch": int(alg_bytes),
-                "peak_source": peaks["source"] + " (copy bandwidth, burst)",
-                "per_launch_us": {f"rot{r}": round(mean[r] * 1e3, 2) for r in ROTS}}
+    roofline = {"bound": "hbm", "kernel": kname, "achieved": kern[dom]["alg_GBps"],
+                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kern[dom]["frac"],
+                "traffic": traffic, "algorithmic_bytes_per_launch": int(alg[dom]),
+                "peak_source": peaks["source"] + " copy bandwidth (burst)"}
 
-    # End to end through the public API, every step: its bf16 input from
-    # pinned host memory to the device, both runs, codes and scales back to
-    # pinned host memory. Steps are pipelined over two buffer sets and three
-    # streams (host->device copy, compute, device->host copy), so step i's
-    # upload overlaps step i-1's download; each buffer set is reused only
-    # after its previous step's download finished.
-    xh = synth.workload(WORKLOAD)["x"].pin_memory()
+    e2e = e2e_run(args, fp4q, synth, torch, dev, xh, world, n)
+
+    cfg = {"workload": f"{WORKLOAD}: {ROWS}x{COLS} bf16 activations, Laplace(0,1), 1% of hidden "
+                       "channels x20; step = NVFP4 B16 + H16 + device abs-max + 4-over-6, and "
+                       "MXFP4 B32 + H128 (codes + scale bytes)",
+           "rows": ROWS, "cols": COLS,
+           "l2": f"inputs larger than L2: each launch reads its own copy of x ({ncopy} copies)",
+           "parallelism": f"replicas x{world} (independent tensors, no collective)",
+           "timing": "launches grouped by kernel (abs-max, NVFP4, MXFP4) behind one GPU sleep; "
+                     "CUDA events at the group boundaries"}
+    line = {"metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic", "config": cfg, "roofline": roofline, "kernels": kern,
+            "e2e": e2e, "gpu_launches": 3 * args.steps, "clocks": clocks}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    if rank == 0 and world == 1 and args.breakdown:
+        rows = breakdown(dev, peaks)
+        with open(args.breakdown, "w") as f:
+            json.dump(rows, f, indent=1)
+        line["breakdown_file"] = os.path.basename(args.breakdown)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line, separators=(",", ":")), flush=True)
+
+
+def e2e_run(args, fp4q, synth, torch, dev, xh, world, n):
+    """The same step end to end through the public API with host buffers:
+    every step uploads the bf16 tensor from pinned host memory, quantizes it
+    twice (the NVFP4 call computes its own abs-max), and downloads codes,
+    scale bytes and the global scale to pinned host memory. Steps are
+    pipelined over two buffer sets and three streams (upload / compute /
+    download), so step i's upload overlaps step i-1's download; a buffer set
+    is reused only after its previous download finished. Wall clock around
+    all steps, max over ranks."""
+    import torch.distributed as dist
+
+    xp = xh.pin_memory()
     nb = 2
-    xd = [torch.empty_like(x) for _ in range(nb)]
-    eo = [{r: fp4q.Quantized(torch.empty(ROWS, COLS // 2, dtype=torch.uint8, device=dev),
-                             torch.empty(ROWS, COLS // 32, dtype=torch.uint8, device=dev),
-                             None, None, None) for r in ROTS} for _ in range(nb)]
-    ch = [{r: torch.empty(ROWS, COLS // 2, dtype=torch.uint8).pin_memory() for r in ROTS}
-          for _ in range(nb)]
-    sh = [{r: torch.empty(ROWS, COLS // 32, dtype=torch.uint8).pin_memory() for r in ROTS}
-          for _ in range(nb)]
+    xd = [torch.empty_like(xp, device=dev) for _ in range(nb)]
+    eo = [[_outputs(fp4q, torch, dev, f, b) for (f, b, _, _) in RUNS] for _ in range(nb)]
+    hosts = [[[torch.empty_like(t, device="cpu").pin_memory()
+               for t in (q.codes, q.scales, q.global_scale) if t is not None] for q in eo[0]]
+             for _ in range(nb)]
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     up = [torch.cuda.Event() for _ in range(nb)]
     done = [torch.cuda.Event() for _ in range(nb)]
@@ -281,71 +337,41 @@ def run_ours(args, rank, world, local_rank):
     for k in range(nb):  # buffers start free
         down[k].record(s_out)
 
-    def e2e_steps(nsteps):
+    def steps(nsteps):
         for i in range(nsteps):
             k = i % nb
             s_in.wait_event(down[k])  # x / outputs of set k no longer in use
             with torch.cuda.stream(s_in):
-                xd[k].copy_(xh, non_blocking=True)
+                xd[k].copy_(xp, non_blocking=True)
                 up[k].record(s_in)
             s_cmp.wait_event(up[k])
             with torch.cuda.stream(s_cmp):
-                for r in ROTS:
-                    fp4q.quantize(xd[k], "mxfp4", 32, "absmax", r, out=eo[k][r])
+                for q, (fmt, block, strat, rot) in zip(eo[k], RUNS):
+                    fp4q.quantize(xd[k], fmt, block, strat, rot, out=q)
                 done[k].record(s_cmp)
             s_out.wait_event(done[k])
             with torch.cuda.stream(s_out):
-                for r in ROTS:
-                    ch[k][r].copy_(eo[k][r].codes, non_blocking=True)
-                    sh[k][r].copy_(eo[k][r].scales, non_blocking=True)
+                for q, hs in zip(eo[k], hosts[k]):
+                    for h, t in zip(hs, [t for t in (q.codes, q.scales, q.global_scale)
+                                         if t is not None]):
+                        h.copy_(t, non_blocking=True)
                 down[k].record(s_out)
         torch.cuda.synchronize()
 
-    e2e_steps(args.warmup)
+    steps(args.warmup)
     if world > 1:
         dist.barrier()
-    te0 = time.perf_counter()
-    e2e_steps(args.steps)
-    te = reduce_max(time.perf_counter() - te0, world, dev)
-    h2d = xh.numel() * xh.element_size()
-    d2h = sum(ch[0][r].numel() + sh[0][r].numel() for r in ROTS)
-    e2e = {"value": elems / te, "unit": "elements/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "ms_per_step": round(te / args.steps * 1e3, 4),
-           "path": "pinned host bf16 -> cudaMemcpyAsync -> fp4q_quantize x2 -> codes+scales "
-                   "to pinned host; two buffer sets, upload / compute / download streams "
-                   "(step i's upload overlaps step i-1's download); wall clock around all "
-                   "steps, synchronised at the end"}
-
-    line = {"metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-            "data": "synthetic",
-            "config": {"workload": f"{WORKLOAD}: MXFP4 E8M0 block 32 on a {ROWS}x{COLS} bf16 "
-                                   "Laplace(0,0.02) weight with 0.1% entries x50; one step = "
-                                   "rot 0 + rot 32 (Hadamard) runs",
-                       "rows": ROWS, "cols": COLS, "format": "mxfp4", "block": 32,
-                       "rot": list(ROTS), "outputs": "packed codes + scale bytes",
-                       "l2": f"inputs larger than L2: each launch reads its own copy of x "
-                             f"({ncopy} copies, {ncopy * n * 2 / 2**20:.0f} MiB in rotation)",
-                       "parallelism": f"replicas x{world} (independent tensors, no collective)",
-                       "soak_s": args.soak,
-                       "timing": "steps queued behind one GPU sleep; the timed region runs all rot-0 "
-                                 "launches then all rot-32 launches back to back (one input copy "
-                                 "each), CUDA events at the start, between the groups and at the "
-                                 "end; per-kernel time = group time / launches"},
-            "roofline": roofline, "e2e": e2e, "gpu_launches": len(ROTS) * args.steps,
-            "launch_note": "every library kernel uses programmatic dependent launch",
-            "clocks": clocks}
-
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
-    if rank == 0 and world == 1 and not args.no_breakdown:
-        line["breakdown"] = breakdown(dev, peaks)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    t0 = time.perf_counter()
+    steps(args.e2e_steps)
+    te = reduce_max(time.perf_counter() - t0, world, dev)
+    h2d = xp.numel() * xp.element_size()
+    d2h = sum(h.numel() * h.element_size() for hs in hosts[0] for h in hs)
+    return {"value": n * len(RUNS) * args.e2e_steps * world / te, "unit": "elements/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+            "ms_per_step": round(te / args.e2e_steps * 1e3, 4),
+            "path": "pinned host bf16 -> device -> fp4q.quantize x2 (NVFP4 computes its abs-max) "
+                    "-> codes, scales, global scale to pinned host; upload/compute/download "
+                    "streams, two buffer sets; wall clock"}
 
 
 # ---------------------------------------------------------------- breakdown
@@ -597,6 +623,21 @@ def breakdown(dev, peaks, reps: int = 10):
 
 # ---------------------------------------------------------------- oracle
 
+def _oracle_step_work(oracle, xs):
+    """The oracle's work for one slice of rows, as the GPU step does it: the
+    slice's abs-max under the 16-wide rotation, NVFP4 4-over-6 with that
+    abs-max, MXFP4 with the 128-wide rotation. Returns elements quantized."""
+    ga = oracle.global_amax(xs, RUNS[0][3])
+    for fmt, block, strat, rot in RUNS:
+        oracle.quantize(xs, fmt, block, strat, rot,
+                        global_amax=ga if fmt == "nvfp4" else None, want_mse=False)
+    return xs.size * len(RUNS)
+
+
+def _host_cores():
+    return len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+
+
 def cpu_baseline(seconds: float):
     """The oracle (C, unchanged) on row slices of the headline tensor, both
     runs: first single-threaded for about seconds / 2, then driven over rows
@@ -610,13 +651,10 @@ def cpu_baseline(seconds: float):
 
     x = synth.bits16(synth.workload(WORKLOAD)["x"])
     oracle.lib()
-    chunk = 64
+    chunk = 16
 
     def work(r0):
-        xs = x[r0:r0 + chunk]
-        for r in ROTS:
-            oracle.quantize(xs, "mxfp4", 32, "absmax", r, want_mse=False)
-        return xs.size * len(ROTS)
+        return _oracle_step_work(oracle, x[r0:r0 + chunk])
 
     done1, t1, r0 = 0, 0.0, 0
     while t1 < seconds / 2:
@@ -626,23 +664,23 @@ def cpu_baseline(seconds: float):
         r0 = (r0 + chunk) % ROWS
     single = done1 / t1
 
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
-    per_round = ROWS // chunk
-    done, rounds = 0, 0
+    cores = _host_cores()
+    done, slices = 0, 0
     with ThreadPoolExecutor(max_workers=cores) as ex:
         t0 = time.perf_counter()
         while True:
-            done += sum(ex.map(work, range(0, ROWS, chunk)))
-            rounds += 1
+            starts = [((slices + i) * chunk) % ROWS for i in range(cores)]
+            done += sum(ex.map(work, starts))
+            slices += cores
             tw = time.perf_counter() - t0
             if tw >= seconds / 2:
                 break
     return {"value": done / tw, "unit": "elements/s", "cores": cores, "kind": "oracle",
-            "sample": f"{rounds} pass(es) over the {ROWS}x{COLS} tensor in {per_round} slices of "
-                      f"{chunk} rows, rot 0 and rot 32 each, the C oracle called from {cores} "
+            "sample": f"{slices} slices of {chunk} rows of the {ROWS}x{COLS} tensor (each: its "
+                      f"abs-max, NVFP4 H16 4-over-6, MXFP4 H128), the C oracle from {cores} "
                       f"threads at once, {tw:.1f} s wall",
             "single_thread": {"value": single, "cores": 1,
-                              "sample": f"{done1 // len(ROTS)} elements, {t1:.1f} s"}}
+                              "sample": f"{done1 // len(RUNS)} elements, {t1:.1f} s"}}
 
 
 def run_reference(args, rank, world):
@@ -659,22 +697,19 @@ def run_reference(args, rank, world):
 
     x = synth.bits16(synth.workload(WORKLOAD)["x"])
     oracle.lib()
-    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else os.cpu_count()
+    cores = _host_cores()
     # size each step so the whole run takes about args.ref_seconds
     t0 = time.perf_counter()
-    oracle.quantize(x[:8], "mxfp4", 32, "absmax", 32, want_mse=False)
-    per_elem = (time.perf_counter() - t0) / (8 * COLS)
+    _oracle_step_work(oracle, x[:4])
+    per_row = (time.perf_counter() - t0) / 4
     per_step_s = args.ref_seconds / max(1, args.steps + args.warmup)
-    rows = int(max(cores, min(ROWS, cores * per_step_s / (per_elem * COLS * len(ROTS)))))
+    rows = int(max(cores, min(ROWS, cores * per_step_s / per_row)))
     rows -= rows % cores
     slice_rows = rows // cores
     r0 = 0
 
     def work(a):
-        xs = x[a:a + slice_rows]
-        for r in ROTS:
-            oracle.quantize(xs, "mxfp4", 32, "absmax", r, want_mse=False)
-        return xs.size * len(ROTS)
+        return _oracle_step_work(oracle, x[a:a + slice_rows])
 
     def step(ex):
         nonlocal r0
@@ -692,21 +727,22 @@ def run_reference(args, rank, world):
             done += step(ex)
         t = time.perf_counter() - t0
     value = done / t
-    sample = (f"{rows} rows x {COLS} of the {ROWS}x{COLS} tensor per step, rot 0 and rot 32, "
-              f"the C oracle called from {cores} threads on {slice_rows}-row slices")
+    sample = (f"{rows} rows x {COLS} of the {ROWS}x{COLS} tensor per step (each slice: its "
+              f"abs-max, NVFP4 H16 4-over-6, MXFP4 H128), the C oracle called from {cores} "
+              f"threads on {slice_rows}-row slices")
     line = {"metric": METRIC, "value": value, "unit": "elements/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "impl": "reference",
-            "config": {"workload": f"{WORKLOAD}: MXFP4 E8M0 block 32, rot 0 + rot 32",
-                       "rows": ROWS, "cols": COLS, "format": "mxfp4", "block": 32,
-                       "rot": list(ROTS), "sample_rows_per_step": rows},
+            "config": {"workload": f"{WORKLOAD}: NVFP4 B16 + H16 + abs-max + 4-over-6, and "
+                                   "MXFP4 B32 + H128",
+                       "rows": ROWS, "cols": COLS, "sample_rows_per_step": rows},
             "cpu_baseline": {"value": value, "unit": "elements/s", "cores": cores,
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "elements/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
-    print(json.dumps(line), flush=True)
+    print(json.dumps(line, separators=(",", ":")), flush=True)
 
 
 # ---------------------------------------------------------------- kernel suite
@@ -774,14 +810,17 @@ def run_suite(rounds: int = 2):
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--e2e-steps", type=int, default=20,
+                    help="end-to-end steps (each uploads the 256 MiB tensor from the host)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--soak", type=float, default=1.0, help="seconds of untimed load before warm-up")
     ap.add_argument("--cpu-seconds", type=float, default=8.0)
     ap.add_argument("--ref-seconds", type=float, default=60.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--breakdown", metavar="FILE", default=None,
+                    help="also time every configuration of every workload; write the table to FILE")
     ap.add_argument("--suite", action="store_true",
                     help="launch every library kernel once per round (for ncu captures)")
     args = ap.parse_args()

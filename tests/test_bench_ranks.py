@@ -83,3 +83,41 @@ def test_reference_arm_json_line():
     assert d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
     assert d["cpu_baseline"]["value"] == d["value"] and d["e2e"]["value"] == d["value"]
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_reference_arm_line_is_compact():
+    """The driver reads the last stdout line: it must be one JSON object of a
+    few KB at most."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                          "--steps", "3", "--warmup", "3", "--ref-seconds", "1"],
+                         capture_output=True, text=True, timeout=600, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    last = out.stdout.strip().splitlines()[-1]
+    assert len(last) < 4096
+    assert isinstance(json.loads(last), dict)
+
+
+@pytest.mark.gpu
+def test_bench_headline_line_is_compact():
+    """Our arm on the GPU: a short run prints, as its last stdout line, one
+    compact JSON object with the contract's keys, the roofline of the
+    dominant kernel and the end-to-end figure."""
+    import json
+    import subprocess
+    out = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "5",
+                          "--warmup", "3", "--e2e-steps", "3", "--soak", "0",
+                          "--no-cpu-baseline"],
+                         capture_output=True, text=True, timeout=900, cwd=ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    last = out.stdout.strip().splitlines()[-1]
+    assert len(last) < 4096
+    d = json.loads(last)
+    for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+              "higher_is_better", "scaling", "vs_baseline", "dtype", "data", "config",
+              "roofline", "e2e", "gpu_launches", "clocks"):
+        assert k in d, k
+    assert d["value"] > 0 and d["config"]["workload"].startswith("c5_activation_channels")
+    assert d["roofline"]["bound"] == "hbm" and 0 < d["roofline"]["frac"] < 2
+    assert d["e2e"]["h2d_bytes_per_step"] == 16384 * 8192 * 2
