@@ -63,7 +63,21 @@ __device__ __forceinline__ uint4 ldg_stream(const uint4* p)
     return v;
 }
 
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+#ifndef FP4Q_UNPACK_PRMT
+#define FP4Q_UNPACK_PRMT 1
+#endif
+// The low bf16 of a word, widened: the byte permute keeps it on the integer
+// ALU (a shift may be issued to the FMA pipe as a multiply).
+__device__ __forceinline__ float bf_lo(uint32_t w)
+{
+#if FP4Q_UNPACK_PRMT
+    uint32_t r;
+    asm("prmt.b32 %0, %1, 0, 0x1044;" : "=r"(r) : "r"(w));
+    return __uint_as_float(r);
+#else
+    return __uint_as_float(w << 16);
+#endif
+}
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 // Raw bf16 words of segment s (elements s*32 .. s*32+31) of an array of n
@@ -283,6 +297,10 @@ __device__ __forceinline__ float e8m0_dec(uint32_t b)
 struct NvConsts {
     float den6, rden6, den4, rden4;
     bool fast;  // both reciprocals finite: the quotient shortcut applies
+    // 2^-105 <= s_g <= 2^110: every nonzero scale S = E4M3(c) s_g lies in
+    // (2^-120, 2^119], so a power-of-two rotation factor k >= 2^-3 can be
+    // folded into fl(1/S) exactly (see candidate_seg and fold_ok below).
+    bool fold;
 };
 
 __device__ __forceinline__ NvConsts nv_consts(float sg)
@@ -293,6 +311,7 @@ __device__ __forceinline__ NvConsts nv_consts(float sg)
     k.rden6 = __frcp_rn(k.den6);
     k.rden4 = __frcp_rn(k.den4);
     k.fast = k.rden6 <= FLT_MAX && k.rden4 <= FLT_MAX;
+    k.fold = sg >= 0x1p-105f && sg <= 0x1p110f;
     return k;
 }
 
@@ -407,8 +426,10 @@ __device__ __forceinline__ f32x2 fma2(f32x2 a, f32x2 b, f32x2 c)
 //  - h = 32, 64 pair lane L with lane L ^ (h / 32): the lower lane needs
 //    p + v, the upper p - v (p the partner's value, v its own), again one
 //    exact product and one rounding: fma(+-1, v, p).
-// All 32 lanes of the warp must call this together.
-template <int ROT>
+// All 32 lanes of the warp must call this together. SCALE = false leaves
+// out the multiply by k_ROT (the caller applies it, or folds it where k_ROT is
+// a power of two: see candidate_seg).
+template <int ROT, bool SCALE = true>
 __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
 {
     if constexpr (ROT > 0) {
@@ -451,11 +472,27 @@ __device__ __forceinline__ void rotate_seg(float (&y)[SEG], int lane)
                 P[i] = fma2(ss, P[i], pk2(plo, phi));
             }
         }
-        const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
+        if constexpr (SCALE) {
+            const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-            upk2(mul2(P[i], kk), y[i], y[i + 16]);
+            for (int i = 0; i < 16; ++i)
+                upk2(mul2(P[i], kk), y[i], y[i + 16]);
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                upk2(P[i], y[i], y[i + 16]);
+        }
     }
+}
+
+// y <- y * k_ROT for a segment left unscaled by rotate_seg<ROT, false>.
+template <int ROT>
+__device__ __forceinline__ void scale_seg(float (&y)[SEG])
+{
+    const f32x2 kk = pk2(HadK<ROT>::k, HadK<ROT>::k);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+        upk2(mul2(pk2(y[i], y[i + 16]), kk), y[i], y[i + 16]);
 }
 
 // Segments per thread (one; kept as a parameter of the kernels' indexing).
@@ -731,6 +768,166 @@ __device__ __forceinline__ void sse_seg(const float (&y)[SEG], const uint32_t (&
         sse_seg_packed<B>(y, q, S, sse);
     else
         sse_seg_scalar<B>(y, q, S, sse);
+}
+
+// One candidate scale per block for a whole segment: the packed E2M1 codes
+// (before zero-scale masking) and, with WANT_SSE, each block's SSE -- the
+// adjacent-pair tree sum of fl(d^2), d = fl(y - fl(value(q) * S)).
+//
+// t holds y (FOLD = false), or the rotated values before their multiply by
+// k = kf, a power of two (FOLD = true): then y = t * kf exactly, r must
+// already be fl(1/S) * kf (exact), u = fl(t * r) = fl(y * fl(1/S)) and
+// d = fma(t, kf, -yhat) = fl(y - yhat); the caller guarantees the exactness
+// conditions (no value of t * kf or fl(1/S) * kf is lost to underflow where it
+// matters).
+//
+// Words w and w + 2 are processed together on packed pairs {i, i + 16}. The
+// products that feed a subtraction or a tree addition are formed as
+// fma(a, b, z) with z a run-time +0 (kernel argument): fl(a * b + 0) equals
+// fl(a * b) (a zero product gives +0, which changes no difference or square
+// below), and ptxas cannot contract such an fma into the following packed
+// add, which it does with a packed multiply. nS holds -S per block, so
+// fma(v, -S, z) = -yhat and d = y + (-yhat).
+#ifndef FP4Q_CAND_SCALAR
+#define FP4Q_CAND_SCALAR 0
+#endif
+
+template <int B>
+__host__ __device__ constexpr int blocks_per_word() { return B < 8 ? 8 / B : 1; }
+
+// Words w and w + 2 of candidate_seg: rl / rh and nSl / nSh hold r and -S of
+// the blocks that word w and word w + 2 touch (8 / B blocks each for B <= 8,
+// else the one block each). Returns their codes qa, qb and, with WANT_SSE,
+// the block SSEs el / eh for B <= 8, or for B >= 16 the packed partial sum
+// P = {sum over word w, sum over word w + 2} (tree levels up to 8 elements).
+template <int B, bool FOLD, bool WANT_SSE>
+__device__ __forceinline__ void candidate_wp(const float (&t)[SEG], int w,
+                                             const float (&rl)[blocks_per_word<B>()],
+                                             const float (&rh)[blocks_per_word<B>()],
+                                             const float (&nSl)[blocks_per_word<B>()],
+                                             const float (&nSh)[blocks_per_word<B>()], float kf,
+                                             uint32_t keep, uint32_t& qa, uint32_t& qb,
+                                             float (&el)[blocks_per_word<B>()],
+                                             float (&eh)[blocks_per_word<B>()], f32x2& P)
+{
+    constexpr int G = B < 8 ? B : 8;  // tree width inside one word
+    const float z = __uint_as_float(~keep);
+    const f32x2 Z = pk2(z, z);
+    float ua[8], ub[8];
+#if FP4Q_CAND_SCALAR
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int i = 8 * w + j;
+        ua[j] = __fmul_rn(t[i], rl[j / G]);
+        ub[j] = __fmul_rn(t[i + 16], rh[j / G]);
+    }
+#else
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int i = 8 * w + j;
+        upk2(mul2(pk2(t[i], t[i + 16]), pk2(rl[j / G], rh[j / G])), ua[j], ub[j]);
+    }
+#endif
+    qa = e2m1_pack8(ua) & keep;  // see encode_seg on `keep`
+    qb = e2m1_pack8(ub) & keep;
+#if FP4Q_CAND_SCALAR
+    if constexpr (WANT_SSE) {
+        float va[8], vb[8], ea[8], eb[8];
+        e2m1_unpack8(qa, va);
+        e2m1_unpack8(qb, vb);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;
+            const float ya = FOLD ? __fmul_rn(t[i], kf) : t[i];
+            const float yb = FOLD ? __fmul_rn(t[i + 16], kf) : t[i + 16];
+            const float da = __fadd_rn(ya, __fmul_rn(va[j], nSl[j / G]));
+            const float db = __fadd_rn(yb, __fmul_rn(vb[j], nSh[j / G]));
+            ea[j] = __fmul_rn(da, da);
+            eb[j] = __fmul_rn(db, db);
+        }
+#pragma unroll
+        for (int h = 1; h < G; h <<= 1)
+#pragma unroll
+            for (int j = 0; j + h < 8; j += 2 * h) {
+                ea[j] = __fadd_rn(ea[j], ea[j + h]);
+                eb[j] = __fadd_rn(eb[j], eb[j + h]);
+            }
+        if constexpr (B <= 8) {
+#pragma unroll
+            for (int k = 0; k < 8 / B; ++k) {
+                el[k] = ea[k * B];
+                eh[k] = eb[k * B];
+            }
+        } else {
+            P = pk2(ea[0], eb[0]);
+        }
+    }
+    return;
+#endif
+    if constexpr (WANT_SSE) {
+        float va[8], vb[8];
+        e2m1_unpack8(qa, va);
+        e2m1_unpack8(qb, vb);
+        f32x2 E[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int i = 8 * w + j;
+            const f32x2 NY = fma2(pk2(va[j], vb[j]), pk2(nSl[j / G], nSh[j / G]), Z);
+            const f32x2 T = pk2(t[i], t[i + 16]);
+            const f32x2 D = FOLD ? fma2(T, pk2(kf, kf), NY) : add2(T, NY);
+            E[j] = fma2(D, D, Z);
+        }
+#pragma unroll
+        for (int h = 1; h < G; h <<= 1)
+#pragma unroll
+            for (int j = 0; j + h < 8; j += 2 * h)
+                E[j] = add2(E[j], E[j + h]);
+        if constexpr (B <= 8) {
+#pragma unroll
+            for (int k = 0; k < 8 / B; ++k)
+                upk2(E[k * B], el[k], eh[k]);
+        } else {
+            P = E[0];
+        }
+    }
+}
+
+template <int B, bool FOLD, bool WANT_SSE>
+__device__ __forceinline__ void candidate_seg(const float (&t)[SEG], const float (&r)[SEG / B],
+                                              const float (&nS)[SEG / B], float kf, uint32_t keep,
+                                              uint32_t (&q)[4], float (&sse)[SEG / B])
+{
+    constexpr int KB = blocks_per_word<B>();
+    f32x2 W[2];
+#pragma unroll
+    for (int w = 0; w < 2; ++w) {
+        float rl[KB], rh[KB], nl[KB], nh[KB], el[KB], eh[KB];
+#pragma unroll
+        for (int k = 0; k < KB; ++k) {
+            rl[k] = r[(8 * w + k * B) / B];
+            rh[k] = r[(8 * w + 16 + k * B) / B];
+            nl[k] = nS[(8 * w + k * B) / B];
+            nh[k] = nS[(8 * w + 16 + k * B) / B];
+        }
+        candidate_wp<B, FOLD, WANT_SSE>(t, w, rl, rh, nl, nh, kf, keep, q[w], q[w + 2], el, eh, W[w]);
+        if constexpr (WANT_SSE && B <= 8) {
+#pragma unroll
+            for (int k = 0; k < KB; ++k) {
+                sse[(8 * w + k * B) / B] = el[k];
+                sse[(8 * w + 16 + k * B) / B] = eh[k];
+            }
+        }
+    }
+    if constexpr (WANT_SSE && B >= 16) {
+        const f32x2 P = add2(W[0], W[1]);
+        if constexpr (B == 16) {
+            upk2(P, sse[0], sse[1]);
+        } else {
+            float lo, hi;
+            upk2(P, lo, hi);
+            sse[0] = __fadd_rn(lo, hi);
+        }
+    }
 }
 
 // SSE of one B-wide block yb against value(RNE_E2M1(yb * r)) * S (`keep` as

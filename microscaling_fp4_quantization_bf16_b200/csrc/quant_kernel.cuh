@@ -24,15 +24,23 @@
 namespace fp4q {
 
 // CTA shape of the direct-load kernel: 128 threads (one segment each). The
-// MXFP4 kernels are also asked to fit 10 CTAs (40 warps) per SM, which caps
-// them at 48 registers, the NVFP4 ones (brute force aside) 7 CTAs (72
-// registers); all measured faster on B200 than 256-thread CTAs at the
-// registers the compiler picks unconstrained.
+// MXFP4 kernels are also asked to fit 9 CTAs (36 warps) per SM, which caps
+// them at 56 registers (at 10 CTAs they spill and ran 5% slower), the NVFP4
+// ones (brute force aside) 7 CTAs (72 registers); all measured faster on B200
+// than 256-thread CTAs at the registers the compiler picks unconstrained.
 constexpr int QTHREADS = 128;
+#ifndef FP4Q_MX_MINB
+#define FP4Q_MX_MINB 9
+#endif
+#ifndef FP4Q_NV_MINB
+#define FP4Q_NV_MINB 7
+#endif
 template <int STRAT>
 struct QMinBlocks {
     static constexpr int value =
-        STRAT == K_MX ? 10 : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE || STRAT == K_UE_BRUTE_FORCE ? 1 : 7);
+        STRAT == K_MX ? FP4Q_MX_MINB
+                      : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE || STRAT == K_UE_BRUTE_FORCE ? 1
+                                                                                              : FP4Q_NV_MINB);
 };
 
 // Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
@@ -100,67 +108,55 @@ __device__ __forceinline__ void brute_search(const float* yb, float amax, int c6
     best_out = best;
 }
 
-// 4-over-6 choice for a whole segment: q, sc, S hold the target-6 result;
-// the target-4 candidate (c4, S4, r4, z4) is encoded, both block SSEs are
-// computed, and target 4 is kept only where its SSE is strictly lower.
-template <int B>
-__device__ __forceinline__ void choose_four_over_six(const float (&y)[SEG], uint32_t (&q)[4],
-                                                     uint32_t (&sc)[SEG / B], float (&S)[SEG / B],
-                                                     float (&sse)[SEG / B], const uint32_t (&c4)[SEG / B],
-                                                     const float (&S4)[SEG / B], const float (&r4)[SEG / B],
-                                                     const bool (&z4)[SEG / B], uint32_t keep)
+// Rotations whose factor k = 1/sqrt(n) is a power of two (16: 2^-2, 64:
+// 2^-3) are applied unscaled and k is folded into the encode and the error
+// (candidate_seg) for the strategies that take that path.
+// MXFP4 abs-max folds k for every rotation width: its scale 2^e is a power of
+// two, so fl(fl(t k) 2^-e) = fl(t (k 2^-e)) whenever k 2^-e is a normal
+// float (a product that underflows rounds to a signed zero code either way);
+// that path writes codes only (the SSE needs fl(t k) itself).
+template <int ROT, int STRAT>
+__host__ __device__ constexpr bool foldable()
 {
-    constexpr int NB = SEG / B;
-    float sse4[NB];
-    uint32_t q4w[4];
-    encode_seg<B, B == 32>(y, r4, z4, keep, q4w);
-    sse_seg<B>(y, q, S, sse);
-    sse_seg<B>(y, q4w, S4, sse4);
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        uint32_t m = 0;
-#pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (sse4[(8 * w + j) / B] < sse[(8 * w + j) / B])
-                m |= 0xFu << (4 * j);
-        q[w] = (q[w] & ~m) | (q4w[w] & m);
-    }
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-        if (sse4[b] < sse[b]) {
-            sc[b] = c4[b];
-            S[b] = S4[b];
-            sse[b] = sse4[b];
-        }
-    }
+    return ((ROT == 16 || ROT == 64) &&
+            (STRAT == K_ABSMAX || STRAT == K_PREVENT_ZERO || STRAT == K_FOUR_OVER_SIX ||
+             STRAT == K_UE_ABSMAX || STRAT == K_UE_PREVENT_ZERO || STRAT == K_UE_FOUR_OVER_SIX)) ||
+           (ROT > 0 && STRAT == K_MX);
+}
+
+template <int ROT>
+__host__ __device__ constexpr float had_k()
+{
+    if constexpr (ROT == 0)
+        return 1.0f;
+    else
+        return HadK<ROT>::k;
 }
 
 // Scale selection, encoding and stores for one 32-element segment s whose
-// (rotated) values are y. nvalid < 32 only for the last segment.
-template <int B, int STRAT>
-__device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s, int nvalid,
+// (rotated) values are y -- before the multiply by k_ROT when
+// foldable<ROT, STRAT>() (rotate_seg<ROT, false>). nvalid < 32 only for the
+// last segment.
+template <int B, int STRAT, int ROT>
+__device__ __forceinline__ void process_segment(float (&y)[SEG], int64_t s, int nvalid,
                                                 const QuantArgs& a, const ScaleTables<STRAT>& tab)
 {
     constexpr int NB = SEG / B;
+    constexpr bool FOLDABLE = foldable<ROT, STRAT>();
     float amax[NB];
     block_amax<B>(y, amax);
+    if constexpr (FOLDABLE) {
+        // max |fl(k t)| = fl(k max |t|): rounding is monotone (exact here anyway)
+#pragma unroll
+        for (int b = 0; b < NB; ++b)
+            amax[b] = __fmul_rn(amax[b], had_k<ROT>());
+    }
 
     float S[NB], r[NB], sse[NB];
     bool zero[NB];
     uint32_t sc[NB], q[4];
-    bool have_sse = false;
 
-    if constexpr (STRAT == K_MX) {
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            const int e = e8m0_exp(amax[b]);
-            sc[b] = (uint32_t)(e + 127);
-            S[b] = pow2f(e);
-            r[b] = __uint_as_float((uint32_t)(127 - e) << 23);  // 2^-e, exact
-            zero[b] = false;
-        }
-        encode_seg<B, true>(y, r, zero, a.keep, q);  // packed: measured faster here
-    } else if constexpr (STRAT == K_MX_BRUTE) {
+    if constexpr (STRAT == K_MX_BRUTE) {
         // MXFP4 MSE-optimised scale: every E8M0 byte 0..254 (S = 2^(byte -
         // 127)), searched like the NVFP4 brute force below -- upward from the
         // abs-max byte - 1, stopped by block_zero_lb (checked from abs-max + 2),
@@ -207,7 +203,6 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
         zero[0] = false;
         sse[0] = best;
         encode_seg<B, true>(y, r, zero, a.keep, q);
-        have_sse = true;
     } else if constexpr (STRAT == K_BRUTE_FORCE) {
         // Exact search with pruning (brute_search), from the abs-max code c6.
         const NvConsts k = tab.k;
@@ -231,166 +226,190 @@ __device__ __forceinline__ void process_segment(const float (&y)[SEG], int64_t s
             sse[b] = best;
         });
         encode_seg<B>(y, r, zero, a.keep, q);
-        have_sse = true;
-    } else if constexpr (is_ue_strat(STRAT)) {
-        // UE5M3 scales, no global scale: the candidate code of target T is
-        // RNE_UE5M3(amax / T) -- one IEEE division for T = 6; for T = 4 the
-        // product by 0.25 is the same correctly rounded quotient.
+    } else if constexpr (STRAT == K_UE_BRUTE_FORCE) {
+        // UE5M3 scales, no global scale: the abs-max code is RNE_UE5M3(amax / 6)
+        // (one IEEE division), then the exact search.
         uint32_t c6[NB];
 #pragma unroll
         for (int b = 0; b < NB; ++b)
             c6[b] = ue5m3_enc(__fdiv_rn(amax[b], 6.0f));
-        if constexpr (STRAT == K_UE_BRUTE_FORCE) {
-            static_for<NB>([&](auto bi) {
-                constexpr int b = decltype(bi)::value;
-                int bc;
-                float best;
-                brute_search<B, 0xFE>(y + b * B, amax[b], (int)c6[b], tab, a.keep, bc, best);
-                sc[b] = (uint32_t)bc;
-                S[b] = tab.S[bc];
-                r[b] = tab.R[bc];
-                zero[b] = (S[b] == 0.0f);
-                sse[b] = best;
-            });
-            encode_seg<B>(y, r, zero, a.keep, q);
-            have_sse = true;
-        } else {
+        static_for<NB>([&](auto bi) {
+            constexpr int b = decltype(bi)::value;
+            int bc;
+            float best;
+            brute_search<B, 0xFE>(y + b * B, amax[b], (int)c6[b], tab, a.keep, bc, best);
+            sc[b] = (uint32_t)bc;
+            S[b] = tab.S[bc];
+            r[b] = tab.R[bc];
+            zero[b] = (S[b] == 0.0f);
+            sse[b] = best;
+        });
+        encode_seg<B>(y, r, zero, a.keep, q);
+    } else {
+        // Abs-max, prevent-zero and 4-over-6 (E4M3 under s_g, or UE5M3), and
+        // MXFP4 abs-max: the candidate scale code(s) of each block -- target 6,
+        // and target 4 for 4-over-6 -- then one fused encode (+ SSE) per
+        // candidate (candidate_seg); 4-over-6 keeps target 4 only where its
+        // block SSE is strictly lower.
+        constexpr bool UE = is_ue_strat(STRAT);
+        constexpr bool MX = STRAT == K_MX;
+        constexpr bool FOUR = STRAT == K_FOUR_OVER_SIX || STRAT == K_UE_FOUR_OVER_SIX;
+        constexpr bool PZ = STRAT == K_PREVENT_ZERO || STRAT == K_UE_PREVENT_ZERO;
+        constexpr int NC = FOUR ? 2 : 1;
+        uint32_t cc[NC][NB];  // [0]: target 6 (or the E8M0 byte), [1]: target 4
+        if constexpr (MX) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+                cc[0][b] = (uint32_t)(e8m0_exp(amax[b]) + 127);
+        } else if constexpr (UE) {
+            // RNE_UE5M3(amax / T): one IEEE division for T = 6; for T = 4 the
+            // product by 0.25 is the same correctly rounded quotient.
 #pragma unroll
             for (int b = 0; b < NB; ++b) {
-                uint32_t c = c6[b];
-                if constexpr (STRAT == K_UE_PREVENT_ZERO)
-                    c = max(c, 1u);
-                sc[b] = c;
-                S[b] = tab.S[c];
-                r[b] = tab.R[c];
-                zero[b] = (S[b] == 0.0f);
+                cc[0][b] = ue5m3_enc(__fdiv_rn(amax[b], 6.0f));
+                if constexpr (FOUR)
+                    cc[NC - 1][b] = ue5m3_enc(__fmul_rn(amax[b], 0.25f));
             }
-            encode_seg<B, B == 32>(y, r, zero, a.keep, q);
-            if constexpr (STRAT == K_UE_FOUR_OVER_SIX) {
-                uint32_t c4[NB];
-                float S4[NB], r4[NB];
-                bool z4[NB];
+        } else {
+            const NvConsts k = tab.k;
+            float qa[NC * NB], qd[NC * NB], qr[NC * NB];
+            uint32_t qc[NC * NB];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                qa[b] = amax[b];
+                qd[b] = k.den6;
+                qr[b] = k.rden6;
+                if constexpr (FOUR) {
+                    qa[NB + b] = amax[b];
+                    qd[NB + b] = k.den4;
+                    qr[NB + b] = k.rden4;
+                }
+            }
+            e4m3_quotient_codes<NC * NB>(qa, qd, qr, k.fast, qc);
+#pragma unroll
+            for (int c = 0; c < NC; ++c)
+#pragma unroll
+                for (int b = 0; b < NB; ++b)
+                    cc[c][b] = qc[c * NB + b];
+        }
+        if constexpr (PZ) {
+#pragma unroll
+            for (int b = 0; b < NB; ++b)
+                cc[0][b] = max(cc[0][b], 1u);
+        }
+        // scale and reciprocal of candidate code c
+        auto scale_of = [&](uint32_t c) -> float { return MX ? pow2f((int)c - 127) : tab.S[c]; };
+        auto rcp_of = [&](uint32_t c) -> float {
+            return MX ? __uint_as_float((254u - c) << 23) : tab.R[c];  // MXFP4: 2^-e, exact
+        };
+        const bool want = FOUR || a.mse != nullptr;
+
+        auto run = [&](auto fold_c) {
+            constexpr bool FOLD = decltype(fold_c)::value;
+            constexpr float kf = FOLD ? had_k<ROT>() : 1.0f;
+            if constexpr (B <= 8) {
+                // Blocks lie inside words: decide one word pair at a time.
+                constexpr int KB = 8 / B;
+                static_for<2>([&](auto wi) {
+                    constexpr int w = decltype(wi)::value;
+                    float rl[NC][KB], rh[NC][KB], nl[NC][KB], nh[NC][KB];
+                    float el[NC][KB] = {}, eh[NC][KB] = {};
+                    uint32_t qa[NC], qb[NC];
+                    f32x2 unused;
+#pragma unroll
+                    for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                        for (int k = 0; k < KB; ++k) {
+                            const uint32_t cl = cc[c][w * KB + k], ch = cc[c][(w + 2) * KB + k];
+                            rl[c][k] = __fmul_rn(rcp_of(cl), kf);
+                            rh[c][k] = __fmul_rn(rcp_of(ch), kf);
+                            nl[c][k] = -scale_of(cl);
+                            nh[c][k] = -scale_of(ch);
+                        }
+                        if (want)
+                            candidate_wp<B, FOLD, true>(y, w, rl[c], rh[c], nl[c], nh[c], kf, a.keep,
+                                                        qa[c], qb[c], el[c], eh[c], unused);
+                        else
+                            candidate_wp<B, FOLD, false>(y, w, rl[c], rh[c], nl[c], nh[c], kf,
+                                                         a.keep, qa[c], qb[c], el[c], eh[c], unused);
+                    }
+                    uint32_t ml = 0, mh = 0, zl = 0, zh = 0;
+                    constexpr uint32_t BM = B == 4 ? 0xFFFFu : 0xFFFFFFFFu;  // nibbles of one block
+#pragma unroll
+                    for (int k = 0; k < KB; ++k) {
+                        const bool fl = FOUR && el[NC - 1][k] < el[0][k];
+                        const bool fh = FOUR && eh[NC - 1][k] < eh[0][k];
+                        const int bl = w * KB + k, bh = (w + 2) * KB + k;
+                        sc[bl] = fl ? cc[NC - 1][bl] : cc[0][bl];
+                        sc[bh] = fh ? cc[NC - 1][bh] : cc[0][bh];
+                        S[bl] = -(fl ? nl[NC - 1][k] : nl[0][k]);
+                        S[bh] = -(fh ? nh[NC - 1][k] : nh[0][k]);
+                        sse[bl] = fl ? el[NC - 1][k] : el[0][k];
+                        sse[bh] = fh ? eh[NC - 1][k] : eh[0][k];
+                        ml |= fl ? BM << (4 * B * k) : 0u;
+                        mh |= fh ? BM << (4 * B * k) : 0u;
+                        zl |= S[bl] == 0.0f ? BM << (4 * B * k) : 0u;
+                        zh |= S[bh] == 0.0f ? BM << (4 * B * k) : 0u;
+                    }
+                    q[w] = ((qa[0] & ~ml) | (qa[NC - 1] & ml)) & ~zl;
+                    q[w + 2] = ((qb[0] & ~mh) | (qb[NC - 1] & mh)) & ~zh;
+                });
+            } else {
+                float rr[NC][NB], nS[NC][NB], se[NC][NB] = {};
+                uint32_t qc[NC][4];
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+#pragma unroll
+                    for (int b = 0; b < NB; ++b) {
+                        rr[c][b] = __fmul_rn(rcp_of(cc[c][b]), kf);
+                        nS[c][b] = -scale_of(cc[c][b]);
+                    }
+                    if (want)
+                        candidate_seg<B, FOLD, true>(y, rr[c], nS[c], kf, a.keep, qc[c], se[c]);
+                    else
+                        candidate_seg<B, FOLD, false>(y, rr[c], nS[c], kf, a.keep, qc[c], se[c]);
+                }
+                bool four[NB];
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
-                    c4[b] = ue5m3_enc(__fmul_rn(amax[b], 0.25f));
-                    S4[b] = tab.S[c4[b]];
-                    r4[b] = tab.R[c4[b]];
-                    z4[b] = (S4[b] == 0.0f);
+                    four[b] = FOUR && se[NC - 1][b] < se[0][b];
+                    sc[b] = four[b] ? cc[NC - 1][b] : cc[0][b];
+                    S[b] = -(four[b] ? nS[NC - 1][b] : nS[0][b]);
+                    sse[b] = four[b] ? se[NC - 1][b] : se[0][b];
                 }
-                choose_four_over_six<B>(y, q, sc, S, sse, c4, S4, r4, z4, a.keep);
-                have_sse = true;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    uint32_t m4 = 0, mz = 0;  // nibbles taken from target 4; of zero scales
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const int b = (8 * w + j) / B;
+                        if (four[b])
+                            m4 |= 0xFu << (4 * j);
+                        if (!MX && S[b] == 0.0f)
+                            mz |= 0xFu << (4 * j);
+                    }
+                    q[w] = ((qc[0][w] & ~m4) | (qc[NC - 1][w] & m4)) & ~mz;
+                }
             }
-        }
-    } else if constexpr (STRAT == K_FOUR_OVER_SIX && B <= 8) {
-        // 4-over-6 for blocks of 4 or 8, one half segment (words w and w + 2)
-        // at a time, so the candidates' temporaries of only half the blocks
-        // are live at once. Same operations as the segment form below.
-        const NvConsts k = tab.k;
-        float qa[2 * NB], qd[2 * NB], qr[2 * NB];
-        uint32_t qc[2 * NB];
+        };
+        bool fold = false;
+        if constexpr (FOLDABLE) {
+            if constexpr (MX) {
+                fold = a.mse == nullptr;
 #pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            qa[b] = amax[b];
-            qd[b] = k.den6;
-            qr[b] = k.rden6;
-            qa[NB + b] = amax[b];
-            qd[NB + b] = k.den4;
-            qr[NB + b] = k.rden4;
-        }
-        e4m3_quotient_codes<2 * NB>(qa, qd, qr, k.fast, qc);
-        constexpr int KB = 8 / B;  // blocks per word
-        static_for<2>([&](auto wi) {
-            constexpr int w = decltype(wi)::value;
-            constexpr int bl = 8 * w / B, bh = (8 * w + 16) / B;  // first block of each word
-            float S6l[KB], S6h[KB], S4l[KB], S4h[KB], r6l[KB], r6h[KB], r4l[KB], r4h[KB];
-            uint32_t z6l = 0, z6h = 0, z4l = 0, z4h = 0;
-            constexpr uint32_t BM = B == 4 ? 0xFFFFu : 0xFFFFFFFFu;  // nibbles of one block
-#pragma unroll
-            for (int t = 0; t < KB; ++t) {
-                S6l[t] = tab.S[qc[bl + t]];
-                r6l[t] = tab.R[qc[bl + t]];
-                S6h[t] = tab.S[qc[bh + t]];
-                r6h[t] = tab.R[qc[bh + t]];
-                S4l[t] = tab.S[qc[NB + bl + t]];
-                r4l[t] = tab.R[qc[NB + bl + t]];
-                S4h[t] = tab.S[qc[NB + bh + t]];
-                r4h[t] = tab.R[qc[NB + bh + t]];
-                z6l |= S6l[t] == 0.0f ? BM << (4 * B * t) : 0u;
-                z6h |= S6h[t] == 0.0f ? BM << (4 * B * t) : 0u;
-                z4l |= S4l[t] == 0.0f ? BM << (4 * B * t) : 0u;
-                z4h |= S4h[t] == 0.0f ? BM << (4 * B * t) : 0u;
+                for (int b = 0; b < NB; ++b)
+                    fold = fold && cc[0][b] <= 127 + 122;  // k 2^-e stays normal
+            } else {
+                fold = UE || tab.k.fold;
             }
-            uint32_t q6l, q6h, q4l, q4h;
-            encode_word_pair<B>(y, w, r6l, r6h, z6l, z6h, a.keep, q6l, q6h);
-            encode_word_pair<B>(y, w, r4l, r4h, z4l, z4h, a.keep, q4l, q4h);
-            float e6l[KB], e6h[KB], e4l[KB], e4h[KB];
-            sse_word_pair<B>(y, w, q6l, q6h, S6l, S6h, e6l, e6h);
-            sse_word_pair<B>(y, w, q4l, q4h, S4l, S4h, e4l, e4h);
-            uint32_t ml = 0, mh = 0;
-#pragma unroll
-            for (int t = 0; t < KB; ++t) {
-                const bool fl = e4l[t] < e6l[t], fh = e4h[t] < e6h[t];
-                ml |= fl ? BM << (4 * B * t) : 0u;
-                mh |= fh ? BM << (4 * B * t) : 0u;
-                sc[bl + t] = fl ? qc[NB + bl + t] : qc[bl + t];
-                S[bl + t] = fl ? S4l[t] : S6l[t];
-                sse[bl + t] = fl ? e4l[t] : e6l[t];
-                sc[bh + t] = fh ? qc[NB + bh + t] : qc[bh + t];
-                S[bh + t] = fh ? S4h[t] : S6h[t];
-                sse[bh + t] = fh ? e4h[t] : e6h[t];
-            }
-            q[w] = (q6l & ~ml) | (q4l & ml);
-            q[w + 2] = (q6h & ~mh) | (q4h & mh);
-        });
-        have_sse = true;
-    } else {
-        // Scale codes of the targets in use: 6, and 4 for 4-over-6.
-        const NvConsts k = tab.k;
-        constexpr bool FOUR = STRAT == K_FOUR_OVER_SIX;
-        constexpr int NQ = FOUR ? 2 * NB : NB;
-        float qa[NQ], qd[NQ], qr[NQ];
-        uint32_t qc[NQ];
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            qa[b] = amax[b];
-            qd[b] = k.den6;
-            qr[b] = k.rden6;
-            if constexpr (FOUR) {
-                qa[NB + b] = amax[b];
-                qd[NB + b] = k.den4;
-                qr[NB + b] = k.rden4;
-            }
+            if (!fold)
+                scale_seg<ROT>(y);
         }
-        e4m3_quotient_codes<NQ>(qa, qd, qr, k.fast, qc);
-#pragma unroll
-        for (int b = 0; b < NB; ++b) {
-            uint32_t c = qc[b];
-            if constexpr (STRAT == K_PREVENT_ZERO)
-                c = max(c, 1u);
-            sc[b] = c;
-            S[b] = tab.S[c];
-            r[b] = tab.R[c];
-            zero[b] = (S[b] == 0.0f);
-        }
-        encode_seg<B, B == 32>(y, r, zero, a.keep, q);  // packed measured faster for B = 32 only
-        if constexpr (FOUR) {
-            float S4[NB], r4[NB];
-            bool z4[NB];
-            uint32_t c4[NB];
-#pragma unroll
-            for (int b = 0; b < NB; ++b) {
-                c4[b] = qc[NB + b];
-                S4[b] = tab.S[c4[b]];
-                r4[b] = tab.R[c4[b]];
-                z4[b] = (S4[b] == 0.0f);
-            }
-            choose_four_over_six<B>(y, q, sc, S, sse, c4, S4, r4, z4, a.keep);
-            have_sse = true;
-        }
+        if (fold)
+            run(std::integral_constant<bool, true>{});
+        else
+            run(std::integral_constant<bool, false>{});
     }
-
-    if (a.mse != nullptr && !have_sse)
-        sse_seg<B>(y, q, S, sse);
 
     float m[NB];
 #pragma unroll
@@ -489,9 +508,91 @@ __global__ void __launch_bounds__(QTHREADS, QMinBlocks<STRAT>::value) quant_kern
 
     float y[SEG];
     unpack_seg(raw, y);
-    rotate_seg<ROT>(y, lane);  // all 32 lanes take part; past the end holds zeros
+    // all 32 lanes take part; past the end holds zeros
+    rotate_seg<ROT, !foldable<ROT, STRAT>()>(y, lane);
     if (s < nseg)
-        process_segment<B, STRAT>(y, s, (int)min((int64_t)SEG, a.n - s * SEG), a, tab);
+        process_segment<B, STRAT, ROT>(y, s, (int)min((int64_t)SEG, a.n - s * SEG), a, tab);
+}
+
+// Persistent form of the direct-load kernel for the one-pass strategies (the
+// searches keep quant_kernel: their registers go to the search). A grid of
+// resident CTAs walks tiles of QTHREADS segments (tile t covers segments
+// t * QTHREADS ..); as soon as a thread has unpacked its segment of the
+// current tile it issues the loads of its segment in the next tile into the
+// same registers, so their latency overlaps this tile's arithmetic, and each
+// CTA builds its scale tables once.
+#ifndef FP4Q_PERSIST
+#define FP4Q_PERSIST 1
+#endif
+#ifndef FP4Q_MXP_MINB
+#define FP4Q_MXP_MINB 6
+#endif
+#ifndef FP4Q_NVP_MINB
+#define FP4Q_NVP_MINB 5
+#endif
+template <int STRAT>
+struct PMinBlocks {
+    static constexpr int value = STRAT == K_MX ? FP4Q_MXP_MINB : FP4Q_NVP_MINB;
+};
+
+template <int STRAT>
+__host__ __device__ constexpr bool use_persist()
+{
+    return FP4Q_PERSIST && STRAT != K_BRUTE_FORCE && STRAT != K_MX_BRUTE && STRAT != K_UE_BRUTE_FORCE &&
+           STRAT != K_MX;  // measured: MXFP4 runs faster at the one-shot kernel's occupancy
+}
+
+template <int B, int ROT, int STRAT>
+__global__ void __launch_bounds__(QTHREADS, PMinBlocks<STRAT>::value)
+    quant_persist_kernel(QuantArgs a, int64_t ntiles)
+{
+    pdl_begin();
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = a.n / SEG;  // every segment is whole (checked by the launcher)
+    const int64_t step = (int64_t)gridDim.x * QTHREADS;
+    const uint4* x4 = reinterpret_cast<const uint4*>(a.x);
+    // segment s's four 128-bit words, or zeros past the end
+    auto fetch = [&](int64_t s, uint4 (&raw)[4]) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            raw[k] = s < nseg ? ldg_stream(x4 + 4 * s + k) : make_uint4(0u, 0u, 0u, 0u);
+    };
+    uint4 raw[4];
+    int64_t s = (int64_t)blockIdx.x * QTHREADS + threadIdx.x;
+    fetch(s, raw);  // in flight while the tables are built
+    __shared__ ScaleTables<STRAT> tab;
+    build_scale_tables<STRAT>(tab, a);
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, s += step) {
+        float y[SEG];
+        unpack_seg(raw, y);
+        if (t + gridDim.x < ntiles)
+            fetch(s + step, raw);  // next tile's loads overlap this tile's arithmetic
+        if (s - lane < nseg) {     // warp-uniform
+            // all 32 lanes take part; past the end holds zeros
+            rotate_seg<ROT, !foldable<ROT, STRAT>()>(y, lane);
+            if (s < nseg)
+                process_segment<B, STRAT, ROT>(y, s, SEG, a, tab);
+        }
+    }
+}
+
+// Resident CTAs per SM of a kernel (queried once per process) times the SM
+// count of the current device.
+template <typename K>
+int64_t resident_ctas(K kernel)
+{
+    static int per_sm = 0;
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    if (per_sm == 0) {
+        int v = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, kernel, QTHREADS, 0) != cudaSuccess)
+            return -1;
+        per_sm = v < 1 ? 1 : v;
+    }
+    return (int64_t)sms * per_sm;
 }
 
 template <int B>
@@ -500,10 +601,19 @@ cudaError_t launch_quant_impl(int strat, int rot, const QuantArgs& a, cudaStream
     const int64_t nseg = (a.n + SEG - 1) / SEG;
 #define FP4Q_QCASE(S_, R_)                                                              \
     if (strat == S_ && rot == R_) {                                                     \
-        constexpr int64_t per_block = (int64_t)QTHREADS;                     \
-        const int64_t nblk = (nseg + per_block - 1) / per_block;                        \
+        const int64_t nblk = (nseg + QTHREADS - 1) / QTHREADS;                          \
         if (nblk <= 0 || nblk > 0x7FFFFFFF)                                             \
             return cudaErrorInvalidValue;                                               \
+        if constexpr (use_persist<S_>()) {                                              \
+          if (a.n % SEG == 0) {                                                         \
+            const int64_t res = resident_ctas(quant_persist_kernel<B, R_, S_>);         \
+            if (res < 0)                                                                \
+                return cudaErrorUnknown;                                                \
+            const int64_t grid = nblk < res ? nblk : res;                               \
+            return launch_pdl(quant_persist_kernel<B, R_, S_>, dim3((unsigned)grid), dim3(QTHREADS), 0, \
+                              st, a, nblk);                                             \
+          }                                                                             \
+        }                                                                               \
         return launch_pdl(quant_kernel<B, R_, S_>, dim3((unsigned)nblk), dim3(QTHREADS), 0, st, a); \
     }
 #define FP4Q_QROTS(S_)      \

@@ -161,10 +161,11 @@ __global__ void __launch_bounds__(TTHREADS)
             y[8 * k + 6] = bf_lo(v[k].w);
             y[8 * k + 7] = bf_hi(v[k].w);
         }
-        rotate_seg<ROT>(y, lane);  // 64/128-wide chunks: neighbouring lanes of this warp
+        // 64/128-wide chunks: neighbouring lanes of this warp
+        rotate_seg<ROT, !foldable<ROT, STRAT>()>(y, lane);
         const int64_t s = tile * TILE_SEGS + c;
         if (s < nseg)  // rows past the end were zero-filled by TMA
-            process_segment<B, STRAT>(y, s, SEG, a, tab);
+            process_segment<B, STRAT, ROT>(y, s, SEG, a, tab);
     }
 }
 
