@@ -31,10 +31,22 @@
  * Conventions for every entry point:
  *  - All array pointers are DEVICE pointers owned by the caller, 16-byte
  *    aligned, dense row-major (leading dimension = cols). The library never
- *    allocates, frees, or keeps memory or state between calls (the one
- *    exception is the fixed scratch float of fp4q_gemm_noalloc), and never
- *    synchronises: work is enqueued on `stream` (0 = legacy default stream)
- *    and the call returns before it completes.
+ *    allocates or frees memory and never synchronises (fp4q_device_errors
+ *    aside): work is enqueued on `stream` (0 = legacy default stream) and
+ *    the call returns before it completes.
+ *  - State the library keeps between calls, all of it listed here:
+ *      * a per-device error counter in device memory (fp4q_device_errors);
+ *      * the CUDA error code of the last failed launch, per host thread
+ *        (fp4q_last_cuda_error);
+ *      * the 256-byte scratch array of fp4q_gemm_noalloc, one per device, and
+ *        its device address, cached per device ordinal on first use;
+ *      * host-side caches of launch facts that do not change while the
+ *        process runs: the driver's tensor-map encoder entry point (TMA
+ *        path) and the resident CTAs per SM of each persistent quantize
+ *        kernel (queried once per kernel);
+ *      * the test hook of fp4q_debug_fail_launches (process-wide);
+ *      * the FP4Q_TMA environment switch, read at every quantize call
+ *        (see fp4q_device_errors).
  *  - Arguments are validated on the host before anything is enqueued; on an
  *    error nothing is launched and outputs are untouched.
  *  - rows == 0 or cols == 0 is an empty tensor: its array pointers may be
@@ -205,8 +217,10 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
  * time on different streams or threads) race on it -- serialise them or use
  * fp4q_gemm; the first call on each device looks the scratch address up
  * (cudaGetSymbolAddress), so make that first call before any stream capture
- * begins. The pages have no counterpart: this is an interface detail. Other
- * arguments, results and errors as fp4q_gemm.
+ * begins. The address is cached for the life of the process: a process
+ * that calls cudaDeviceReset on a device must not call this entry point on
+ * that device afterwards. The pages have no counterpart: this is an
+ * interface detail. Other arguments, results and errors as fp4q_gemm.
  */
 fp4q_status fp4q_gemm_noalloc(const uint8_t* a_codes, const uint8_t* a_mma_scales,
                               const float* a_global_scale, const uint8_t* b_codes,
@@ -390,6 +404,17 @@ const char* fp4q_status_string(fp4q_status s);
 
 /* The cudaError_t of the last FP4Q_ERR_CUDA returned on this host thread. */
 int fp4q_last_cuda_error(void);
+
+/*
+ * Test hook for the CUDA-error path (the pages have no counterpart). While
+ * cuda_error is nonzero, every entry point that would enqueue work validates
+ * its arguments as usual and then, instead of enqueuing anything, returns
+ * FP4Q_ERR_CUDA with cuda_error recorded for fp4q_last_cuda_error: no kernel,
+ * memset or copy is issued and outputs are untouched. 0 restores normal
+ * operation. Process-wide and not synchronised with calls in flight on other
+ * threads; for tests only.
+ */
+void fp4q_debug_fail_launches(int cuda_error);
 
 /*
  * Pipeline health. The TMA-fed quantize kernel waits on shared-memory

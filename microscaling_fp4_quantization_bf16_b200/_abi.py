@@ -42,6 +42,7 @@ SIGNATURES = {
     "fp4q_gemm": (_i32, [_p, _p, _p, _p, _p, _p, _i64, _i64, _i64, _i32, _p, _p, _i32, _p]),
     "fp4q_status_string": (C.c_char_p, [_i32]),
     "fp4q_last_cuda_error": (_i32, []),
+    "fp4q_debug_fail_launches": (None, [_i32]),
     "fp4q_device_errors": (_i32, []),
 }
 

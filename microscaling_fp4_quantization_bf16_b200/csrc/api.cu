@@ -7,6 +7,8 @@
 #include <cstdlib>
 #include <cstring>
 
+#include <atomic>
+
 #include <cuda.h>
 
 #include "fp4q.h"
@@ -23,6 +25,10 @@ namespace {
 
 thread_local int g_last_cuda_error = 0;
 
+// Test hook (fp4q_debug_fail_launches): a CUDA error code that every entry
+// point reports, after validating its arguments, instead of enqueuing work.
+std::atomic<int> g_injected_error{0};
+
 fp4q_status cuda_status(cudaError_t e)
 {
     if (e == cudaSuccess)
@@ -30,6 +36,9 @@ fp4q_status cuda_status(cudaError_t e)
     g_last_cuda_error = (int)e;
     return FP4Q_ERR_CUDA;
 }
+
+// The injected error of the test hook, or cudaSuccess.
+cudaError_t injected() { return static_cast<cudaError_t>(g_injected_error.load(std::memory_order_relaxed)); }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -191,6 +200,8 @@ fp4q_status quantize_impl(const void* x, int64_t rows, int64_t cols, fp4q_format
         return FP4Q_ERR_ALIGN;
     if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
         return FP4Q_ERR_ALIAS;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     if (n == 0)
         return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
 
@@ -234,6 +245,40 @@ fp4q_status quantize_impl(const void* x, int64_t rows, int64_t cols, fp4q_format
 }
 
 }  // namespace
+
+namespace fp4q {
+
+fp4q_status gemm_args_status(const uint8_t* a_codes, const uint8_t* a_mma_scales,
+                             const float* a_global_scale, const uint8_t* b_codes,
+                             const uint8_t* b_mma_scales, const float* b_global_scale, int64_t M,
+                             int64_t N, int64_t K, int fmt, const void* d, int d_dtype)
+{
+    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
+        return FP4Q_ERR_UNSUPPORTED;
+    if (d_dtype != FP4Q_OUT_F32 && d_dtype != FP4Q_OUT_BF16)
+        return FP4Q_ERR_UNSUPPORTED;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    const int64_t nalign = d_dtype == FP4Q_OUT_F32 ? 4 : 8;  // 16-byte output rows
+    if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || N % nalign != 0 || M > 0x7FFFFFFF ||
+        N > 0x7FFFFFFF || K > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    if (a_codes == nullptr || a_mma_scales == nullptr || b_codes == nullptr ||
+        b_mma_scales == nullptr || d == nullptr)
+        return FP4Q_ERR_NULL;
+    if (nv && (a_global_scale == nullptr || b_global_scale == nullptr))
+        return FP4Q_ERR_NULL;
+    if (!aligned16(a_codes) || !aligned16(a_mma_scales) || !aligned16(b_codes) ||
+        !aligned16(b_mma_scales) || !aligned16(d) ||
+        (nv && (!aligned4(a_global_scale) || !aligned4(b_global_scale))))
+        return FP4Q_ERR_ALIGN;
+    return FP4Q_OK;
+}
+
+cudaError_t injected_launch_error() { return injected(); }
+
+fp4q_status record_cuda_error(cudaError_t e) { return cuda_status(e); }
+
+}  // namespace fp4q
 
 extern "C" {
 
@@ -279,6 +324,8 @@ fp4q_status fp4q_dequantize(const uint8_t* codes, const uint8_t* scales,
         return FP4Q_ERR_NULL;
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     DequantArgs a;
     a.codes = codes;
     a.scales = scales;
@@ -308,6 +355,8 @@ fp4q_status fp4q_dequantize_unrotate(const uint8_t* codes, const uint8_t* scales
         return FP4Q_ERR_NULL;
     if (!aligned16(codes) || !aligned16(scales) || !aligned16(out) || (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     DequantArgs a;
     a.codes = codes;
     a.scales = scales;
@@ -337,6 +386,8 @@ fp4q_status fp4q_scales_to_mma(const uint8_t* scales, int64_t rows, int64_t K, f
         return FP4Q_ERR_SHAPE;
     if (scales == nullptr || mma_scales == nullptr)
         return FP4Q_ERR_NULL;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     return cuda_status(launch_scales_to_mma(scales, rows, K, sfv, mma_scales, stream));
 }
 
@@ -346,24 +397,17 @@ fp4q_status fp4q_gemm(const uint8_t* a_codes, const uint8_t* a_mma_scales,
                       int64_t N, int64_t K, fp4q_format fmt, float* alpha_out, void* d,
                       fp4q_dtype d_dtype, cudaStream_t stream)
 {
-    if (fmt != FP4Q_FMT_NVFP4 && fmt != FP4Q_FMT_MXFP4)
-        return FP4Q_ERR_UNSUPPORTED;
-    if (d_dtype != FP4Q_OUT_F32 && d_dtype != FP4Q_OUT_BF16)
-        return FP4Q_ERR_UNSUPPORTED;
-    const bool nv = fmt == FP4Q_FMT_NVFP4;
-    const int64_t nalign = d_dtype == FP4Q_OUT_F32 ? 4 : 8;  // 16-byte output rows
-    if (M <= 0 || N <= 0 || K <= 0 || K % 32 != 0 || N % nalign != 0 || M > 0x7FFFFFFF ||
-        N > 0x7FFFFFFF || K > 0x7FFFFFFF)
-        return FP4Q_ERR_SHAPE;
-    if (a_codes == nullptr || a_mma_scales == nullptr || b_codes == nullptr ||
-        b_mma_scales == nullptr || alpha_out == nullptr || d == nullptr)
+    fp4q_status st0 = fp4q::gemm_args_status(a_codes, a_mma_scales, a_global_scale, b_codes,
+                                             b_mma_scales, b_global_scale, M, N, K, fmt, d, d_dtype);
+    if (st0 != FP4Q_OK)
+        return st0;
+    if (alpha_out == nullptr)
         return FP4Q_ERR_NULL;
-    if (nv && (a_global_scale == nullptr || b_global_scale == nullptr))
-        return FP4Q_ERR_NULL;
-    if (!aligned16(a_codes) || !aligned16(a_mma_scales) || !aligned16(b_codes) ||
-        !aligned16(b_mma_scales) || !aligned16(d) || !aligned4(alpha_out) ||
-        (nv && (!aligned4(a_global_scale) || !aligned4(b_global_scale))))
+    if (!aligned4(alpha_out))
         return FP4Q_ERR_ALIGN;
+    const bool nv = fmt == FP4Q_FMT_NVFP4;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     fp4q_status st = cuda_status(
         launch_alpha(nv ? a_global_scale : nullptr, nv ? b_global_scale : nullptr, alpha_out, stream));
     if (st != FP4Q_OK)
@@ -399,6 +443,8 @@ fp4q_status fp4q_block_mse(const void* x, const uint8_t* codes, const uint8_t* s
     if (!aligned16(x) || !aligned16(codes) || !aligned16(scales) || !aligned16(block_mse) ||
         (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     MseArgs a;
     a.x = static_cast<const uint16_t*>(x);
     a.codes = codes;
@@ -437,6 +483,8 @@ fp4q_status fp4q_focus_fwd(const void* w, const void* c, int64_t rows, int64_t c
         return FP4Q_ERR_ALIGN;
     if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
         return FP4Q_ERR_ALIAS;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     if (n == 0)
         return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
 
@@ -484,6 +532,8 @@ fp4q_status fp4q_focus_bwd(const void* w, const void* g, const void* c, int64_t 
         return FP4Q_ERR_NULL;
     if (!aligned16(w) || !aligned16(g) || !aligned16(c) || !aligned16(dc))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     FocusBwdArgs a;
     a.w = static_cast<const uint16_t*>(w);
     a.g = static_cast<const uint16_t*>(g);
@@ -550,6 +600,8 @@ fp4q_status fp4q_focus_update(const void* w, const void* g, float* c, void* c_ha
     if (!aligned16(w) || !aligned16(g) || !aligned16(c) || !aligned16(c_half) || !aligned16(m) ||
         !aligned16(v))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     const bool adam = opt == FP4Q_OPT_ADAM;
     FocusUpdateArgs a;
     a.w = static_cast<const uint16_t*>(w);
@@ -592,6 +644,8 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
         return FP4Q_ERR_ALIGN;
     if (nv && global_amax_in != nullptr && global_amax_in == global_scale_out)
         return FP4Q_ERR_ALIAS;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     if (n == 0)
         return nv ? cuda_status(launch_set_one(global_scale_out, stream)) : FP4Q_OK;
 
@@ -646,6 +700,8 @@ fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt
     if (!aligned16(w) || !aligned16(scales) || !aligned16(U) || !aligned16(perm) ||
         !aligned16(work) || !aligned16(codes) || (nv && !aligned4(global_scale)))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     GptqArgs a;
     a.w = static_cast<const uint16_t*>(w);
     a.scales = scales;
@@ -678,6 +734,8 @@ fp4q_status fp4q_global_amax(const void* x, int64_t rows, int64_t cols, int rot,
         return FP4Q_ERR_NULL;
     if (!aligned16(x) || !aligned4(amax_out))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), stream);
     if (e != cudaSuccess || n == 0)
         return cuda_status(e);
@@ -695,6 +753,8 @@ fp4q_status fp4q_e2m1_encode(const float* u, int64_t n, uint8_t* out, cudaStream
         return FP4Q_ERR_NULL;
     if (!aligned16(u) || !aligned16(out))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     return cuda_status(launch_e2m1_encode(u, n, out, stream));
 }
 
@@ -708,6 +768,8 @@ fp4q_status fp4q_e4m3_encode(const float* v, int64_t n, uint8_t* out, cudaStream
         return FP4Q_ERR_NULL;
     if (!aligned16(v) || !aligned16(out))
         return FP4Q_ERR_ALIGN;
+    if (cudaError_t ie = injected())
+        return cuda_status(ie);
     return cuda_status(launch_e4m3_encode(v, n, out, stream));
 }
 
@@ -726,6 +788,8 @@ const char* fp4q_status_string(fp4q_status s)
 }
 
 int fp4q_last_cuda_error(void) { return g_last_cuda_error; }
+
+void fp4q_debug_fail_launches(int cuda_error) { g_injected_error.store(cuda_error); }
 
 int fp4q_device_errors(void)
 {

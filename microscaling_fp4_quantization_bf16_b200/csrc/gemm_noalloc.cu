@@ -17,8 +17,9 @@
 
 namespace {
 
-// Scratch floats of this entry point: alpha needs one; the array is kept small
-// and fixed (256 bytes) and a request above it is rejected.
+// Scratch floats of this entry point: alpha needs one. The array has a fixed
+// size of 256 bytes, and the use is checked against it at compile time (no
+// call can ask for more).
 constexpr int kScratchFloats = 64;
 constexpr int kAlphaFloats = 1;
 static_assert(kAlphaFloats <= kScratchFloats, "scratch too small for alpha");
@@ -30,7 +31,10 @@ std::mutex g_addr_lock;
 float* g_addr[kMaxDevices] = {};
 
 // Device address of the scratch array on the current device, looked up with
-// cudaGetSymbolAddress on the first call per device and cached.
+// cudaGetSymbolAddress on the first call per device and cached for the life
+// of the process. The cache is not invalidated: after cudaDeviceReset the
+// module is loaded again (possibly at another address), so a process that
+// resets a device must not call this entry point on it afterwards.
 cudaError_t scratch_address(float** out)
 {
     int dev = 0;
@@ -60,9 +64,15 @@ extern "C" fp4q_status fp4q_gemm_noalloc(const uint8_t* a_codes, const uint8_t* 
                                          int64_t K, fp4q_format fmt, void* d, fp4q_dtype d_dtype,
                                          cudaStream_t stream)
 {
+    fp4q_status st = fp4q::gemm_args_status(a_codes, a_mma_scales, a_global_scale, b_codes,
+                                            b_mma_scales, b_global_scale, M, N, K, fmt, d, d_dtype);
+    if (st != FP4Q_OK)
+        return st;
+    if (cudaError_t ie = fp4q::injected_launch_error())
+        return fp4q::record_cuda_error(ie);
     float* alpha = nullptr;
-    if (scratch_address(&alpha) != cudaSuccess)
-        return FP4Q_ERR_CUDA;
+    if (cudaError_t e = scratch_address(&alpha))
+        return fp4q::record_cuda_error(e);
     // alpha is written by the first kernel of the call before the GEMM reads it;
     // nothing in the scratch has to start at zero.
     return fp4q_gemm(a_codes, a_mma_scales, a_global_scale, b_codes, b_mma_scales, b_global_scale,

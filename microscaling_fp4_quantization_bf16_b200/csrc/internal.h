@@ -8,7 +8,21 @@
 #include <cuda.h>
 #include <cuda_runtime_api.h>
 
+#include "fp4q.h"
+
 namespace fp4q {
+
+// Host-side helpers of the C-ABI layer (api.cu). gemm_args_status: the
+// argument checks of fp4q_gemm other than alpha_out. injected_launch_error:
+// the error set with fp4q_debug_fail_launches, or cudaSuccess.
+// record_cuda_error: FP4Q_ERR_CUDA with e kept for fp4q_last_cuda_error (or
+// FP4Q_OK for cudaSuccess).
+fp4q_status gemm_args_status(const uint8_t* a_codes, const uint8_t* a_mma_scales,
+                             const float* a_global_scale, const uint8_t* b_codes,
+                             const uint8_t* b_mma_scales, const float* b_global_scale, int64_t M,
+                             int64_t N, int64_t K, int fmt, const void* d, int d_dtype);
+cudaError_t injected_launch_error();
+fp4q_status record_cuda_error(cudaError_t e);
 
 // Launch with programmatic stream serialization (see pdl_begin in
 // fp4q_device.cuh); returns the launch status.

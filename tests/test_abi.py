@@ -239,3 +239,68 @@ def test_header_is_plain_c(tmp_path):
                             "-I" + os.path.dirname(HEADER), "-I" + cuda_inc, "-c", str(f),
                             "-o", str(tmp_path / (name + ".o"))], capture_output=True, text=True)
         assert r.returncode == 0, r.stderr
+
+
+def test_injected_cuda_error_every_entry_point(lib):
+    """The CUDA-error path, host side only: with fp4q_debug_fail_launches set,
+    every entry point that enqueues work validates its (valid) arguments,
+    returns FP4Q_ERR_CUDA with the injected code for fp4q_last_cuda_error,
+    and touches nothing. Host buffers stand in for the device arrays: no
+    kernel, memset or copy may reach them (on a machine without a GPU a
+    CUDA call would fail with a different code)."""
+    import numpy as np
+
+    bufs = [np.full(1 << 16, 0xA5, np.uint8) for _ in range(12)]
+    for b in bufs:
+        assert b.ctypes.data % 16 == 0
+    p = [b.ctypes.data for b in bufs]
+    X, CODES, SCALES, GS, OUT, MSE, C, G, M, V, U, W = p
+    NVF, ADAM, F32 = NV, 1, 0
+    calls = {
+        "fp4q_quantize": lambda: lib.fp4q_quantize(X, 4, 64, NVF, 16, 0, 0, None, GS, CODES, SCALES,
+                                                   MSE, OUT, F32, None),
+        "fp4q_quantize_mma": lambda: lib.fp4q_quantize_mma(X, 4, 64, NVF, 0, 0, None, GS, CODES,
+                                                           SCALES, None),
+        "fp4q_dequantize": lambda: lib.fp4q_dequantize(CODES, SCALES, GS, 4, 64, NVF, 16, OUT, F32,
+                                                       None),
+        "fp4q_dequantize_unrotate": lambda: lib.fp4q_dequantize_unrotate(
+            CODES, SCALES, GS, 4, 64, NVF, 16, 32, OUT, F32, None),
+        "fp4q_block_mse": lambda: lib.fp4q_block_mse(X, CODES, SCALES, GS, 4, 64, NVF, 16, 0, MSE,
+                                                     None),
+        "fp4q_focus_fwd": lambda: lib.fp4q_focus_fwd(X, C, 4, 64, NVF, 16, 8, None, GS, OUT, F32,
+                                                     None, None, None),
+        "fp4q_focus_bwd": lambda: lib.fp4q_focus_bwd(X, G, C, 4, 64, 8, OUT, None),
+        "fp4q_focus_update": lambda: lib.fp4q_focus_update(X, G, C, W, M, V, 4, 64, 8, ADAM, 1e-3,
+                                                           0.9, 0.999, 1e-8, 1, None),
+        "fp4q_focus_step": lambda: lib.fp4q_focus_step(X, 4, 64, NVF, 16, 8, None, GS, C, W, M, V,
+                                                       MSE, ADAM, 1e-3, 0.9, 0.999, 1e-8, 1, None),
+        "fp4q_gptq": lambda: lib.fp4q_gptq(X, 4, 128, NVF, 16, SCALES, GS, U, None, OUT, CODES,
+                                           None),
+        "fp4q_global_amax": lambda: lib.fp4q_global_amax(X, 4, 64, 0, GS, None),
+        "fp4q_e2m1_encode": lambda: lib.fp4q_e2m1_encode(X, 64, CODES, None),
+        "fp4q_e4m3_encode": lambda: lib.fp4q_e4m3_encode(X, 64, CODES, None),
+        "fp4q_scales_to_mma": lambda: lib.fp4q_scales_to_mma(SCALES, 4, 64, NVF, OUT, None),
+        "fp4q_gemm": lambda: lib.fp4q_gemm(X, SCALES, GS, CODES, U, MSE, 128, 128, 64, NVF, M, OUT,
+                                           F32, None),
+        "fp4q_gemm_noalloc": lambda: lib.fp4q_gemm_noalloc(X, SCALES, GS, CODES, U, MSE, 128, 128,
+                                                           64, NVF, OUT, F32, None),
+    }
+    # every entry point that can enqueue work is covered
+    launching = set(declared_functions()) - {
+        "fp4q_status_string", "fp4q_last_cuda_error", "fp4q_device_errors",
+        "fp4q_mma_scale_bytes", "fp4q_debug_fail_launches"}
+    assert set(calls) == launching
+    code = 719  # cudaErrorLaunchFailure
+    lib.fp4q_debug_fail_launches(code)
+    try:
+        for name, call in calls.items():
+            lib.fp4q_debug_fail_launches(code + len(name))  # a distinct code per entry point
+            assert call() == CUDA, name
+            assert lib.fp4q_last_cuda_error() == code + len(name), name
+        # validation still comes first
+        assert lib.fp4q_quantize(None, 4, 64, NVF, 16, 0, 0, None, GS, CODES, SCALES, None, None,
+                                 0, None) == NULL
+    finally:
+        lib.fp4q_debug_fail_launches(0)
+    for b in bufs:
+        assert (b == 0xA5).all()
