@@ -26,6 +26,13 @@
 #include "cutlass/numeric_types.h"
 #include "cutlass/util/packed_stride.hpp"
 
+// CuTe reports a tensor-map encode that the driver rejects only through
+// assert() (after printing the descriptor's fields); compiled with NDEBUG the
+// GEMM would then be launched with that descriptor. Keep assertions on here.
+#ifdef NDEBUG
+#error "the GEMM units must be compiled with assertions enabled (see above)"
+#endif
+
 // One GEMM configuration in its own namespace: ELEM_A is the CUTLASS
 // block-scaled FP4 type, ELEM_D the output type.
 #define FP4Q_GEMM_CONFIG(NS, ELEM_A, ELEM_D)                                                      \
@@ -91,6 +98,11 @@ cudaError_t run_fp4_gemm(const uint8_t* a, const uint8_t* sfa, const uint8_t* b,
     args.epilogue.thread.alpha = 1.0f;
     args.epilogue.thread.beta = 0.0f;
     args.epilogue.thread.alpha_ptr = alpha;
+    // The driver rejects every tensor-map encode once the context holds an
+    // error (a kernel that faulted earlier leaves a sticky one, 700 for an
+    // illegal address): report it here instead of reaching the encode.
+    if (cudaError_t e = cudaPeekAtLastError(); e != cudaSuccess)
+        return e;
     Gemm g;
     if (g.can_implement(args) != cutlass::Status::kSuccess)
         return cudaErrorInvalidValue;

@@ -35,12 +35,16 @@ constexpr int QTHREADS = 128;
 #ifndef FP4Q_NV_MINB
 #define FP4Q_NV_MINB 7
 #endif
+#ifndef FP4Q_BRUTE_MINB
+#define FP4Q_BRUTE_MINB 1
+#endif
 template <int STRAT>
 struct QMinBlocks {
     static constexpr int value =
         STRAT == K_MX ? FP4Q_MX_MINB
-                      : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE || STRAT == K_UE_BRUTE_FORCE ? 1
-                                                                                              : FP4Q_NV_MINB);
+                      : (STRAT == K_BRUTE_FORCE || STRAT == K_MX_BRUTE || STRAT == K_UE_BRUTE_FORCE
+                             ? FP4Q_BRUTE_MINB
+                             : FP4Q_NV_MINB);
 };
 
 // Per-CTA constants of the NVFP4 kernels, built once by every CTA: the
@@ -69,18 +73,21 @@ struct ScaleTables {
 // win. Codes below c6 - 4 are skipped when saturation_lb at c6 - 5 exceeds the
 // best SSE, else searched as well (ties then go to the lower code). A
 // non-finite block maximum searches every code in order, as the definition
-// does.
+// does. (Evaluating two codes at once on packed f32x2 lanes gave the same
+// results and ran 2-20% slower: the search is bound by its conversions and
+// integer work, not its FP32 issue slots.)
 template <int B, int MAXC, class Tab>
 __device__ __forceinline__ void brute_search(const float* yb, float amax, int c6, const Tab& tab,
                                              uint32_t keep, int& bc_out, float& best_out)
 {
     const bool finite = amax <= FLT_MAX;
     const int lo = finite ? max(1, c6 - 4) : 1;
+    auto check = [&](int c) { return finite && c >= c6 + 5 && (c - c6 - 5) % 3 == 0; };
     float best = 0.0f;
     int bc = lo;
 #pragma unroll 1
     for (int c = lo; c <= MAXC; ++c) {
-        if (finite && c >= c6 + 5 && (c - c6 - 5) % 3 == 0 && block_zero_lb<B>(yb, tab.R[c]) > best)
+        if (check(c) && block_zero_lb<B>(yb, tab.R[c]) > best)
             break;
         const float v = block_sse<B>(yb, tab.R[c], tab.S[c], keep);
         if (c == lo || v < best) {

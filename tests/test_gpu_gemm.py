@@ -99,3 +99,43 @@ def test_quantize_mma_equals_quantize_then_convert(gpu, fmt, block, strat, rot, 
     assert np.array_equal(f.scales.cpu().numpy(), conv.cpu().numpy())
     if fmt == "nvfp4":
         assert f.global_scale.item() == q.global_scale.item()
+
+
+@pytest.mark.parametrize("fmt,block", [("nvfp4", 16), ("mxfp4", 32)])
+def test_gemm_benchmarked_shape_sampled_rows(gpu, fmt, block):
+    """The benchmarked LLM layer, 8192 x 4096 x 14336 with bf16 output: 2048
+    output tiles of 128 x 128 through the persistent tile scheduler (many
+    waves on 148 SMs) and 56 K iterations of 256 each. Sampled rows of D,
+    spread over the M tiles (first and last included), against the oracle's
+    product of the same codes and scales, within the fp32 summation bound."""
+    M, N, K = 8192, 4096, 14336
+    a = synth.laplace_outliers(M, K, seed=21)
+    w = synth.gaussian(N, K, seed=22, std=0.02)
+    qa = gpu.quantize(a.cuda(), fmt, block, "absmax", 0)
+    qw = gpu.quantize(w.cuda(), fmt, block, "absmax", 0)
+    del a, w
+    sa = gpu.scales_to_mma(qa.scales, K, fmt)
+    sw = gpu.scales_to_mma(qw.scales, K, fmt)
+    d = gpu.gemm(qa.codes, sa, qa.global_scale, qw.codes, sw, qw.global_scale, fmt, torch.bfloat16)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = np.unique(np.concatenate([np.linspace(0, M - 1, 16).astype(np.int64),
+                                     rng.choice(M, 8, replace=False)]))
+    ga = None if qa.global_scale is None else float(qa.global_scale.item())
+    gw = None if qw.global_scale is None else float(qw.global_scale.item())
+    ridx = torch.from_numpy(rows).cuda()
+    ac = qa.codes[ridx].cpu().numpy()
+    asc = qa.scales[ridx].cpu().numpy()
+    wc, wsc = qw.codes.cpu().numpy(), qw.scales.cpu().numpy()
+    want = oracle.fp4_gemm(ac, asc, ga, wc, wsc, gw, fmt).astype(np.float64)
+    da = np.abs(oracle.dequantize(ac, asc, 1.0, len(rows), K, fmt, block)).astype(np.float64)
+    mag = np.empty((len(rows), N))
+    for n0 in range(0, N, 512):
+        dw = oracle.dequantize(wc[n0:n0 + 512], wsc[n0:n0 + 512], 1.0, 512, K, fmt, block)
+        mag[:, n0:n0 + 512] = da @ np.abs(dw).astype(np.float64).T
+    alpha = (ga * gw) if fmt == "nvfp4" else 1.0
+    got = d[ridx].float().cpu().numpy().astype(np.float64)
+    tol = K * 2.0 ** -24 * mag * abs(alpha) + 2.0 ** -8 * np.abs(want) + 1e-30
+    bad = np.abs(got - want) > tol
+    assert not bad.any(), f"{bad.sum()} of {bad.size} outside the fp32 summation bound"
+    assert np.abs(want).max() > 0
