@@ -69,8 +69,36 @@ __global__ void __launch_bounds__(256) gptq_gather_kernel(GptqArgs a)
     a.work[t] = __uint_as_float((uint32_t)a.w[i * a.K + column_of(a, j)] << 16);
 }
 
+// E2M1 code of u (RNE, saturating, sign kept) and its exact value, one
+// element (see e2m1_pack8 for the operand order of the conversions).
+__device__ __forceinline__ uint32_t e2m1_code1(float u)
+{
+    uint32_t r;
+    asm("{\n\t.reg .b8 q;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\t"
+        "cvt.u32.u8 %0, q;\n\t}"
+        : "=r"(r)
+        : "f"(u), "f"(0.0f));
+    return r & 0xFu;
+}
+
+__device__ __forceinline__ float e2m1_value1(uint32_t q)
+{
+    uint32_t h;
+    const unsigned short t = (unsigned short)q;
+    asm("{\n\t.reg .b8 q0, q1;\n\t"
+        "mov.b16 {q0, q1}, %1;\n\t"
+        "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t}"
+        : "=r"(h)
+        : "h"(t));
+    return h2_to_f2(h).x;
+}
+
 // One warp per row; lane l holds positions l, l + 32, l + 64, l + 96 of the
-// batch. U's 128 x 128 diagonal block sits in shared memory.
+// batch. U's 128 x 128 diagonal block sits in shared memory. The lane that
+// owns a position quantizes it and broadcasts the error; the errors (which
+// replace the batch's dead weights in work) and the codes are written once
+// per lane at the end of the batch.
 __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs a, int64_t b0)
 {
     extern __shared__ float us[];  // [GB][GB]
@@ -86,19 +114,18 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs 
     if (i >= a.rows)
         return;  // whole warps
     float* wr = a.work + i * a.K + b0;
-    float w[4], S[4], R[4];
-    int64_t word[4];
-    uint32_t shift[4];
+    float w[4], S[4], R[4], er[4];
+    uint32_t qs[4];
+    int64_t col[4];
 #pragma unroll
     for (int t = 0; t < 4; ++t) {
         const int p = lane + 32 * t;
         w[t] = wr[p];
-        const int64_t col = column_of(a, b0 + p);
-        S[t] = scale_at(a, i, col);
+        col[t] = column_of(a, b0 + p);
+        S[t] = scale_at(a, i, col[t]);
         R[t] = S[t] == 0.0f ? 0.0f : guarded_rcp(S[t]);
-        const int64_t e = i * a.K + col;
-        word[t] = e >> 3;
-        shift[t] = 4u * (uint32_t)(e & 7);
+        er[t] = 0.0f;
+        qs[t] = 0u;
     }
 #pragma unroll
     for (int s = 0; s < 4; ++s) {
@@ -110,16 +137,12 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs 
                 uint32_t q = 0;
                 float deq = 0.0f;
                 if (S[s] != 0.0f) {
-                    float u[4] = {__fmul_rn(w[s], R[s]), 0.0f, 0.0f, 0.0f};
-                    q = e2m1_pack4(u) & 0xFu;
-                    float v[4];
-                    e2m1_unpack4(q, v);
-                    deq = __fmul_rn(v[0], S[s]);
+                    q = e2m1_code1(__fmul_rn(w[s], R[s]));
+                    deq = __fmul_rn(e2m1_value1(q), S[s]);
                 }
                 err = __fdiv_rn(__fsub_rn(w[s], deq), us[jj * GB + jj]);
-                if (q != 0)
-                    atomicOr(reinterpret_cast<unsigned*>(a.codes) + word[s], q << shift[s]);
-                wr[jj] = err;  // the batch's errors replace its dead weights
+                er[s] = err;
+                qs[s] = q;
             }
             err = __shfl_sync(0xFFFFFFFFu, err, o);
             const float* urow = us + jj * GB + lane;
@@ -128,6 +151,14 @@ __global__ void __launch_bounds__(ROWS_PER_CTA * 32) gptq_batch_kernel(GptqArgs 
                 if (t > s || (t == s && lane > o))
                     w[t] = __fmaf_rn(-err, urow[32 * t], w[t]);
             }
+        }
+    }
+#pragma unroll
+    for (int t = 0; t < 4; ++t) {
+        wr[lane + 32 * t] = er[t];
+        if (qs[t] != 0) {
+            const int64_t e = i * a.K + col[t];
+            atomicOr(reinterpret_cast<unsigned*>(a.codes) + (e >> 3), qs[t] << (4u * (uint32_t)(e & 7)));
         }
     }
 }
@@ -208,35 +239,44 @@ __global__ void __launch_bounds__(TTHREADS) gptq_trailing_kernel(GptqArgs a, int
                                   : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
         const float* ut = ub + buf * (GB * TC);
-        float acc[8][4];
+        // acc[p][c] = {sum of row 2p, sum of row 2p + 1} at column c: each lane
+        // of the packed fma is the same single-rounding fma as the scalar chain
+        f32x2 acc[4][4];
 #pragma unroll
-        for (int r = 0; r < 8; ++r)
+        for (int p = 0; p < 4; ++p)
 #pragma unroll
             for (int c = 0; c < 4; ++c)
-                acc[r][c] = 0.0f;
+                acc[p][c] = pk2(0.0f, 0.0f);
 #pragma unroll 4
         for (int jj = 0; jj < GB; ++jj) {
             const float4 e0 = reinterpret_cast<const float4*>(es + jj * TR)[ty];
             const float4 e1 = reinterpret_cast<const float4*>(es + jj * TR + TR / 2)[ty];
             const float4 u0 = reinterpret_cast<const float4*>(ut + jj * TC)[tx];
-            const float er[8] = {e0.x, e0.y, e0.z, e0.w, e1.x, e1.y, e1.z, e1.w};
-            const float uc[4] = {u0.x, u0.y, u0.z, u0.w};
+            const f32x2 ep[4] = {pk2(e0.x, e0.y), pk2(e0.z, e0.w), pk2(e1.x, e1.y), pk2(e1.z, e1.w)};
+            const f32x2 ud[4] = {pk2(u0.x, u0.x), pk2(u0.y, u0.y), pk2(u0.z, u0.z), pk2(u0.w, u0.w)};
 #pragma unroll
-            for (int r = 0; r < 8; ++r)
+            for (int p = 0; p < 4; ++p)
 #pragma unroll
                 for (int c = 0; c < 4; ++c)
-                    acc[r][c] = __fmaf_rn(er[r], uc[c], acc[r][c]);
+                    acc[p][c] = fma2(ep[p], ud[c], acc[p][c]);
         }
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const int64_t row = r0 + (r < 4 ? 4 * ty + r : TR / 2 + 4 * ty + r - 4);
             if (row >= a.rows)
                 continue;
+            float t[4];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                float lo, hi;
+                upk2(acc[r / 2][c], lo, hi);
+                t[c] = (r & 1) ? hi : lo;
+            }
             float4 v = old[r];
-            v.x = __fsub_rn(v.x, acc[r][0]);
-            v.y = __fsub_rn(v.y, acc[r][1]);
-            v.z = __fsub_rn(v.z, acc[r][2]);
-            v.w = __fsub_rn(v.w, acc[r][3]);
+            v.x = __fsub_rn(v.x, t[0]);
+            v.y = __fsub_rn(v.y, t[1]);
+            v.z = __fsub_rn(v.z, t[2]);
+            v.w = __fsub_rn(v.w, t[3]);
             *reinterpret_cast<float4*>(a.work + row * a.K + k0 + 4 * tx) = v;
         }
         __syncthreads();  // this U buffer is free for the copy two items ahead
