@@ -70,10 +70,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS)
 
 
-# The sources the headline quantize kernels are compiled from (the kernel
-# template, its block-16 / block-32 instantiation units, the headers).
-HEADLINE_KERNEL_SOURCES = ("fp4q_device.cuh", "internal.h", "quant_b16.cu", "quant_b32.cu",
-                           "quant_kernel.cuh", "quant_tma.cuh")
+# The sources the quantize kernels are compiled from (the kernel template,
+# its instantiation units, the headers): recorded counters are keyed by them.
+HEADLINE_KERNEL_SOURCES = ("fp4q_device.cuh", "internal.h", "quant_b4.cu", "quant_b8.cu",
+                           "quant_b16.cu", "quant_b32.cu", "quant_kernel.cuh", "quant_tma.cuh")
 
 
 def kernel_source_hash():
@@ -85,17 +85,22 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(kernel: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernels
-    have not changed since it was taken; else None."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+def recorded(kernel: str, field: str, path: str = "traffic.json"):
+    """A per-launch counter (DRAM bytes, executed FP32 operations) from a
+    committed ncu summary under profiles/, if the kernels have not changed
+    since it was taken; else None."""
+    p = os.path.join(ROOT, "profiles", path)
     if not os.path.exists(p):
         return None
     d = json.load(open(p))
     e = d.get(kernel)
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
-    return e.get("dram_bytes_per_launch")
+    return e.get(field)
+
+
+def recorded_traffic(kernel: str):
+    return recorded(kernel, "dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------- clocks
@@ -274,7 +279,7 @@ def run_ours(args, rank, world, local_rank):
         kern[tag] = {"us": round(us[k + 1], 2), "alg_GBps": round(gbs, 1),
                      "frac": round(gbs / peaks["hbm_gbs"], 4)}
     dom = max(RUN_TAGS, key=lambda t: kern[t]["us"])
-    kname = {"nvfp4_b16_h16_4over6": "quant_kernel<16, 16, 2> (NVFP4 B16, H16, 4-over-6)",
+    kname = {"nvfp4_b16_h16_4over6": "quant_persist_kernel<16, 16, 2> (NVFP4 B16, H16, 4-over-6)",
              "mxfp4_b32_h128": "quant_kernel<32, 128, 4> (MXFP4 B32, H128)"}[dom]
     traffic = recorded_traffic(kname)
     roofline = {"bound": "hbm", "kernel": kname, "achieved": kern[dom]["alg_GBps"],
@@ -412,13 +417,18 @@ def breakdown(dev, peaks, reps: int = 10):
              "hbm_frac": round(gbs / peaks["hbm_gbs"], 4), "bytes_per_elem": round(bpe, 5),
              "launches": launches}
         if fp32_ops is not None:
-            # exhaustive-equivalent rate: the ops a search over all 126 codes
-            # would issue, per second. The kernel skips the codes that its exact
-            # lower bounds exclude, so this can exceed the FP32 peak; the FP32
-            # pipe utilisation it really reaches is in the ncu summary.
-            d["fp32_ops_exhaustive_equiv_per_s"] = fp32_ops / secs
-            d["fp32_exhaustive_equiv_frac"] = round(fp32_ops / secs / fp32_peak, 4)
+            # the searches: FP32 operations the kernel executed in one launch
+            # (ncu counts of FADD, FMUL, FFMA and twice the packed FADD2, FMUL2,
+            # FFMA2, on this workload, profiles/fp32_ops.json) per second,
+            # against the non-FMA FP32 peak (148 SMs x 128 lanes x 1.965 GHz)
             d["bound"] = "alu"
+            d["fp32_peak_T"] = round(fp32_peak / 1e12, 2)
+            if fp32_ops > 0:
+                d["fp32_ops_per_launch"] = fp32_ops
+                d["fp32_T_per_s"] = round(fp32_ops / secs / 1e12, 2)
+                d["fp32_frac"] = round(fp32_ops / secs / fp32_peak, 4)
+            else:
+                d["fp32_frac"] = None  # no count recorded for these sources
         if note:
             d["note"] = note
         rows_out.append(d)
@@ -440,8 +450,10 @@ def breakdown(dev, peaks, reps: int = 10):
                 for _ in range(nc)]
             dqb = 0 if dq is None else torch.tensor([], dtype=dq).element_size()
             bpe = bytes_per_elem(block, mse=want_mse, dq=dqb)
-            ncodes = {"nvfp4": 126, "mxfp4": 255, "ue5m3": 254}[fmt]
-            ops = n * ncodes * 5 if strat == "brute_force" else None
+            ops = None
+            if strat == "brute_force":
+                ops = recorded(f"{wl} {fmt} B{block} brute_force H{rot}", "fp32_ops_per_launch",
+                               "fp32_ops.json") or 0
             label = "mse_grid (E8M0 brute force)" if (strat == "brute_force" and fmt == "mxfp4") else strat
             tag = f"{wl} {fmt} B{block} {label} H{rot}"
             if nv:
@@ -517,8 +529,8 @@ def breakdown(dev, peaks, reps: int = 10):
     torch.cuda.empty_cache()
     quant_runs("c5_activation_channels", [("nvfp4", 16, "four_over_six", 16),
                                           ("mxfp4", 32, "absmax", 128)])
-    # the headline's kernels on a tensor 8x larger (256 MiB of bf16): the same
-    # code with the launch ramp and tail amortised over 134M elements
+    # MXFP4 without rotation and with the 32-wide rotation (the C2 runs) on the
+    # 256 MiB tensor, where launch ramp and tail are amortised over 134M elements
     quant_runs("c5_activation_channels", [("mxfp4", 32, "absmax", 0), ("mxfp4", 32, "absmax", 32)])
     # W4A4 GEMM on the block-scaled tensor cores, LLM layer shapes (tokens x hidden
     # -> out): operands quantized (abs-max) once, scales in MMA layout; timed: the
