@@ -76,7 +76,7 @@ def focus_coeffs(rows: int, cols: int, sub: int, seed: int, lo: float = 0.9,
 
 
 def gptq_problem(rows: int, cols: int, tokens: int, seed: int, damp: float = 0.01,
-                 act_order: bool = True) -> dict:
+                 act_order: bool = True, rot: int = 0) -> dict:
     """Inputs of the GPTQ error-feedback step for one synthetic linear layer:
     W ~ N(0, 0.02^2) bf16 [rows, cols]; calibration inputs X [tokens, cols] with
     per-channel scales U[0.1, 2.1], 1% of the channels x20 and a random mixing
@@ -84,7 +84,11 @@ def gptq_problem(rows: int, cols: int, tokens: int, seed: int, damp: float = 0.0
     H = X^T X / tokens + damp * mean(diag) * I; the processing order (columns by
     decreasing diag(H) when act_order, else the identity); and the upper
     Cholesky factor U of H^-1 in that order, all computed in float64 and
-    handed over as fp32 / int32 (the caller's preparation)."""
+    handed over as fp32 / int32 (the caller's preparation). rot > 0: the
+    calibration inputs are taken in the rotated basis X R (R the block-diagonal
+    normalised Sylvester Hadamard of width rot), so h, perm and u are those of
+    R H R (h_orig keeps H); the weights stay as drawn (the rotation of W is the
+    quantizer's own, applied by the GPTQ call)."""
     rng = np.random.default_rng(seed)
     w = gaussian(rows, cols, seed=seed + 1, std=0.02)
     x = rng.standard_normal((tokens, cols)) * rng.uniform(0.1, 2.1, cols)
@@ -92,10 +96,18 @@ def gptq_problem(rows: int, cols: int, tokens: int, seed: int, damp: float = 0.0
     x = x @ (np.eye(cols) + 0.3 * rng.standard_normal((cols, cols)) / np.sqrt(cols))
     h = x.T @ x / tokens
     h += damp * float(np.mean(np.diag(h))) * np.eye(cols)
+    out = {"w": w}
+    if rot:
+        # the damping term commutes with R (R R = I, and the trace is invariant)
+        import scipy.linalg
+        r = np.kron(np.eye(cols // rot), scipy.linalg.hadamard(rot) / np.sqrt(rot))
+        out["h_orig"] = h
+        h = r @ h @ r
     perm = np.argsort(-np.diag(h), kind="stable") if act_order else np.arange(cols)
     hp = h[np.ix_(perm, perm)]
     u = np.linalg.cholesky(np.linalg.inv(hp)).T     # upper: H^-1 = U^T U
-    return {"w": w, "h": h, "perm": perm.astype(np.int32), "u": np.ascontiguousarray(u, np.float32)}
+    out.update({"h": h, "perm": perm.astype(np.int32), "u": np.ascontiguousarray(u, np.float32)})
+    return out
 
 
 def workload(name: str, rows: int | None = None, cols: int | None = None) -> dict:

@@ -84,7 +84,7 @@ def lib():
         L.ref_rne_ue5m3_bits_range.restype = None
         L.ref_rne_ue5m3_bits_range.argtypes = [C.c_uint32, i64, p]
         L.ref_gptq.restype = i32
-        L.ref_gptq.argtypes = [p, i64, i64, i32, i32, p, C.c_float, p, p, p]
+        L.ref_gptq.argtypes = [p, i64, i64, i32, i32, i32, p, C.c_float, p, p, p]
         L.ref_float_to_fp16.restype = C.c_uint16
         L.ref_float_to_fp16.argtypes = [C.c_float]
         f32 = C.c_float
@@ -352,11 +352,13 @@ def focus_bwd(w_bf16, g_bf16, c_fp16, sub=8):
     return dc
 
 
-def gptq(w_bf16, scales, global_scale, U, perm=None, fmt="nvfp4", block=16):
+def gptq(w_bf16, scales, global_scale, U, perm=None, fmt="nvfp4", block=16, rot=0):
     """GPTQ error feedback with static groups (fixed block scales); U: fp32
     [K, K] upper Cholesky factor of the inverse Hessian in processing order;
-    perm: int32 [K] processing position -> original column (None: identity).
-    Returns packed codes [rows, K/2] in the original column order."""
+    perm: int32 [K] processing position -> original column (None: identity);
+    rot > 0: the rows are first rotated blockwise (MR-GPTQ), and scales, U and
+    perm belong to the rotated basis. Returns packed codes [rows, K/2] in the
+    original column order."""
     w = _u16(w_bf16)
     rows, K = w.shape
     scales = np.ascontiguousarray(scales, np.uint8)
@@ -364,7 +366,7 @@ def gptq(w_bf16, scales, global_scale, U, perm=None, fmt="nvfp4", block=16):
     pm = None if perm is None else np.ascontiguousarray(perm, np.int32)
     codes = np.zeros((rows, K // 2), np.uint8)
     sg = 1.0 if global_scale is None else float(global_scale)
-    rc = lib().ref_gptq(_ptr(w), rows, K, _fmt(fmt), block, _ptr(scales), sg, _ptr(U), _ptr(pm),
+    rc = lib().ref_gptq(_ptr(w), rows, K, _fmt(fmt), block, rot, _ptr(scales), sg, _ptr(U), _ptr(pm),
                         _ptr(codes))
     if rc != 0:
         raise ValueError(f"oracle rejected arguments (rc={rc})")

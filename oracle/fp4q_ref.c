@@ -791,12 +791,18 @@ int ref_fp4_gemm(const uint8_t* a_codes, const uint8_t* a_scales, float a_sg, co
  *   then every position k after the block: t = fma sum of e_j * U[j][k] over
  *     the block's j ascending from t = 0, and w_k = w_k - t.
  * Codes are written at the original column (packed as in R8). Rows are
- * independent. */
-int ref_gptq(const uint16_t* w, int64_t rows, int64_t K, int fmt, int block,
+ * independent.
+ * rot > 0: the rotation of MR-GPTQ comes first -- each row is rotated chunk by
+ * chunk (rot-wide blockwise Hadamard of the original column order, exactly
+ * the quantizer's rotation, load_row) and the error feedback runs on the
+ * rotated fp32 weights; scales, U and perm then belong to the rotated basis
+ * (static scales from ref_quantize with the same rot; U from the Hessian of
+ * the rotated inputs). The codes are those of the rotated weights. */
+int ref_gptq(const uint16_t* w, int64_t rows, int64_t K, int fmt, int block, int rot,
              const uint8_t* scales, float sg, const float* U, const int32_t* perm,
              uint8_t* codes)
 {
-    if (!valid_common(rows, K, fmt, block, 0) || K % 128 != 0)
+    if (!valid_common(rows, K, fmt, block, rot) || K % 128 != 0)
         return REF_ERR_ARG;
     if (perm) {
         uint8_t* seen = (uint8_t*)calloc((size_t)K, 1);
@@ -812,12 +818,14 @@ int ref_gptq(const uint16_t* w, int64_t rows, int64_t K, int fmt, int block,
             return REF_ERR_ARG;
     }
     float* W = (float*)malloc(sizeof(float) * (size_t)K);
+    float* Y = (float*)malloc(sizeof(float) * (size_t)K);
     float E[128];
     int64_t nb = K / block;
     memset(codes, 0, (size_t)(rows * K / 2));
     for (int64_t i = 0; i < rows; i++) {
+        load_row(w + i * K, K, rot, Y);
         for (int64_t j = 0; j < K; j++)
-            W[j] = ref_bf16_to_float(w[i * K + (perm ? perm[j] : j)]);
+            W[j] = Y[perm ? perm[j] : j];
         for (int64_t b0 = 0; b0 < K; b0 += 128) {
             for (int jj = 0; jj < 128; jj++) {
                 int64_t j = b0 + jj;
@@ -846,6 +854,7 @@ int ref_gptq(const uint16_t* w, int64_t rows, int64_t K, int fmt, int block,
         }
     }
     free(W);
+    free(Y);
     return REF_OK;
 }
 

@@ -149,3 +149,75 @@ def test_rejects_bad_arguments(ref):
     with pytest.raises(ValueError):
         ref.gptq(bf16_bits(np.zeros((2, 192))), np.zeros((2, 12), np.uint8), 1.0,
                  np.eye(192, dtype=np.float32), None, "nvfp4", 16)        # K % 128
+
+
+# ------------------------------------------- rotation in front (MR-GPTQ)
+
+def hadamard_rows(w, n):
+    """w times the block-diagonal normalised Sylvester Hadamard of width n, in
+    float64 (scipy's matrix, rows taken chunk by chunk)."""
+    import scipy.linalg
+    rows, K = w.shape
+    return (w.reshape(rows, K // n, n) @ scipy.linalg.hadamard(n)).reshape(rows, K) / np.sqrt(n)
+
+
+@pytest.mark.parametrize("fmt,block,strat,rot", [("nvfp4", 16, "absmax", 16), ("mxfp4", 32, "absmax", 128),
+                                                 ("ue5m3", 8, "four_over_six", 32)])
+def test_rotated_no_feedback_is_rotated_round_to_nearest(ref, fmt, block, strat, rot):
+    # with U diagonal, GPTQ behind the rotation is the quantizer's own
+    # round-to-nearest of the rotated rows with the same scales: the rotation
+    # is the quantizer's (same chunks, stages and factor), in any order
+    x = synth.workload("c5_activation_channels", rows=12, cols=256)["x"]
+    xb = synth.bits16(x)
+    q = ref.quantize(xb, fmt, block, strat, rot)
+    rng = np.random.default_rng(2)
+    U = np.diag(rng.uniform(0.5, 2, 256)).astype(np.float32)
+    for perm in (None, rng.permutation(256).astype(np.int32)):
+        codes = ref.gptq(xb, q["scales"], q["global_scale"], U, perm, fmt, block, rot=rot)
+        assert np.array_equal(codes, q["codes"])
+    # and the rotation does change the codes (the case exercises it)
+    assert not np.array_equal(ref.gptq(xb, q["scales"], q["global_scale"], U, None, fmt, block),
+                              q["codes"])
+
+
+def test_rotated_dyadic_case_equals_unblocked_float64(ref):
+    # Dyadic weights rotated by the 16-wide Hadamard (factor 1/4: exact): the
+    # rotated values are short dyadic fractions in fp32 and float64 alike, so
+    # the oracle (rotation, then blocked fp32 GPTQ) must equal float64 GPTQ run
+    # on scipy's rotation of the same rows, code for code.
+    rng = np.random.default_rng(8)
+    rows, K = 5, 256
+    w = rng.integers(-24, 25, size=(rows, K)) / 16.0
+    U = np.eye(K)
+    mask = np.triu(rng.random((K, K)) < 0.02, 1)
+    U[mask] = rng.choice([-0.25, -0.125, 0.125, 0.25], size=int(mask.sum()))
+    perm = rng.permutation(K)
+    scales = np.full((rows, K // 32), 127, np.uint8)           # E8M0 2^0
+    got = ref.unpack_codes(ref.gptq(bf16_bits(w), scales, None, U.astype(np.float32),
+                                    perm.astype(np.int32), "mxfp4", 32, rot=16))
+    want = gptq_f64_unblocked(hadamard_rows(w, 16), np.ones((rows, K)), U, perm)
+    assert np.array_equal(got.astype(np.int64), want)
+
+
+@pytest.mark.parametrize("rot", [16, 128])
+def test_rotated_error_feedback_and_loss_identity(ref, rot):
+    # Behind the rotation, GPTQ's codes lower the layer loss below the rotated
+    # round-to-nearest's, measured in the rotated basis with R H R; taken back
+    # to the original basis (Ŵ R, R R = I) the same loss is measured with H:
+    # the two must agree (float64), which pins the basis in which the scales,
+    # U and the codes live.
+    d = synth.gptq_problem(16, 256, 2048, seed=4, rot=rot)
+    wb = synth.bits16(d["w"])
+    q = ref.quantize(wb, "nvfp4", 16, "absmax", rot)
+    sg = q["global_scale"]
+    codes = ref.gptq(wb, q["scales"], sg, d["u"], d["perm"], "nvfp4", 16, rot=rot)
+    S = per_element_scales(ref, q["scales"], "nvfp4", 16, sg)
+    w = f32_of_bf16(wb).astype(np.float64)
+    wr = hadamard_rows(w, rot)                                   # the rotated weights
+    val = lambda c: np.where(ref.unpack_codes(c) >= 8, -1, 1) * E2M1_MAG[ref.unpack_codes(c) & 7] * S
+    loss_rot = lambda c: float(np.einsum("ij,jk,ik->", val(c) - wr, d["h"], val(c) - wr))
+    l_gptq, l_rtn = loss_rot(codes), loss_rot(q["codes"])
+    assert l_gptq < 0.8 * l_rtn, (l_gptq, l_rtn)
+    back = hadamard_rows(val(codes), rot)                        # Ŵ R: the original basis
+    l_orig = float(np.einsum("ij,jk,ik->", back - w, d["h_orig"], back - w))
+    assert abs(l_orig - l_gptq) <= 1e-6 * l_gptq, (l_orig, l_gptq)
