@@ -596,6 +596,20 @@ def breakdown(dev, peaks, reps: int = 10):
                      "us": round(gsecs * 1e6, 1), "tflops": round(gflops / gsecs / 1e12, 2),
                      "bound": "fp32 fma", "fma_frac": round(gflops / gsecs / 1e12 / fma_peak, 4),
                      "peak_tflops": round(fma_peak, 1), "launches": 1 + 2 * 32 - 1})
+    # MR-GPTQ: the 128-wide blockwise rotation in front (MXFP4 B32 with the
+    # MSE-optimised E8M0 grid as static scales of the rotated weights; U from
+    # the rotated-basis Hessian), the same layer size
+    gd = synth.gptq_problem(4096, 4096, 4096, seed=11, rot=128)
+    gqs = fp4q.quantize(gw, "mxfp4", 32, "brute_force", 128)
+    gU = torch.from_numpy(gd["u"]).to(dev)
+    gperm = torch.from_numpy(gd["perm"]).to(dev)
+    gsecs = timeit([lambda: fp4q.gptq(gw, gqs.scales, None, gU, gperm, "mxfp4", 32, work=gwork, out=gout,
+                                      rot=128)])
+    rows_out.append({"run": "mr-gptq (rotation 128 + error feedback) mxfp4 B32 4096x4096 "
+                            "(static MSE-grid scales, act order)",
+                     "us": round(gsecs * 1e6, 1), "tflops": round(gflops / gsecs / 1e12, 2),
+                     "bound": "fp32 fma", "fma_frac": round(gflops / gsecs / 1e12 / fma_peak, 4),
+                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 2 * 32 - 1})
     del gd, gw, gqs, gU, gperm, gwork, gout
     torch.cuda.empty_cache()
     # FOCUS

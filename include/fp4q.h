@@ -367,6 +367,15 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
  * w         bf16 [rows, cols], cols a multiple of 128.
  * fmt, block, scales [rows, cols/block], global_scale (NVFP4 s_g, device):
  *           the static block scales; any format.
+ * rot       0, or 16 / 32 / 64 / 128: MR-GPTQ's rotation first -- every row
+ *           is rotated chunk by chunk exactly as fp4q_quantize rotates it
+ *           (blockwise normalised Walsh-Hadamard, fp32) and the feedback runs
+ *           on the rotated weights; scales, global_scale, U and perm are then
+ *           those of the rotated basis (scales from fp4q_quantize with the
+ *           same rot; U from the Hessian of the rotated inputs, R H R). The
+ *           codes are the rotated weights' (fp4q_dequantize_unrotate takes
+ *           them back). With rot > 0 a row is staged in shared memory:
+ *           cols * 4 bytes must not exceed 227 KB (else SHAPE).
  * U         fp32 [cols, cols] row-major (only the upper triangle is read).
  * perm      int32 [cols]: processing position -> original column, a
  *           permutation (entries outside 0..cols-1 are counted by
@@ -376,7 +385,7 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
  * Launches: 1 memset + 1 + 2 * cols/128 - 1 kernels. Rows are independent.
  */
 fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
-                      const uint8_t* scales, const float* global_scale, const float* U,
+                      int rot, const uint8_t* scales, const float* global_scale, const float* U,
                       const int32_t* perm, float* work, uint8_t* codes, cudaStream_t stream);
 
 /*

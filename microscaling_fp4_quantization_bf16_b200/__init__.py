@@ -231,10 +231,12 @@ def focus_step(w: torch.Tensor, state: FocusState, fmt="nvfp4", block: int = 16,
 
 def gptq(w: torch.Tensor, scales: torch.Tensor, global_scale: Optional[torch.Tensor],
          U: torch.Tensor, perm: Optional[torch.Tensor] = None, fmt="nvfp4", block: int = 16,
-         work: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+         work: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+         rot: int = 0) -> torch.Tensor:
     """GPTQ error feedback with static groups (fixed block scales); returns the
     packed codes uint8 [rows, cols/2]. U: fp32 [cols, cols] upper Cholesky
-    factor of the inverse Hessian in processing order; perm: int32 [cols]."""
+    factor of the inverse Hessian in processing order; perm: int32 [cols];
+    rot > 0: MR-GPTQ's blockwise rotation first (see fp4q_gptq)."""
     _check(w, torch.bfloat16, "w")
     _check(scales, torch.uint8, "scales")
     _check(U, torch.float32, "U")
@@ -245,7 +247,7 @@ def gptq(w: torch.Tensor, scales: torch.Tensor, global_scale: Optional[torch.Ten
         work = torch.empty(rows, cols, dtype=torch.float32, device=w.device)
     if out is None:
         out = torch.empty(rows, cols // 2, dtype=torch.uint8, device=w.device)
-    _abi.call("fp4q_gptq", w.data_ptr(), rows, cols, _fmt(fmt), block, scales.data_ptr(),
+    _abi.call("fp4q_gptq", w.data_ptr(), rows, cols, _fmt(fmt), block, rot, scales.data_ptr(),
               _ptr(global_scale), U.data_ptr(), _ptr(perm), work.data_ptr(), out.data_ptr(),
               _stream())
     return out

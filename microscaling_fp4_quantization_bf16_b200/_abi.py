@@ -31,7 +31,7 @@ SIGNATURES = {
                                  _f32, _f32, _i64, _p]),
     "fp4q_focus_step": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p,
                                _i32, _f32, _f32, _f32, _f32, _i64, _p]),
-    "fp4q_gptq": (_i32, [_p, _i64, _i64, _i32, _i32, _p, _p, _p, _p, _p, _p, _p]),
+    "fp4q_gptq": (_i32, [_p, _i64, _i64, _i32, _i32, _i32, _p, _p, _p, _p, _p, _p, _p]),
     "fp4q_global_amax": (_i32, [_p, _i64, _i64, _i32, _p, _p]),
     "fp4q_e2m1_encode": (_i32, [_p, _i64, _p, _p]),
     "fp4q_e4m3_encode": (_i32, [_p, _i64, _p, _p]),

@@ -682,13 +682,15 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
 }
 
 fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
-                      const uint8_t* scales, const float* global_scale, const float* U,
+                      int rot, const uint8_t* scales, const float* global_scale, const float* U,
                       const int32_t* perm, float* work, uint8_t* codes, cudaStream_t stream)
 {
-    fp4q_status st = check_format(rows, cols, fmt, block, 0);
+    fp4q_status st = check_format(rows, cols, fmt, block, rot);
     if (st != FP4Q_OK)
         return st;
     if (cols % 128 != 0 || rows > 0x7FFFFFFF)
+        return FP4Q_ERR_SHAPE;
+    if (rot > 0 && cols * 4 > kGptqRowBytes)
         return FP4Q_ERR_SHAPE;
     const bool nv = fmt == FP4Q_FMT_NVFP4;
     const int64_t n = rows * cols;
@@ -714,6 +716,7 @@ fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt
     a.K = cols;
     a.fmt = (int)fmt;
     a.block = block;
+    a.rot = rot;
     cudaError_t e = cudaGetSymbolAddress(reinterpret_cast<void**>(&a.err), g_fp4q_device_errors);
     if (e == cudaSuccess)
         e = cudaMemsetAsync(codes, 0, (size_t)(n / 2), stream);

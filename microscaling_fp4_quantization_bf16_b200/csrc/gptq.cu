@@ -8,7 +8,9 @@
 // upper Cholesky factor of the inverse Hessian in that order. Work proceeds
 // in batches of 128 positions ("lazy batch updates"):
 //
-//   gptq_gather_kernel   work[i][j] = W[i][perm[j]] widened to fp32
+//   gptq_gather_kernel   work[i][j] = W[i][perm[j]] widened to fp32 (with a
+//                        rotation: gptq_rotate_gather_kernel, the row rotated
+//                        blockwise first, as the quantizer rotates it)
 //   gptq_batch_kernel    one warp per row runs the 128 positions of a batch
 //                        in order: quantize with the fixed scale, error
 //                        e = (w - value * S) / U[j][j], spread inside the batch
@@ -67,6 +69,39 @@ __global__ void __launch_bounds__(256) gptq_gather_kernel(GptqArgs a)
         return;
     const int64_t i = t / a.K, j = t - i * a.K;
     a.work[t] = __uint_as_float((uint32_t)a.w[i * a.K + column_of(a, j)] << 16);
+}
+
+// MR-GPTQ's rotation in front: one CTA per row. Every thread rotates 32-element
+// segments of the row exactly as the quantizer does (rotate_seg: widening,
+// butterfly stages in ascending order, the factor k_ROT; 64/128-wide chunks
+// span neighbouring lanes, so whole warps take part) into a shared copy of
+// the row in original column order, which is then gathered into processing
+// order: work[i][j] = rotated(W)[i][perm[j]].
+template <int ROT>
+__global__ void __launch_bounds__(1024) gptq_rotate_gather_kernel(GptqArgs a)
+{
+    extern __shared__ float rowbuf[];  // [K]
+    pdl_begin();
+    const int64_t i = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int64_t nseg = a.K / SEG;
+    const int64_t nseg_warps = (nseg + 31) / 32 * 32;  // whole warps per pass
+    const uint16_t* wrow = a.w + i * a.K;
+    for (int64_t sg = threadIdx.x; sg < nseg_warps; sg += blockDim.x) {
+        float y[SEG];
+        load_seg_bf16(wrow, a.K, sg, y);  // zeros past the row
+        rotate_seg<ROT>(y, lane);
+        if (sg < nseg) {
+            float4* o = reinterpret_cast<float4*>(rowbuf + sg * SEG);
+#pragma unroll
+            for (int k = 0; k < SEG / 4; ++k)
+                o[k] = make_float4(y[4 * k], y[4 * k + 1], y[4 * k + 2], y[4 * k + 3]);
+        }
+    }
+    __syncthreads();
+    float* wo = a.work + i * a.K;
+    for (int64_t j = threadIdx.x; j < a.K; j += blockDim.x)
+        wo[j] = rowbuf[column_of(a, j)];
 }
 
 // E2M1 code of u (RNE, saturating, sign kept) and its exact value, one
@@ -306,7 +341,29 @@ cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
     if (e != cudaSuccess)
         return e;
     const int64_t n = a.rows * a.K;
-    e = launch_pdl(gptq_gather_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a);
+    if (a.rot == 0) {
+        e = launch_pdl(gptq_gather_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a);
+    } else {
+        const size_t row_smem = sizeof(float) * (size_t)a.K;
+        const int64_t nseg_warps = (a.K / SEG + 31) / 32 * 32;
+        const unsigned threads = (unsigned)(nseg_warps < 1024 ? nseg_warps : 1024);
+        if ((int64_t)row_smem > kGptqRowBytes)
+            return cudaErrorInvalidValue;
+        auto launch_rot = [&](auto kern) {
+            cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)row_smem);
+            if (r != cudaSuccess)
+                return r;
+            return launch_pdl(kern, dim3((unsigned)a.rows), dim3(threads), row_smem, st, a);
+        };
+        switch (a.rot) {
+        case 16: e = launch_rot(gptq_rotate_gather_kernel<16>); break;
+        case 32: e = launch_rot(gptq_rotate_gather_kernel<32>); break;
+        case 64: e = launch_rot(gptq_rotate_gather_kernel<64>); break;
+        case 128: e = launch_rot(gptq_rotate_gather_kernel<128>); break;
+        default: e = cudaErrorInvalidValue;
+        }
+    }
     const unsigned row_ctas = (unsigned)((a.rows + ROWS_PER_CTA - 1) / ROWS_PER_CTA);
     const unsigned row_tiles = (unsigned)((a.rows + TR - 1) / TR);
     for (int64_t b0 = 0; b0 < a.K && e == cudaSuccess; b0 += GB) {

@@ -151,7 +151,11 @@ struct GptqArgs {
     unsigned* err;          // device error counter
     int64_t rows, K;
     int fmt, block;         // fmt: 0 NVFP4, 1 MXFP4, 2 UE5M3
+    int rot;                // 0, or the width of the blockwise rotation applied first
 };
+
+// Largest row (bytes of fp32) the rotated GPTQ path stages in shared memory.
+constexpr int64_t kGptqRowBytes = 227 * 1024;
 
 // Each launcher returns cudaErrorInvalidValue for a combination it does not
 // provide (the ABI layer validates before calling), else the launch status.

@@ -167,11 +167,13 @@ def test_other_entry_points_validation(lib):
     assert fs(fmt=UE) == UNSUP
     # GPTQ error feedback
     gq = lambda **k: L.fp4q_gptq(k.get("w", A), 4, k.get("cols", 256), k.get("fmt", NV),
-                                 k.get("block", 16), A, k.get("gs", A2), A3, k.get("perm"),
-                                 k.get("work", A), k.get("codes", A2), None)
+                                 k.get("block", 16), k.get("rot", 0), A, k.get("gs", A2), A3,
+                                 k.get("perm"), k.get("work", A), k.get("codes", A2), None)
     assert gq(cols=192) == SHAPE      # cols % 128
     assert gq(cols=200) == SHAPE      # cols % block
     assert gq(block=64) == UNSUP
+    assert gq(rot=24) == UNSUP
+    assert gq(rot=128, cols=58368) == SHAPE   # rotated rows staged in 227 KB of shared memory
     assert gq(gs=None) == NULL        # NVFP4 needs s_g
     assert gq(work=None) == NULL
     assert gq(perm=MIS) == ALIGN
@@ -274,7 +276,7 @@ def test_injected_cuda_error_every_entry_point(lib):
                                                            0.9, 0.999, 1e-8, 1, None),
         "fp4q_focus_step": lambda: lib.fp4q_focus_step(X, 4, 64, NVF, 16, 8, None, GS, C, W, M, V,
                                                        MSE, ADAM, 1e-3, 0.9, 0.999, 1e-8, 1, None),
-        "fp4q_gptq": lambda: lib.fp4q_gptq(X, 4, 128, NVF, 16, SCALES, GS, U, None, OUT, CODES,
+        "fp4q_gptq": lambda: lib.fp4q_gptq(X, 4, 128, NVF, 16, 16, SCALES, GS, U, None, OUT, CODES,
                                            None),
         "fp4q_global_amax": lambda: lib.fp4q_global_amax(X, 4, 64, 0, GS, None),
         "fp4q_e2m1_encode": lambda: lib.fp4q_e2m1_encode(X, 64, CODES, None),

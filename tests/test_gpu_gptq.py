@@ -16,7 +16,7 @@ def u16(t):
     return synth.bits16(t)
 
 
-def run_gpu(gpu, wb, scales, sg, U, perm, fmt, block):
+def run_gpu(gpu, wb, scales, sg, U, perm, fmt, block, rot=0):
     w = torch.from_numpy(wb.view(np.int16)).view(torch.bfloat16).cuda()
     sc = torch.from_numpy(np.ascontiguousarray(scales)).cuda()
     gs = None if sg is None else torch.tensor([sg], dtype=torch.float32, device="cuda")
@@ -24,7 +24,7 @@ def run_gpu(gpu, wb, scales, sg, U, perm, fmt, block):
     pd = None if perm is None else torch.from_numpy(np.ascontiguousarray(perm, np.int32)).cuda()
     guard = torch.full((w.shape[0] * w.shape[1] // 2 + 64,), 0xA5, dtype=torch.uint8, device="cuda")
     codes = gpu.gptq(w, sc, gs, Ud, pd, fmt, block, out=guard[: w.shape[0] * w.shape[1] // 2]
-                     .view(w.shape[0], -1))
+                     .view(w.shape[0], -1), rot=rot)
     torch.cuda.synchronize()
     assert torch.all(guard[-64:] == 0xA5), "write past the end of the codes"
     return codes.cpu().numpy()
@@ -86,3 +86,20 @@ def test_gptq_out_of_range_order_is_counted(gpu):
     perm[5] = 128
     run_gpu(gpu, wb, q["scales"], None, d["u"], perm, "mxfp4", 32)
     assert gpu._abi.load().fp4q_device_errors() > 0
+
+
+@pytest.mark.parametrize("fmt,block,strat,rot", [("nvfp4", 16, "absmax", 16), ("mxfp4", 32, "brute_force", 128),
+                                                 ("ue5m3", 8, "four_over_six", 32), ("nvfp4", 32, "brute_force", 64)])
+def test_gptq_rotated_small_layers(gpu, fmt, block, strat, rot):
+    """MR-GPTQ's blockwise rotation in front of the feedback (static scales from
+    the rotated quantizer, U from the rotated-basis Hessian), every code."""
+    for rows, K, seed in ((37, 256, 5), (9, 384, 6), (70, 128, 7), (3, 1152, 8)):
+        d = synth.gptq_problem(rows, K, 1024, seed=seed, rot=rot)
+        wb = u16(d["w"])
+        q = oracle.quantize(wb, fmt, block, strat, rot, want_mse=False)
+        sg = q["global_scale"] if fmt == "nvfp4" else None
+        want = oracle.gptq(wb, q["scales"], sg, d["u"], d["perm"], fmt, block, rot=rot)
+        got = run_gpu(gpu, wb, q["scales"], sg, d["u"], d["perm"], fmt, block, rot=rot)
+        bad = np.nonzero(got != want)
+        assert bad[0].size == 0, f"{fmt} B{block} {strat} H{rot} {rows}x{K}: {bad[0].size} bytes differ"
+    assert gpu._abi.load().fp4q_device_errors() == 0
