@@ -52,7 +52,10 @@
  *  - rows == 0 or cols == 0 is an empty tensor: its array pointers may be
  *    NULL, nothing is read or written except that NVFP4 global_scale_out
  *    receives 1.0 (and fp4q_global_amax writes 0).
- *  - Inputs must be finite. Outputs must not overlap inputs or each other
+ *  - Inputs must be finite, and so must their rotation (a blockwise Hadamard
+ *    sum of inputs near the bf16 maximum can exceed the fp32 range; the
+ *    codes of such a block are then unspecified). Outputs must not overlap
+ *    inputs or each other
  *    (arrays an entry point documents as read and overwritten are the
  *    exception: they are updated in place).
  *  - FP4Q_ERR_CUDA means a launch was rejected by the CUDA runtime; the

@@ -416,3 +416,54 @@ def test_side_stream(gpu):
     assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales)
     assert torch.equal(a.mse.view(torch.int32), b.mse.view(torch.int32))
     assert gpu._abi.load().fp4q_device_errors() == 0
+
+
+# ---------------------------------------------- folded rotation factor
+
+@pytest.mark.parametrize("rot", [16, 64])
+def test_fold_boundaries_nvfp4(gpu, rot):
+    """NVFP4 / UE5M3 behind a 16- or 64-wide rotation fold the factor 1/sqrt(n)
+    (a power of two) into the reciprocal when s_g lies in [2^-105, 2^110]; just
+    inside and outside both ends (s_g = amax / 2688, amax supplied), with data
+    at the scale of the blocks, codes, scales, MSE and dq equal the oracle's."""
+    rng = np.random.default_rng(rot)
+    lo, hi = 2.0 ** -105 * 2688, 2.0 ** 110 * 2688
+    for ga in (lo * 0.999, lo * 1.001, hi * 0.999, hi * 1.001, 3.0e38):
+        # data at the blocks' scale, small enough that no butterfly sum overflows
+        a = rng.standard_normal((6, 256)) * (ga / (2 * rot))
+        a[0, :16] = ga / (2 * rot)    # a constant block (one large butterfly sum)
+        a[1, 3] = ga * 1e-30          # an element far below its block's scale
+        x = synth.to_bf16(np.clip(a, -3.3e38, 3.3e38))
+        for fmt, block, strat in [("nvfp4", 16, "four_over_six"), ("nvfp4", 4, "absmax"),
+                                  ("nvfp4", 8, "prevent_zero")]:
+            for mse, dq in ((True, torch.float32), (False, None)):
+                g = gpu_quantize(gpu, x, fmt, block, strat, rot, gamax=float(np.float32(ga)), mse=mse, dq=dq)
+                o = oracle_quantize(x, fmt, block, strat, rot, gamax=float(np.float32(ga)), mse=mse, dq=dq)
+                compare_quant(g, o, fmt, f"fold {fmt} B{block} {strat} H{rot} ga={ga:.3e} mse={mse}")
+
+
+@pytest.mark.parametrize("rot", [16, 32, 64, 128])
+def test_fold_mxfp4(gpu, rot):
+    """MXFP4 folds 1/sqrt(n) into its power-of-two reciprocal when codes only are
+    wanted and 2^-e stays normal after the fold (e <= 122, checked per
+    segment). Ordinary, large and tiny blocks in one tensor, with and without
+    the MSE output (which never folds). For 16- and 32-wide rotations, chunks
+    of equal values put a rotated block maximum at 2^125 (e = 123: the unfolded
+    branch) with every rotated value finite; for 64 and 128 that maximum would
+    need a butterfly sum beyond the fp32 range (inputs whose rotation
+    overflows are outside the contract)."""
+    rng = np.random.default_rng(rot + 1)
+    a = rng.standard_normal((8, 512))
+    a[1] *= 2.0 ** 100             # large blocks, folded
+    a[3] *= 2.0 ** -120            # tiny blocks (subnormal products)
+    a[4, ::7] = 0.0
+    if rot in (16, 32):
+        # t = rot * c in the first butterfly output (finite), y = t k >= 2^125
+        c = 2.0 ** 123 if rot == 16 else 1.5 * 2.0 ** 122
+        a[2, :rot] = c             # one chunk: e = 123, unfolded
+        a[2, 2 * rot:3 * rot] = c / 4  # e = 121: folded
+    x = synth.to_bf16(a)
+    for mse, dq in ((False, None), (True, torch.bfloat16), (False, torch.float32)):
+        g = gpu_quantize(gpu, x, "mxfp4", 32, "absmax", rot, mse=mse, dq=dq)
+        o = oracle_quantize(x, "mxfp4", 32, "absmax", rot, mse=mse, dq=dq)
+        compare_quant(g, o, "mxfp4", f"mx fold H{rot} mse={mse} dq={dq}")
