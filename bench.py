@@ -280,7 +280,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(gbs / peaks["hbm_gbs"], 4)}
     dom = max(RUN_TAGS, key=lambda t: kern[t]["us"])
     kname = {"nvfp4_b16_h16_4over6": "quant_persist_kernel<16, 16, 2> (NVFP4 B16, H16, 4-over-6)",
-             "mxfp4_b32_h128": "quant_kernel<32, 128, 4> (MXFP4 B32, H128)"}[dom]
+             "mxfp4_b32_h128": "quant_tma_kernel<32, 128, 4> (MXFP4 B32, H128, TMA-fed)"}[dom]
     traffic = recorded_traffic(kname)
     roofline = {"bound": "hbm", "kernel": kname, "achieved": kern[dom]["alg_GBps"],
                 "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": kern[dom]["frac"],

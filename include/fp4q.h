@@ -434,10 +434,11 @@ void fp4q_debug_fail_launches(int cuda_error);
  * correct operation never produces) makes the kernel leave early and adds
  * one to a per-device counter instead of hanging the GPU. This call
  * synchronises with the current device, returns the counter and clears it
- * (-1 if the read failed). Environment: FP4Q_TMA=1 routes quantize calls
- * whose flattened length is a multiple of 64 (all strategies but brute
- * force) to the TMA-fed kernel; the default direct-load kernel computes the
- * same bits.
+ * (-1 if the read failed). Environment: by default the TMA-fed kernel takes
+ * MXFP4 quantize calls behind a 64- or 128-wide rotation and the direct-load
+ * kernel every other call; FP4Q_TMA=1 routes every call whose flattened
+ * length is a multiple of 64 (all strategies but brute force) to the TMA-fed
+ * kernel, FP4Q_TMA=0 none. Both kernels compute the same bits.
  */
 int fp4q_device_errors(void);
 

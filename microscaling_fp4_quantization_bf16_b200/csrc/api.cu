@@ -91,15 +91,20 @@ EncodeTiledFn encode_tiled()
     return fn;
 }
 
-// FP4Q_TMA=1 routes eligible quantize calls (flattened length a multiple of
-// 64, not brute force) to the TMA-fed kernel; both kernels compute the same
-// bits. The direct-load kernel is the default: on B200 it measured faster at
-// every size for unrotated inputs and at all but the largest sizes with a
-// 32-wide rotation.
-bool tma_requested()
+// Which loader feeds an eligible quantize call (flattened length a multiple of
+// 64, not a search; both kernels compute the same bits). By default the
+// TMA-fed kernel takes MXFP4 behind a 64- or 128-wide rotation -- measured on
+// B200: 66 against 78 us on a 16384 x 8192 tensor (its 4-stage copy ring hides
+// the load latency that, with the cross-lane butterfly stages, bounds the
+// direct kernel) -- and the direct-load kernel everything else (faster there,
+// e.g. 4-over-6 behind a 16-wide rotation 107 against 111 us). FP4Q_TMA=1
+// routes every eligible call to the TMA-fed kernel, FP4Q_TMA=0 none.
+bool use_tma(int strat, int rot)
 {
     const char* v = std::getenv("FP4Q_TMA");
-    return v != nullptr && std::strcmp(v, "0") != 0;
+    if (v != nullptr && v[0] != '\0')
+        return std::strcmp(v, "0") != 0;
+    return strat == K_MX && (rot == 64 || rot == 128);
 }
 
 // View of x as [n / 64, 64] bf16 rows of 128 bytes, box 64 x 64, 128-byte swizzle.
@@ -122,7 +127,7 @@ cudaError_t launch_quant(int block, int strat, int rot, const QuantArgs& a, cuda
 {
     const bool tma_shape = a.n % 64 == 0 && a.n / 64 < ((int64_t)1 << 31);
     const bool tma_strat = strat != K_BRUTE_FORCE && strat != K_MX_BRUTE && !is_ue_strat(strat);
-    if (tma_strat && tma_shape && tma_requested()) {
+    if (tma_strat && tma_shape && use_tma(strat, rot)) {
         CUtensorMap map;
         if (make_row_map(&map, a.x, a.n)) {
             int dev = 0, sms = 0;

@@ -25,7 +25,13 @@ constexpr int TMA_ROW_ELEMS = 64;                        // one 128-byte row
 constexpr int TILE_ROWS = TMA_TILE_ROWS;                 // 8 KB per stage
 constexpr int TILE_BYTES = TILE_ROWS * TMA_ROW_ELEMS * 2;
 constexpr int TILE_SEGS = TILE_ROWS * TMA_ROW_ELEMS / SEG;  // 128 segments
-constexpr int STAGES = 4;
+#ifndef FP4Q_TMA_STAGES
+#define FP4Q_TMA_STAGES 4
+#endif
+#ifndef FP4Q_TMA_MINB
+#define FP4Q_TMA_MINB 1
+#endif
+constexpr int STAGES = FP4Q_TMA_STAGES;
 constexpr int CONSUMER_WARPS = TILE_SEGS / 32;           // one segment per thread
 constexpr int TTHREADS = (CONSUMER_WARPS + 1) * 32;      // + one producer warp
 constexpr uint32_t WAIT_LIMIT = 1u << 24;                // polls before giving up
@@ -81,7 +87,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
 }
 
 template <int B, int ROT, int STRAT>
-__global__ void __launch_bounds__(TTHREADS)
+__global__ void __launch_bounds__(TTHREADS, FP4Q_TMA_MINB)
     quant_tma_kernel(const __grid_constant__ CUtensorMap tmap, QuantArgs a, int64_t ntiles,
                      unsigned* err)
 {
@@ -176,8 +182,11 @@ cudaError_t launch_tma_one(const CUtensorMap& map, const QuantArgs& a, int64_t n
 {
     auto kern = quant_tma_kernel<B, ROT, STRAT>;
     int per_sm = 0;
-    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TTHREADS,
-                                                                  TMA_SMEM_BYTES);
+    cudaError_t e = cudaSuccess;
+    if (TMA_SMEM_BYTES > 48 * 1024)
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TMA_SMEM_BYTES);
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, TTHREADS, TMA_SMEM_BYTES);
     if (e != cudaSuccess)
         return e;
     per_sm = per_sm < 1 ? 1 : per_sm;

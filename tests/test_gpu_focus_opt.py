@@ -245,8 +245,9 @@ def test_empty_inputs(gpu):
     torch.cuda.synchronize()
     assert gs.item() == 1.0
     u = torch.eye(128, device="cuda")
-    assert L.fp4q_gptq(w.data_ptr(), 0, 128, 1, 32, c.data_ptr(), None, u.data_ptr(), None,
-                       c.data_ptr(), c.data_ptr(), None) == 0
+    for rot in (0, 128):
+        assert L.fp4q_gptq(w.data_ptr(), 0, 128, 1, 32, rot, c.data_ptr(), None, u.data_ptr(), None,
+                           c.data_ptr(), c.data_ptr(), None) == 0
     q = gpu.quantize(w, "ue5m3", 16, "four_over_six")
     torch.cuda.synchronize()
     assert q.codes.numel() == 0 and q.global_scale is None

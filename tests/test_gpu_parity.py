@@ -137,10 +137,9 @@ def shapes_for(block, rot):
 @pytest.mark.parametrize("loads", ["direct", "tma"])
 @pytest.mark.parametrize("fmt,block,strat,rot", COMBOS)
 def test_quantize_small_shapes(gpu, monkeypatch, loads, fmt, block, strat, rot):
-    """Every combination through the direct-load kernel and (FP4Q_TMA=1,
-    flattened length a multiple of 64) the TMA-fed kernel."""
-    if loads == "tma":
-        monkeypatch.setenv("FP4Q_TMA", "1")
+    """Every combination through the direct-load kernel (FP4Q_TMA=0) and
+    (FP4Q_TMA=1, flattened length a multiple of 64) the TMA-fed kernel."""
+    monkeypatch.setenv("FP4Q_TMA", "1" if loads == "tma" else "0")
     for k, (rows, cols) in enumerate(shapes_for(block, rot)):
         x = mixed(rows, cols, seed=1000 * block + rot + k)
         dq = (None, torch.float32, torch.bfloat16)[k % 3]
@@ -393,8 +392,7 @@ def test_focus_small(gpu, fmt, block, sub):
 def test_multi_tile_tma_tails(gpu, monkeypatch, loads):
     """Row counts around the 4096-element TMA tile and the persistent grid,
     including a last tile that is mostly past the end of the tensor."""
-    if loads == "tma":
-        monkeypatch.setenv("FP4Q_TMA", "1")
+    monkeypatch.setenv("FP4Q_TMA", "1" if loads == "tma" else "0")
     for rows, cols in ((65, 64), (64 * 3 + 1, 128), (4096 * 2 + 64, 64), (1, 4096 * 4)):
         x = mixed(rows, cols, seed=rows)
         for fmt, block, strat, rot in (("nvfp4", 16, "four_over_six", 16), ("mxfp4", 32, "absmax", 64),
