@@ -168,56 +168,75 @@ __device__ __forceinline__ void scales_of(const uint32_t (&sc)[NB], float sg, fl
 
 // ------------------------------------------------------------ dequantize
 
-// One thread per EPT consecutive elements (EPT = 8 for bf16 output, 4 for
-// fp32): its 16 output bytes are one store, and a warp's stores cover 512
-// contiguous bytes. A thread's elements lie in one block unless B = 4 < EPT.
+// Each thread dequantizes DQ_ITEMS groups of EPT consecutive elements (EPT
+// = 8 for bf16 output, 4 for fp32): group k of thread (warp w, lane l) starts
+// at element ((w * DQ_ITEMS + k) * 32 + l) * EPT, so each load and each
+// 16-byte store instruction of a warp covers contiguous memory, and all the
+// groups' loads are issued before the first store. A group's elements lie in
+// one block unless B = 4 < EPT.
+constexpr int DQ_ITEMS = 4;
+
 template <int B, int FMT, int EPT>
 __global__ void __launch_bounds__(ATHREADS) dequant_kernel(DequantArgs a)
 {
     pdl_begin();
-    constexpr int NS = EPT > B ? EPT / B : 1;  // scale bytes per thread
+    constexpr int NS = EPT > B ? EPT / B : 1;  // scale bytes per group
     const int64_t t = (int64_t)blockIdx.x * ATHREADS + threadIdx.x;
-    const int64_t e0 = t * EPT;
-    if (e0 >= a.n)
-        return;
-    const int nvalid = (int)min((int64_t)EPT, a.n - e0);  // a multiple of 4
-    uint32_t q;
-    if (EPT == 8 && nvalid == 8)
-        q = *reinterpret_cast<const uint32_t*>(a.codes + e0 / 2);
-    else
-        q = *reinterpret_cast<const uint16_t*>(a.codes + e0 / 2);
-    uint32_t sc[NS];
+    const int64_t base = (t >> 5) * (32 * DQ_ITEMS) + (t & 31);  // group index of k = 0
+    uint32_t q[DQ_ITEMS], sc[DQ_ITEMS][NS];
 #pragma unroll
-    for (int k = 0; k < NS; ++k)
-        sc[k] = (k * B < nvalid) ? (uint32_t)a.scales[e0 / B + k] : 0u;
-    const float sg = FMT == 0 ? *a.sg : 1.0f;
-    float S[NS];
-    scales_of<NS, FMT>(sc, sg, S);
-    float v[EPT];
-    if constexpr (EPT == 8)
-        e2m1_unpack8(q, v);
-    else
-        e2m1_unpack4(q, v);
-    float yh[EPT];
+    for (int k = 0; k < DQ_ITEMS; ++k) {
+        const int64_t e0 = (base + 32 * k) * EPT;
+        q[k] = 0u;
 #pragma unroll
-    for (int j = 0; j < EPT / 2; ++j) {
-        const f32x2 Y = mul2(pk2(v[2 * j], v[2 * j + 1]), pk2(S[(2 * j) / B], S[(2 * j + 1) / B]));
-        upk2(Y, yh[2 * j], yh[2 * j + 1]);
-    }
-    if constexpr (EPT == 8) {  // bf16
-        uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + e0;
-        uint4 w;
-        w.x = pack_bf16x2(yh[0], yh[1]);
-        w.y = pack_bf16x2(yh[2], yh[3]);
-        w.z = pack_bf16x2(yh[4], yh[5]);
-        w.w = pack_bf16x2(yh[6], yh[7]);
-        if (nvalid == 8)
-            *reinterpret_cast<uint4*>(o) = w;
+        for (int m = 0; m < NS; ++m)
+            sc[k][m] = 0u;
+        if (e0 >= a.n)
+            continue;
+        const int nvalid = (int)min((int64_t)EPT, a.n - e0);  // a multiple of 4
+        if (EPT == 8 && nvalid == 8)
+            q[k] = *reinterpret_cast<const uint32_t*>(a.codes + e0 / 2);
         else
-            *reinterpret_cast<uint2*>(o) = make_uint2(w.x, w.y);
-    } else {  // fp32
-        *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + e0) =
-            make_float4(yh[0], yh[1], yh[2], yh[3]);
+            q[k] = *reinterpret_cast<const uint16_t*>(a.codes + e0 / 2);
+#pragma unroll
+        for (int m = 0; m < NS; ++m)
+            sc[k][m] = (m * B < nvalid) ? (uint32_t)a.scales[e0 / B + m] : 0u;
+    }
+    const float sg = FMT == 0 ? *a.sg : 1.0f;
+#pragma unroll
+    for (int k = 0; k < DQ_ITEMS; ++k) {
+        const int64_t e0 = (base + 32 * k) * EPT;
+        if (e0 >= a.n)
+            break;  // later groups start further on
+        const int nvalid = (int)min((int64_t)EPT, a.n - e0);
+        float S[NS];
+        scales_of<NS, FMT>(sc[k], sg, S);
+        float v[EPT];
+        if constexpr (EPT == 8)
+            e2m1_unpack8(q[k], v);
+        else
+            e2m1_unpack4(q[k], v);
+        float yh[EPT];
+#pragma unroll
+        for (int j = 0; j < EPT / 2; ++j) {
+            const f32x2 Y = mul2(pk2(v[2 * j], v[2 * j + 1]), pk2(S[(2 * j) / B], S[(2 * j + 1) / B]));
+            upk2(Y, yh[2 * j], yh[2 * j + 1]);
+        }
+        if constexpr (EPT == 8) {  // bf16
+            uint16_t* o = reinterpret_cast<uint16_t*>(a.out) + e0;
+            uint4 w;
+            w.x = pack_bf16x2(yh[0], yh[1]);
+            w.y = pack_bf16x2(yh[2], yh[3]);
+            w.z = pack_bf16x2(yh[4], yh[5]);
+            w.w = pack_bf16x2(yh[6], yh[7]);
+            if (nvalid == 8)
+                *reinterpret_cast<uint4*>(o) = w;
+            else
+                *reinterpret_cast<uint2*>(o) = make_uint2(w.x, w.y);
+        } else {  // fp32
+            *reinterpret_cast<float4*>(reinterpret_cast<float*>(a.out) + e0) =
+                make_float4(yh[0], yh[1], yh[2], yh[3]);
+        }
     }
 }
 
@@ -225,7 +244,8 @@ template <int B, int FMT>
 static cudaError_t launch_dequant_b(const DequantArgs& a, cudaStream_t st)
 {
     const int ept = a.out_kind == 2 ? 8 : 4;
-    const int64_t nthr = (a.n + ept - 1) / ept;
+    const int64_t groups = (a.n + ept - 1) / ept;
+    const int64_t nthr = (groups + 32 * DQ_ITEMS - 1) / (32 * DQ_ITEMS) * 32;  // whole warps
     if (!grid_ok(nthr))
         return cudaErrorInvalidValue;
     const unsigned g = grid_for(nthr);
