@@ -278,6 +278,53 @@ cudaError_t launch_dequant(int fmt, int block, const DequantArgs& a, cudaStream_
     }
 }
 
+// Per-warp staging for store_seg_values_warp: 32 lanes' outputs as rows of
+// 16-byte chunks (4 for bf16, 8 for fp32) plus one chunk of padding, so that
+// neither the row writes nor the transposed reads meet more than two-way bank
+// conflicts.
+constexpr int kStageChunks = 32 * 9;
+
+// Stores the SEG values of every lane's segment s (fp32 for kind 1, bf16 for
+// kind 2; all 32 lanes of the warp call it). A warp of 32 whole segments goes
+// through st (the warp's staging area), so that each 16-byte store
+// instruction covers 512 contiguous bytes; otherwise each active lane stores
+// its own segment.
+__device__ __forceinline__ void store_seg_values_warp(void* out, int kind, int64_t s, bool active, int nvalid,
+                                                      const float (&v)[SEG], uint4* st)
+{
+    const int lane = threadIdx.x & 31;
+    if (!__all_sync(0xFFFFFFFFu, active && nvalid == SEG)) {
+        if (active)
+            store_seg_values(out, kind, s, nvalid, v);
+        return;
+    }
+    if (kind == 2) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+            st[lane * 5 + k] = make_uint4(pack_bf16x2(v[8 * k], v[8 * k + 1]), pack_bf16x2(v[8 * k + 2], v[8 * k + 3]),
+                                          pack_bf16x2(v[8 * k + 4], v[8 * k + 5]), pack_bf16x2(v[8 * k + 6], v[8 * k + 7]));
+        __syncwarp();
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(out) + (s - lane) * SEG);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int c = 32 * k + lane;
+            o[c] = st[(c >> 2) * 5 + (c & 3)];
+        }
+    } else {
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+            st[lane * 9 + k] = make_uint4(__float_as_uint(v[4 * k]), __float_as_uint(v[4 * k + 1]),
+                                          __float_as_uint(v[4 * k + 2]), __float_as_uint(v[4 * k + 3]));
+        __syncwarp();
+        uint4* o = reinterpret_cast<uint4*>(reinterpret_cast<float*>(out) + (s - lane) * SEG);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int c = 32 * k + lane;
+            o[c] = st[(c >> 3) * 9 + (c & 7)];
+        }
+    }
+}
+
 // Dequantize and undo the blockwise rotation: one segment per thread, the
 // segment's values decoded, then rotated again by the normalised transform
 // (its own inverse; 64/128-wide chunks span neighbouring lanes, so whole warps
@@ -288,6 +335,7 @@ cudaError_t launch_dequant(int fmt, int block, const DequantArgs& a, cudaStream_
 template <int B, int FMT, int ROT>
 __global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
 {
+    __shared__ uint4 stage[ATHREADS / 32][kStageChunks];
     pdl_begin();
     constexpr int NB = SEG / B;
     const int lane = threadIdx.x & 31;
@@ -313,8 +361,7 @@ __global__ void __launch_bounds__(ATHREADS) dequant_rot_kernel(DequantArgs a)
     for (int i = 0; i < SEG; ++i)
         yh[i] = __uint_as_float(__float_as_uint(yh[i]) & a.keep);
     rotate_seg<ROT>(yh, lane);
-    if (active)
-        store_seg_values(a.out, a.out_kind, s, nvalid, yh);
+    store_seg_values_warp(a.out, a.out_kind, s, active, nvalid, yh, stage[threadIdx.x >> 5]);
 }
 
 template <int B, int FMT>
@@ -498,20 +545,23 @@ __device__ __forceinline__ void load_coeffs(const uint16_t* c, int64_t s, int nv
 template <int B, int SUB, bool MX>
 __global__ void __launch_bounds__(STHREADS) focus_fwd_kernel(FocusFwdArgs a)
 {
+    __shared__ uint4 stage[STHREADS / 32][kStageChunks];
     pdl_begin();
     constexpr int NB = SEG / B;
     constexpr int NK = SEG / SUB;
     const int64_t nseg = (a.n + SEG - 1) / SEG;
     const int64_t s = (int64_t)blockIdx.x * STHREADS + threadIdx.x;
+    const int lane = threadIdx.x & 31;
     float sg = 1.0f;
     if constexpr (!MX) {
         sg = global_scale_of(*a.amax);
         if (a.sg_out != nullptr && s == 0)
             *a.sg_out = sg;
     }
-    if (s >= nseg)
+    if (s - lane >= nseg)  // warp-uniform: the warp's stores are staged together
         return;
-    const int nvalid = (int)min((int64_t)SEG, a.n - s * SEG);
+    const bool active = s < nseg;  // an inactive lane loads nothing (zeros) and stores nothing
+    const int nvalid = active ? (int)min((int64_t)SEG, a.n - s * SEG) : 0;
     float y[SEG], ck[NK];
     load_seg_bf16(a.w, a.n, s, y);
     load_coeffs<NK>(a.c, s, nvalid, SUB, ck);
@@ -535,8 +585,8 @@ __global__ void __launch_bounds__(STHREADS) focus_fwd_kernel(FocusFwdArgs a)
     encode_seg<SUB, true>(y, r, zk, a.keep, q);  // packed: measured faster here
     float yh[SEG];
     decode_seg<B>(q, S, yh);
-    store_seg_values(a.w_hat, a.out_kind, s, nvalid, yh);
-    if (a.codes != nullptr) {
+    store_seg_values_warp(a.w_hat, a.out_kind, s, active, nvalid, yh, stage[threadIdx.x >> 5]);
+    if (a.codes != nullptr && active) {
         if (nvalid == SEG) {
             *reinterpret_cast<uint4*>(a.codes + s * (SEG / 2)) = make_uint4(q[0], q[1], q[2], q[3]);
             store_bytes<NB>(a.scales + s * NB, sc);
