@@ -37,7 +37,9 @@ CASES = [("nvfp4", 16, "absmax"), ("nvfp4", 4, "prevent_zero"), ("mxfp4", 32, "b
 @pytest.mark.parametrize("fmt,block,strat", CASES)
 @pytest.mark.parametrize("act_order", [True, False])
 def test_gptq_small_layers(gpu, fmt, block, strat, act_order):
-    for rows, K, seed in ((37, 256, 1), (9, 384, 2), (70, 128, 3)):
+    # (45, 1152): nine batches, the trailing updates beside the next batch
+    # kernel, a partial CTA of rows
+    for rows, K, seed in ((37, 256, 1), (9, 384, 2), (70, 128, 3), (45, 1152, 4)):
         d = synth.gptq_problem(rows, K, 1024, seed=seed, act_order=act_order)
         wb = u16(d["w"])
         q = oracle.quantize(wb, fmt, block, strat, 0, want_mse=False)
