@@ -51,6 +51,7 @@ enum KStrat { K_ABSMAX = 0, K_PREVENT_ZERO = 1, K_FOUR_OVER_SIX = 2, K_BRUTE_FOR
               K_UE_ABSMAX = 6, K_UE_PREVENT_ZERO = 7, K_UE_FOUR_OVER_SIX = 8, K_UE_BRUTE_FORCE = 9 };
 
 __host__ __device__ constexpr bool is_ue_strat(int s) { return s >= K_UE_ABSMAX && s <= K_UE_BRUTE_FORCE; }
+__host__ __device__ constexpr bool is_mx_strat(int s) { return s == K_MX || s == K_MX_BRUTE; }
 
 struct QuantArgs {
     const uint16_t* x;      // bf16 [n]

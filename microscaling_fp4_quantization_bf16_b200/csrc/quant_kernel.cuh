@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(QTHREADS, QMinBlocks<STRAT>::value) quant_kern
         return;
 
     float y[SEG];
-    unpack_seg(raw, y);
+    unpack_seg<!is_mx_strat(STRAT)>(raw, y);
     // all 32 lanes take part; past the end holds zeros
     rotate_seg<ROT, !foldable<ROT, STRAT>()>(y, lane);
     if (s < nseg)
@@ -571,7 +571,7 @@ __global__ void __launch_bounds__(QTHREADS, PMinBlocks<STRAT>::value)
     build_scale_tables<STRAT>(tab, a);
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, s += step) {
         float y[SEG];
-        unpack_seg(raw, y);
+        unpack_seg<!is_mx_strat(STRAT)>(raw, y);
         if (t + gridDim.x < ntiles)
             fetch(s + step, raw);  // next tile's loads overlap this tile's arithmetic
         if (s - lane < nseg) {     // warp-uniform
