@@ -8,9 +8,11 @@
 // upper Cholesky factor of the inverse Hessian in that order. Work proceeds
 // in batches of 128 positions ("lazy batch updates"):
 //
-//   gptq_gather_kernel   work[i][j] = W[i][perm[j]] widened to fp32 (with a
-//                        rotation: gptq_rotate_gather_kernel, the row rotated
-//                        blockwise first, as the quantizer rotates it)
+//   gptq_rotate_gather_kernel  work[i][j] = W[i][perm[j]] widened to fp32, the
+//                        row staged in shared memory (rotated blockwise first
+//                        when MR-GPTQ's rotation is asked for, as the
+//                        quantizer rotates it); gptq_gather_kernel for rows
+//                        too long to stage
 //   gptq_batch_kernel    first applies the previous batch's update to its
 //                        own 128 columns (the trailing arithmetic below),
 //                        then eight rows per warp (four lanes each) run the
@@ -86,7 +88,9 @@ __global__ void __launch_bounds__(256) gptq_gather_kernel(GptqArgs a)
 // butterfly stages in ascending order, the factor k_ROT; 64/128-wide chunks
 // span neighbouring lanes, so whole warps take part) into a shared copy of
 // the row in original column order, which is then gathered into processing
-// order: work[i][j] = rotated(W)[i][perm[j]].
+// order: work[i][j] = rotated(W)[i][perm[j]]. With ROT = 0 it is the plain
+// gather with the row staged in shared memory, so that the permuted reads
+// hit shared memory and the row is read from HBM with 128-bit loads.
 template <int ROT>
 __global__ void __launch_bounds__(1024) gptq_rotate_gather_kernel(GptqArgs a)
 {
@@ -558,10 +562,11 @@ cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
     if (e != cudaSuccess)
         return e;
     const int64_t n = a.rows * a.K;
-    if (a.rot == 0) {
+    const size_t row_smem = sizeof(float) * (size_t)a.K;
+    if (a.rot == 0 && (int64_t)row_smem > kGptqRowBytes) {
+        // a row too long to stage: each element read through the permutation
         e = launch_pdl(gptq_gather_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, st, a);
     } else {
-        const size_t row_smem = sizeof(float) * (size_t)a.K;
         const int64_t nseg_warps = (a.K / SEG + 31) / 32 * 32;
         const unsigned threads = (unsigned)(nseg_warps < 1024 ? nseg_warps : 1024);
         if ((int64_t)row_smem > kGptqRowBytes)
@@ -574,6 +579,7 @@ cudaError_t launch_gptq(const GptqArgs& a, cudaStream_t st)
             return launch_pdl(kern, dim3((unsigned)a.rows), dim3(threads), row_smem, st, a);
         };
         switch (a.rot) {
+        case 0: e = launch_rot(gptq_rotate_gather_kernel<0>); break;
         case 16: e = launch_rot(gptq_rotate_gather_kernel<16>); break;
         case 32: e = launch_rot(gptq_rotate_gather_kernel<32>); break;
         case 64: e = launch_rot(gptq_rotate_gather_kernel<64>); break;
