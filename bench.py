@@ -782,11 +782,11 @@ SUITE = ["quant MXFP4 B32 rot0", "quant MXFP4 B32 rot32", "quant MXFP4 B32 rot12
          "FOCUS calibration step NVFP4 B16 sub8 Adam", "FOCUS update from gradient sub8 Adam"]
 
 
-def run_suite(rounds: int = 2):
-    """Launches each library kernel once per round, in SUITE order, on an
+def run_suite(passes: int = 2):
+    """Launches each library kernel once per pass, in SUITE order, on an
     8192 x 8192 bf16 Student-t tensor (134 MB, larger than L2): the small,
     fixed launch list that the per-kernel ncu captures profile (skip the first
-    round, capture the second)."""
+    pass, capture the second)."""
     import torch
 
     import microscaling_fp4_quantization_bf16_b200 as fp4q
@@ -808,7 +808,7 @@ def run_suite(rounds: int = 2):
     gsw = torch.empty(1, device=dev)
     torch.cuda.synchronize()
     outs = {}
-    for _ in range(rounds):
+    for _ in range(passes):
         outs[0] = fp4q.quantize(x, "mxfp4", 32, "absmax", 0)
         outs[1] = fp4q.quantize(x, "mxfp4", 32, "absmax", 32)
         outs[2] = fp4q.quantize(x, "mxfp4", 32, "absmax", 128)
@@ -829,7 +829,7 @@ def run_suite(rounds: int = 2):
                                    lr=1e-4)
         outs[16] = fp4q.focus_update(w, g, st_upd, 8, lr=1e-4)
         torch.cuda.synchronize()
-    print(json.dumps({"suite": SUITE, "rounds": rounds, "shape": [R, C],
+    print(json.dumps({"suite": SUITE, "passes": passes, "shape": [R, C],
                       "device_errors": fp4q._abi.load().fp4q_device_errors()}))
 
 
