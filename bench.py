@@ -591,11 +591,12 @@ def breakdown(dev, peaks, reps: int = 10):
     gsecs = timeit([lambda: fp4q.gptq(gw, gqs.scales, gqs.global_scale, gU, gperm, "nvfp4", 16,
                                       work=gwork, out=gout)])
     gflops = 2.0 * 4096 * 128 * sum(4096 - b0 - 128 for b0 in range(0, 4096, 128))
+    # launches per call: the gather, 32 batch kernels, 30 trailing updates
     fma_peak = 148 * 128 * 2 * 1.965e9 / 1e12
     rows_out.append({"run": "gptq error feedback nvfp4 B16 4096x4096 (static MSE-optimal scales, act order)",
                      "us": round(gsecs * 1e6, 1), "tflops": round(gflops / gsecs / 1e12, 2),
                      "bound": "fp32 fma", "fma_frac": round(gflops / gsecs / 1e12 / fma_peak, 4),
-                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 2 * 32 - 1})
+                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 32 + 30})
     # MR-GPTQ: the 128-wide blockwise rotation in front (MXFP4 B32 with the
     # MSE-optimised E8M0 grid as static scales of the rotated weights; U from
     # the rotated-basis Hessian), the same layer size
@@ -609,7 +610,7 @@ def breakdown(dev, peaks, reps: int = 10):
                             "(static MSE-grid scales, act order)",
                      "us": round(gsecs * 1e6, 1), "tflops": round(gflops / gsecs / 1e12, 2),
                      "bound": "fp32 fma", "fma_frac": round(gflops / gsecs / 1e12 / fma_peak, 4),
-                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 2 * 32 - 1})
+                     "peak_tflops": round(fma_peak, 1), "launches": 1 + 32 + 30})
     del gd, gw, gqs, gU, gperm, gwork, gout
     torch.cuda.empty_cache()
     # FOCUS

@@ -385,7 +385,9 @@ fp4q_status fp4q_focus_step(const void* w, int64_t rows, int64_t cols, fp4q_form
  *           fp4q_device_errors and read column 0); NULL = natural order.
  * work      fp32 [rows, cols] caller scratch (overwritten).
  * codes     uint8 [rows, cols/2] (zeroed, then written).
- * Launches: 1 memset + 1 + 2 * cols/128 - 1 kernels. Rows are independent.
+ * Launches: 1 memset + 2 * cols/128 - 1 kernels (2 when cols == 128): a
+ * gather, one kernel per batch, and the trailing updates, each of which runs
+ * beside the next batch's kernel in the same stream. Rows are independent.
  */
 fp4q_status fp4q_gptq(const void* w, int64_t rows, int64_t cols, fp4q_format fmt, int block,
                       int rot, const uint8_t* scales, const float* global_scale, const float* U,
